@@ -1,0 +1,170 @@
+/*
+ * mnb.h -- C ABI of libmnb.so: the MatMulNBits operator (weight-only 4-bit
+ * block-quantized matmul) on NVIDIA B200 (sm_100a).
+ *
+ * The operator, as the model cards that ship it describe it:
+ *   "Mega-ASR -- INT4 ONNX (GPTQ-calibrated)", intro and "Conversion details":
+ *     MatMulNBits, 4 bits, block_size=32, is_symmetric=False; the decoder is
+ *     ~95% MatMul ops ("Compression vs original").
+ *   "int4 STT weights for sherpa-onnx", "Why int4 rather than the usual int8":
+ *     weight-only, in blocks, activations untouched.
+ *   "qwen3-asr-0.6b-onnx-int4-merged", "Provenance": block_size=64.
+ *   "Qwen3-ASR-0.6B -- ONNX for the browser", "Pick a variant": q4 (fp32
+ *     float tensors) and q4f16 (fp16 float tensors).
+ *
+ * Definitions (standard asymmetric int4):
+ *   w[n][k] = (q[n][k] - zp[n][b]) * scale[n][b],  b = k / bs,
+ *   zp = 8 for every block when no zero-point tensor is given,
+ *   Y[m][n] = sum_k X[m][k] * w[n][k]              (Y = X . dequant(W)^T).
+ *
+ * Layout (row-major, contiguous, element 0 first):
+ *   packed  uint8 [N][K/2]: element 2j of a row in the LOW nibble of byte j,
+ *           element 2j+1 in the high nibble (equivalently [N][K/bs][bs/2]).
+ *   scales  fp32 or fp16 [N][K/bs].
+ *   zp      uint8 [N][ceil((K/bs)/2)]: block b in byte b/2, low nibble when b
+ *           is even; an odd count leaves the last high nibble 0.  NULL = no
+ *           zero points (zp = 8).
+ *   X       [M][K] and Y [M][N] in the activation dtype.
+ *
+ * Conventions shared by every entry point:
+ *   - Every pointer argument is a DEVICE pointer allocated and owned by the
+ *     caller, except the size outputs of mnb_packed_sizes (host pointers).
+ *     The library allocates no device memory and keeps no pointer after the
+ *     call returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream).  Work is enqueued asynchronously; nothing synchronizes.
+ *   - Arguments are validated on the host first; a failed check returns a
+ *     negative MNB_ERR_* code, launches nothing, and sets a thread-local
+ *     message readable with mnb_last_error().
+ *   - Pointers to packed weights, activations and outputs must be 16-byte
+ *     aligned (MNB_ERR_ALIGN otherwise); scales and zero points need only
+ *     their element alignment.
+ *   - Inputs must be finite.  Inputs and outputs must not overlap.
+ */
+#ifndef MNB_H
+#define MNB_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MNB_API __attribute__((visibility("default")))
+#else
+#define MNB_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { MNB_F32 = 0, MNB_F16 = 1 } mnb_dtype;
+
+enum {
+    MNB_OK = 0,
+    MNB_ERR_INVALID_ARG = -1, /* NULL pointer, negative size, unknown dtype     */
+    MNB_ERR_SHAPE = -2,       /* bs not 32/64, K % bs != 0, size too large      */
+    MNB_ERR_ALIGN = -3,       /* a pointer is not aligned as documented         */
+    MNB_ERR_UNSUPPORTED = -4, /* a valid request this build does not serve      */
+    MNB_ERR_CUDA = -5,        /* a CUDA runtime call or launch failed           */
+    MNB_ERR_TIMEOUT = -6      /* a device-side bounded wait gave up (see below) */
+};
+
+/* Flags for mnb_gemv / mnb_gemm. */
+enum {
+    /* Launch with programmatic dependent launch: the kernel may start while
+     * the previous kernel on `stream` is still running, and reads its WEIGHTS
+     * (packed, scales, zp) before waiting for that kernel to finish; it reads X
+     * and writes Y only after the wait.  Pass it only when no kernel still in
+     * flight on the stream writes this call's weights. */
+    MNB_FLAG_PDL = 1
+};
+
+/* Message describing the last failed call on this host thread ("" if none). */
+MNB_API const char *mnb_last_error(void);
+
+/* Library version string. */
+MNB_API const char *mnb_version(void);
+
+/* Bytes of the packed tensors of one [N, K] weight.  Host-only, no CUDA call.
+ * Pages: byte counts of "qwen3-asr-0.6b-onnx-int4-merged" ("Why": 962 MB ->
+ * 340 MB) follow from this layout with fp32 scales and packed 4-bit zp.
+ * Errors: MNB_ERR_INVALID_ARG (NULL output, N < 0, bad dtype),
+ *         MNB_ERR_SHAPE (bs not 32/64, K <= 0 or K % bs != 0). */
+MNB_API int mnb_packed_sizes(int64_t N, int64_t K, int bs, mnb_dtype scale_t, int has_zp,
+                     size_t *packed_bytes, size_t *scale_bytes, size_t *zp_bytes);
+
+/* Block-wise round-to-nearest quantization of fp32 W [N][K] into the packed
+ * layout ("Mega-ASR -- INT4 ONNX", "Conversion details": block_size=32,
+ * is_symmetric=False, bits=4; "Qwen3-ASR-0.6B -- ONNX for the browser": RTN).
+ *   has_zp = 1: lo = min(0, min v), hi = max(0, max v), scale = (hi - lo)/15,
+ *               zp = clamp(rint(-lo/scale), 0, 15),
+ *               q = clamp(rint(v/scale + zp), 0, 15)  (IEEE divide, then add;
+ *               rint rounds half to even); scale == 0 gives zp = q = 0.
+ *   has_zp = 0: zp = 8 implied, scale = max|v| / 7, q = clamp(rint(v/scale) + 8,
+ *               0, 15); scale == 0 gives q = 8.  zp may be NULL.
+ *   scale_t = MNB_F16 stores fp16_rn of the fp32 scale (q uses the fp32 one).
+ * Results are bit-identical to a scalar fp32 evaluation of these formulas.
+ * Writes packed, scales and (has_zp) zp completely.
+ * Errors: MNB_ERR_INVALID_ARG, MNB_ERR_SHAPE, MNB_ERR_ALIGN (W or packed not
+ *         16-byte aligned), MNB_ERR_CUDA. */
+MNB_API int mnb_quantize_rtn(const float *W, int64_t N, int64_t K, int bs, int has_zp,
+                     uint8_t *packed, void *scales, mnb_dtype scale_t, uint8_t *zp,
+                     void *stream);
+
+/* W_out[n][k] = (q - zp) * scale, rounded once to out_t (fp32 or fp16) from
+ * the exact product.  zp NULL = 8.
+ * Errors: MNB_ERR_INVALID_ARG, MNB_ERR_SHAPE, MNB_ERR_ALIGN, MNB_ERR_CUDA. */
+MNB_API int mnb_dequantize(const uint8_t *packed, const void *scales, mnb_dtype scale_t,
+                   const uint8_t *zp, int64_t N, int64_t K, int bs, void *W_out,
+                   mnb_dtype out_t, void *stream);
+
+/* Decode-shaped MatMulNBits, 1 <= M <= 16 (the autoregressive step of
+ * "Qwen3-ASR-0.6B -- ONNX for the browser", "Graph contracts": decoder_step,
+ * input_embeds [1, 1, 1024]).  Y = X . dequant(W)^T.
+ *   act_t  = dtype of X and Y (fp32 or fp16); scale_t = dtype of scales.
+ *   Accumulation is fp32.  Bandwidth-bound: streams the packed weights once.
+ * Errors: MNB_ERR_INVALID_ARG, MNB_ERR_SHAPE, MNB_ERR_ALIGN,
+ *         MNB_ERR_UNSUPPORTED (M > 16), MNB_ERR_CUDA. */
+MNB_API int mnb_gemv(const void *X, mnb_dtype act_t, const uint8_t *packed, const void *scales,
+             mnb_dtype scale_t, const uint8_t *zp, void *Y, int64_t M, int64_t N, int64_t K,
+             int bs, unsigned flags, void *stream);
+
+/* Prefill-shaped MatMulNBits on the tensor cores, any M >= 1 (tuned for
+ * M >= 64: the full-length prefill of "Mega-ASR -- INT4 ONNX", "What's in this
+ * repo": decoder_prefill).  Y = X . dequant(W)^T with fp16 X and Y; each
+ * weight is dequantized to fp16_rn((q - zp) * scale) and the products are
+ * accumulated in fp32.
+ *   act_t must be MNB_F16; N must be a multiple of 128 and K of 64.
+ * A device-side wait that exceeds its iteration limit makes the kernel stop,
+ * sets a bit in the library's device status word (see mnb_device_status) and
+ * leaves Y incomplete; the call itself returned MNB_OK by then.
+ * Errors: MNB_ERR_INVALID_ARG, MNB_ERR_SHAPE, MNB_ERR_ALIGN,
+ *         MNB_ERR_UNSUPPORTED (fp32 activations), MNB_ERR_CUDA. */
+MNB_API int mnb_gemm(const void *X, mnb_dtype act_t, const uint8_t *packed, const void *scales,
+             mnb_dtype scale_t, const uint8_t *zp, void *Y, int64_t M, int64_t N, int64_t K,
+             int bs, unsigned flags, void *stream);
+
+/* int8 embedding lookup ("Qwen3-ASR-0.6B -- ONNX for the browser",
+ * "Building the prompt" step 4 and "Pick a variant": embed_tokens.int8.bin +
+ * embed_scales.f32.bin):
+ *   out[t][d] = round_out_t( fp32(table[ids[t]][d]) * row_scales[ids[t]] ),
+ * the product taken in fp32 and rounded once more to fp16 when out_t is fp16.
+ *   table int8 [V][D], row_scales fp32 [V], ids int32 [T], out [T][D].
+ * An id outside [0, V) yields a zero row and, when status != NULL, sets bit 0
+ * of the device int *status (atomic OR; the caller clears it).  Never traps.
+ * Requires D % 16 == 0 and 16-byte aligned table and out.
+ * Errors: MNB_ERR_INVALID_ARG, MNB_ERR_SHAPE, MNB_ERR_ALIGN, MNB_ERR_CUDA. */
+MNB_API int mnb_embed_gather(const int8_t *table, const float *row_scales, int64_t V, int64_t D,
+                     const int32_t *ids, int64_t T, void *out, mnb_dtype out_t, int *status,
+                     void *stream);
+
+/* Reads (and, if clear != 0, zeroes) the library's device status word on the
+ * current device: bit 0 = a GEMM mbarrier wait timed out.  Synchronizes the
+ * device.  Errors: MNB_ERR_INVALID_ARG (NULL), MNB_ERR_CUDA. */
+MNB_API int mnb_device_status(unsigned *status_out, int clear);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MNB_H */

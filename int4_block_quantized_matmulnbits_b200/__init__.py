@@ -1,0 +1,156 @@
+"""MatMulNBits (weight-only int4, block-quantized) for NVIDIA B200 -- Python binding.
+
+A thin ctypes layer over ``libmnb.so`` (the sm_100a kernels and their C ABI,
+declared in ``include/mnb.h``).  Every function here has the name of the C
+entry point it calls and only marshals arguments: torch tensors become device
+pointers, dtypes become ``mnb_dtype`` values, the stream defaults to torch's
+current stream.  All arithmetic runs in the CUDA kernels; there is no CPU path.
+If the library cannot be loaded, importing this package raises.
+
+Layout (see ``include/mnb.h``): packed uint8 [N, K/2] (element 2j in the low
+nibble of byte j), scales fp32/fp16 [N, K/bs], zero points uint8
+[N, ceil(K/bs/2)] (block b in byte b/2, low nibble for even b) or None (zp=8).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "MnbError", "MNB_F32", "MNB_F16", "MNB_FLAG_PDL", "lib_path",
+    "mnb_last_error", "mnb_version", "mnb_packed_sizes", "mnb_quantize_rtn", "mnb_dequantize",
+    "mnb_gemv", "mnb_gemm", "mnb_embed_gather", "mnb_device_status",
+]
+
+MNB_F32, MNB_F16 = 0, 1
+MNB_FLAG_PDL = 1
+_ERRORS = {-1: "MNB_ERR_INVALID_ARG", -2: "MNB_ERR_SHAPE", -3: "MNB_ERR_ALIGN",
+           -4: "MNB_ERR_UNSUPPORTED", -5: "MNB_ERR_CUDA", -6: "MNB_ERR_TIMEOUT"}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_HERE, "libmnb.so")
+
+
+class MnbError(RuntimeError):
+    def __init__(self, fn, code, msg):
+        super().__init__(f"{fn} -> {_ERRORS.get(code, code)}: {msg}")
+        self.code = code
+
+
+def _load():
+    # (Re)build in-tree when libmnb.so is missing or older than its sources;
+    # a no-op otherwise.  Raises if nvcc fails: there is no fallback path.
+    from . import build as _build
+
+    _build.build()
+    lib = ctypes.CDLL(lib_path)
+    i64, i32, u32, vp, sz = ctypes.c_int64, ctypes.c_int, ctypes.c_uint, ctypes.c_void_p, ctypes.c_size_t
+    P = ctypes.POINTER
+    sig = {
+        "mnb_last_error": ([], ctypes.c_char_p),
+        "mnb_version": ([], ctypes.c_char_p),
+        "mnb_packed_sizes": ([i64, i64, i32, i32, i32, P(sz), P(sz), P(sz)], i32),
+        "mnb_quantize_rtn": ([vp, i64, i64, i32, i32, vp, vp, i32, vp, vp], i32),
+        "mnb_dequantize": ([vp, vp, i32, vp, i64, i64, i32, vp, i32, vp], i32),
+        "mnb_gemv": ([vp, i32, vp, vp, i32, vp, vp, i64, i64, i64, i32, u32, vp], i32),
+        "mnb_gemm": ([vp, i32, vp, vp, i32, vp, vp, i64, i64, i64, i32, u32, vp], i32),
+        "mnb_embed_gather": ([vp, vp, i64, i64, vp, i64, vp, i32, vp, vp], i32),
+        "mnb_device_status": ([P(u32), i32], i32),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes, f.restype = args, res
+    return lib
+
+
+_lib = _load()
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _dt(t):
+    if t.dtype == torch.float32:
+        return MNB_F32
+    if t.dtype == torch.float16:
+        return MNB_F16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(fn, rc):
+    if rc != 0:
+        raise MnbError(fn, rc, _lib.mnb_last_error().decode())
+
+
+def mnb_last_error() -> str:
+    return _lib.mnb_last_error().decode()
+
+
+def mnb_version() -> str:
+    return _lib.mnb_version().decode()
+
+
+def mnb_packed_sizes(N, K, bs, scale_dtype=torch.float16, has_zp=True):
+    """(packed_bytes, scale_bytes, zp_bytes) of one [N, K] weight."""
+    p, s, z = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    st = MNB_F16 if scale_dtype == torch.float16 else MNB_F32
+    _check("mnb_packed_sizes", _lib.mnb_packed_sizes(N, K, bs, st, int(bool(has_zp)),
+                                                     ctypes.byref(p), ctypes.byref(s), ctypes.byref(z)))
+    return p.value, s.value, z.value
+
+
+def mnb_quantize_rtn(W, N, K, bs, has_zp, packed, scales, zp, stream=None):
+    """Block-wise RTN of fp32 W [N, K] into packed / scales / zp (all device tensors)."""
+    _check("mnb_quantize_rtn", _lib.mnb_quantize_rtn(
+        _ptr(W), N, K, bs, int(bool(has_zp)), _ptr(packed), _ptr(scales), _dt(scales),
+        _ptr(zp), _stream(stream)))
+
+
+def mnb_dequantize(packed, scales, zp, N, K, bs, W_out, stream=None):
+    """W_out [N, K] (fp32 or fp16) = (q - zp) * scale, one rounding."""
+    _check("mnb_dequantize", _lib.mnb_dequantize(
+        _ptr(packed), _ptr(scales), _dt(scales), _ptr(zp), N, K, bs, _ptr(W_out), _dt(W_out),
+        _stream(stream)))
+
+
+def mnb_gemv(X, packed, scales, zp, Y, M, N, K, bs, flags=0, stream=None):
+    """Y [M, N] = X [M, K] . dequant(W)^T for 1 <= M <= 16 (decode kernel)."""
+    _check("mnb_gemv", _lib.mnb_gemv(
+        _ptr(X), _dt(X), _ptr(packed), _ptr(scales), _dt(scales), _ptr(zp), _ptr(Y),
+        M, N, K, bs, flags, _stream(stream)))
+
+
+def mnb_gemm(X, packed, scales, zp, Y, M, N, K, bs, flags=0, stream=None):
+    """Y [M, N] = X [M, K] . dequant(W)^T on the tensor cores (fp16 X and Y)."""
+    _check("mnb_gemm", _lib.mnb_gemm(
+        _ptr(X), _dt(X), _ptr(packed), _ptr(scales), _dt(scales), _ptr(zp), _ptr(Y),
+        M, N, K, bs, flags, _stream(stream)))
+
+
+def mnb_embed_gather(table, row_scales, V, D, ids, T, out, status=None, stream=None):
+    """out [T, D] = int8 table rows [ids] * row_scales[ids] (fp32 product, fp16 if out is fp16)."""
+    _check("mnb_embed_gather", _lib.mnb_embed_gather(
+        _ptr(table), _ptr(row_scales), V, D, _ptr(ids), T, _ptr(out), _dt(out), _ptr(status),
+        _stream(stream)))
+
+
+def mnb_device_status(clear=False) -> int:
+    """The library's device status word (bit 0: a GEMM wait timed out); synchronizes."""
+    v = ctypes.c_uint()
+    _check("mnb_device_status", _lib.mnb_device_status(ctypes.byref(v), int(bool(clear))))
+    return v.value

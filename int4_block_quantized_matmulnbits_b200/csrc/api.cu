@@ -1,0 +1,211 @@
+// api.cu -- the extern "C" entry points of libmnb: host-side argument checks,
+// then the launchers of the kernel files.  Nothing here touches the device
+// before every check has passed.
+#include <stdarg.h>
+#include <stdio.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace mnb {
+
+static thread_local char g_msg[512] = "";
+
+int fail(int code, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+void clear_error() { g_msg[0] = 0; }
+
+int check_launch(const char *what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return fail(MNB_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return MNB_OK;
+}
+
+// Limits: sizes fit comfortably in 32-bit element indices of one row and in
+// 64-bit byte offsets overall.
+static const int64_t kMaxDim = (int64_t)1 << 30;
+
+static int check_weight_shape(const char *fn, int64_t N, int64_t K, int bs) {
+    if (N < 0 || K < 0)
+        return fail(MNB_ERR_INVALID_ARG, "%s: negative size (N=%lld K=%lld)", fn, (long long)N,
+                    (long long)K);
+    if (bs != 32 && bs != 64)
+        return fail(MNB_ERR_SHAPE, "%s: block size %d not in {32, 64}", fn, bs);
+    if (K == 0 || K % bs != 0)
+        return fail(MNB_ERR_SHAPE, "%s: K=%lld is not a positive multiple of bs=%d", fn,
+                    (long long)K, bs);
+    if (N > kMaxDim || K > kMaxDim)
+        return fail(MNB_ERR_SHAPE, "%s: N or K above 2^30", fn);
+    return MNB_OK;
+}
+
+static int check_dtype(const char *fn, const char *what, int t) {
+    if (t != MNB_F32 && t != MNB_F16)
+        return fail(MNB_ERR_INVALID_ARG, "%s: unknown %s dtype %d", fn, what, t);
+    return MNB_OK;
+}
+
+static int check_matmul_args(const char *fn, const void *X, int act_t, const uint8_t *packed,
+                             const void *scales, int scale_t, void *Y, int64_t M, int64_t N,
+                             int64_t K, int bs) {
+    int rc;
+    if ((rc = check_dtype(fn, "activation", act_t)) || (rc = check_dtype(fn, "scale", scale_t)))
+        return rc;
+    if ((rc = check_weight_shape(fn, N, K, bs)))
+        return rc;
+    if (M < 0)
+        return fail(MNB_ERR_INVALID_ARG, "%s: negative M", fn);
+    if (M > kMaxDim)
+        return fail(MNB_ERR_SHAPE, "%s: M above 2^30", fn);
+    if (M > 0 && N > 0 && (!X || !packed || !scales || !Y))
+        return fail(MNB_ERR_INVALID_ARG, "%s: NULL X, packed, scales or Y", fn);
+    if (!aligned(X, 16) || !aligned(packed, 16) || !aligned(Y, 16))
+        return fail(MNB_ERR_ALIGN, "%s: X, packed and Y must be 16-byte aligned", fn);
+    if (!aligned(scales, scale_t == MNB_F32 ? 4 : 2))
+        return fail(MNB_ERR_ALIGN, "%s: scales misaligned", fn);
+    return MNB_OK;
+}
+
+}  // namespace mnb
+
+using namespace mnb;
+
+extern "C" {
+
+const char *mnb_last_error(void) { return g_msg; }
+
+const char *mnb_version(void) { return "mnb 0.1 (sm_100a)"; }
+
+int mnb_packed_sizes(int64_t N, int64_t K, int bs, mnb_dtype scale_t, int has_zp,
+                     size_t *packed_bytes, size_t *scale_bytes, size_t *zp_bytes) {
+    clear_error();
+    int rc;
+    if (!packed_bytes || !scale_bytes || !zp_bytes)
+        return fail(MNB_ERR_INVALID_ARG, "mnb_packed_sizes: NULL output pointer");
+    if ((rc = check_dtype("mnb_packed_sizes", "scale", scale_t)))
+        return rc;
+    if ((rc = check_weight_shape("mnb_packed_sizes", N, K, bs)))
+        return rc;
+    int64_t nb = K / bs;
+    *packed_bytes = (size_t)(N * (K / 2));
+    *scale_bytes = (size_t)(N * nb * (scale_t == MNB_F32 ? 4 : 2));
+    *zp_bytes = has_zp ? (size_t)(N * ((nb + 1) / 2)) : 0;
+    return MNB_OK;
+}
+
+int mnb_quantize_rtn(const float *W, int64_t N, int64_t K, int bs, int has_zp, uint8_t *packed,
+                     void *scales, mnb_dtype scale_t, uint8_t *zp, void *stream) {
+    clear_error();
+    const char *fn = "mnb_quantize_rtn";
+    int rc;
+    if ((rc = check_dtype(fn, "scale", scale_t)) || (rc = check_weight_shape(fn, N, K, bs)))
+        return rc;
+    if (N == 0)
+        return MNB_OK;
+    if (!W || !packed || !scales || (has_zp && !zp))
+        return fail(MNB_ERR_INVALID_ARG, "%s: NULL pointer", fn);
+    if (!aligned(W, 16) || !aligned(packed, 16))
+        return fail(MNB_ERR_ALIGN, "%s: W and packed must be 16-byte aligned", fn);
+    if (!aligned(scales, scale_t == MNB_F32 ? 4 : 2))
+        return fail(MNB_ERR_ALIGN, "%s: scales misaligned", fn);
+    return launch_quantize_rtn(W, N, K, bs, has_zp ? 1 : 0, packed, scales, scale_t == MNB_F16,
+                               has_zp ? zp : nullptr, (cudaStream_t)stream);
+}
+
+int mnb_dequantize(const uint8_t *packed, const void *scales, mnb_dtype scale_t, const uint8_t *zp,
+                   int64_t N, int64_t K, int bs, void *W_out, mnb_dtype out_t, void *stream) {
+    clear_error();
+    const char *fn = "mnb_dequantize";
+    int rc;
+    if ((rc = check_dtype(fn, "scale", scale_t)) || (rc = check_dtype(fn, "output", out_t)) ||
+        (rc = check_weight_shape(fn, N, K, bs)))
+        return rc;
+    if (N == 0)
+        return MNB_OK;
+    if (!packed || !scales || !W_out)
+        return fail(MNB_ERR_INVALID_ARG, "%s: NULL pointer", fn);
+    if (!aligned(packed, 16) || !aligned(W_out, 16))
+        return fail(MNB_ERR_ALIGN, "%s: packed and W_out must be 16-byte aligned", fn);
+    if (!aligned(scales, scale_t == MNB_F32 ? 4 : 2))
+        return fail(MNB_ERR_ALIGN, "%s: scales misaligned", fn);
+    return launch_dequantize(packed, scales, scale_t == MNB_F16, zp, N, K, bs, W_out,
+                             out_t == MNB_F16, (cudaStream_t)stream);
+}
+
+int mnb_gemv(const void *X, mnb_dtype act_t, const uint8_t *packed, const void *scales,
+             mnb_dtype scale_t, const uint8_t *zp, void *Y, int64_t M, int64_t N, int64_t K,
+             int bs, unsigned flags, void *stream) {
+    clear_error();
+    const char *fn = "mnb_gemv";
+    int rc = check_matmul_args(fn, X, act_t, packed, scales, scale_t, Y, M, N, K, bs);
+    if (rc)
+        return rc;
+    if (M > 16)
+        return fail(MNB_ERR_UNSUPPORTED, "%s: M=%lld > 16 (use mnb_gemm)", fn, (long long)M);
+    if (flags & ~(unsigned)MNB_FLAG_PDL)
+        return fail(MNB_ERR_INVALID_ARG, "%s: unknown flags 0x%x", fn, flags);
+    if (M == 0 || N == 0)
+        return MNB_OK;
+    return launch_gemv(X, act_t == MNB_F16, packed, scales, scale_t == MNB_F16, zp, Y, (int)M,
+                       (int)N, (int)K, bs, flags, (cudaStream_t)stream);
+}
+
+int mnb_gemm(const void *X, mnb_dtype act_t, const uint8_t *packed, const void *scales,
+             mnb_dtype scale_t, const uint8_t *zp, void *Y, int64_t M, int64_t N, int64_t K,
+             int bs, unsigned flags, void *stream) {
+    clear_error();
+    const char *fn = "mnb_gemm";
+    int rc = check_matmul_args(fn, X, act_t, packed, scales, scale_t, Y, M, N, K, bs);
+    if (rc)
+        return rc;
+    if (act_t != MNB_F16)
+        return fail(MNB_ERR_UNSUPPORTED, "%s: the tensor-core path takes fp16 activations", fn);
+    if (N % 128 != 0 || K % 64 != 0)
+        return fail(MNB_ERR_SHAPE, "%s: N=%lld must be a multiple of 128 and K=%lld of 64", fn,
+                    (long long)N, (long long)K);
+    if (flags & ~(unsigned)MNB_FLAG_PDL)
+        return fail(MNB_ERR_INVALID_ARG, "%s: unknown flags 0x%x", fn, flags);
+    if (M == 0 || N == 0)
+        return MNB_OK;
+    return launch_gemm(X, packed, scales, scale_t == MNB_F16, zp, Y, (int)M, (int)N, (int)K, bs,
+                       flags, (cudaStream_t)stream);
+}
+
+int mnb_embed_gather(const int8_t *table, const float *row_scales, int64_t V, int64_t D,
+                     const int32_t *ids, int64_t T, void *out, mnb_dtype out_t, int *status,
+                     void *stream) {
+    clear_error();
+    const char *fn = "mnb_embed_gather";
+    int rc;
+    if ((rc = check_dtype(fn, "output", out_t)))
+        return rc;
+    if (V < 0 || D < 0 || T < 0)
+        return fail(MNB_ERR_INVALID_ARG, "%s: negative size", fn);
+    if (D % 16 != 0 || D > kMaxDim || V > ((int64_t)1 << 31) - 1 || T > kMaxDim)
+        return fail(MNB_ERR_SHAPE, "%s: D must be a multiple of 16; V < 2^31", fn);
+    if (T == 0 || D == 0)
+        return MNB_OK;
+    if (!ids || !out || (V > 0 && (!table || !row_scales)))
+        return fail(MNB_ERR_INVALID_ARG, "%s: NULL pointer", fn);
+    if (!aligned(table, 16) || !aligned(out, 16) || !aligned(row_scales, 4) || !aligned(ids, 4) ||
+        !aligned(status, 4))
+        return fail(MNB_ERR_ALIGN, "%s: table and out must be 16-byte aligned", fn);
+    return launch_embed_gather(table, row_scales, V, D, ids, T, out, out_t == MNB_F16, status,
+                               (cudaStream_t)stream);
+}
+
+int mnb_device_status(unsigned *status_out, int clear) {
+    clear_error();
+    if (!status_out)
+        return fail(MNB_ERR_INVALID_ARG, "mnb_device_status: NULL output");
+    return read_device_status(status_out, clear);
+}
+
+}  // extern "C"

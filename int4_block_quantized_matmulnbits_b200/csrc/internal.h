@@ -1,0 +1,30 @@
+// internal.h -- launchers implemented in the kernel files, called by api.cu
+// after the host-side argument checks.  Each returns an MNB_* status.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mnb {
+
+int launch_quantize_rtn(const float *W, int64_t N, int64_t K, int bs, int has_zp, uint8_t *packed,
+                        void *scales, int scale_f16, uint8_t *zp, cudaStream_t s);
+
+int launch_dequantize(const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,
+                      int64_t N, int64_t K, int bs, void *out, int out_f16, cudaStream_t s);
+
+int launch_gemv(const void *X, int act_f16, const uint8_t *packed, const void *scales,
+                int scale_f16, const uint8_t *zp, void *Y, int M, int N, int K, int bs,
+                unsigned flags, cudaStream_t s);
+
+int launch_gemm(const void *X, const uint8_t *packed, const void *scales, int scale_f16,
+                const uint8_t *zp, void *Y, int M, int N, int K, int bs, unsigned flags,
+                cudaStream_t s);
+
+int launch_embed_gather(const int8_t *table, const float *row_scales, int64_t V, int64_t D,
+                        const int32_t *ids, int64_t T, void *out, int out_f16, int *status,
+                        cudaStream_t s);
+
+int read_device_status(unsigned *out, int clear);
+
+}  // namespace mnb

@@ -1,0 +1,106 @@
+"""Quantized linears and the decoder-shaped passes that chain them.
+
+The decoders of "Mega-ASR -- INT4 ONNX (GPTQ-calibrated)" and "Qwen3-ASR-0.6B
+-- ONNX for the browser" spend ~95% of their work in MatMulNBits
+("Compression vs original"): per token, 28 layers x 7 projections plus the
+lm_head (decoder_step), and the same projections over all prompt tokens in
+decoder_init / decoder_prefill.  These classes hold the packed weights in HBM
+and issue the library calls of one such pass; every call is one CUDA kernel
+of libmnb, optionally captured into a CUDA graph.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import (MNB_FLAG_PDL, mnb_dequantize, mnb_embed_gather, mnb_gemm, mnb_gemv,
+               mnb_packed_sizes, mnb_quantize_rtn)
+
+
+class QLinear:
+    """One MatMulNBits weight [N, K]: packed uint8 [N, K/2], scales [N, K/bs], zp or None."""
+
+    def __init__(self, N, K, bs, has_zp=True, scale_dtype=torch.float16, device="cuda", name=""):
+        self.N, self.K, self.bs, self.has_zp, self.name = N, K, bs, has_zp, name
+        pb, sb, zb = mnb_packed_sizes(N, K, bs, scale_dtype, has_zp)
+        self.packed = torch.empty((N, K // 2), dtype=torch.uint8, device=device)
+        self.scales = torch.empty((N, K // bs), dtype=scale_dtype, device=device)
+        self.zp = torch.empty((N, (K // bs + 1) // 2), dtype=torch.uint8, device=device) if has_zp else None
+        self.nbytes = pb + sb + zb
+
+    @classmethod
+    def quantize(cls, W, bs, has_zp=True, scale_dtype=torch.float16, name="", stream=None):
+        """RTN-quantize an fp32 [N, K] device tensor with mnb_quantize_rtn."""
+        N, K = W.shape
+        q = cls(N, K, bs, has_zp, scale_dtype, W.device, name)
+        mnb_quantize_rtn(W.contiguous(), N, K, bs, has_zp, q.packed, q.scales, q.zp, stream)
+        return q
+
+    def dequantize(self, dtype=torch.float16, stream=None):
+        out = torch.empty((self.N, self.K), dtype=dtype, device=self.packed.device)
+        mnb_dequantize(self.packed, self.scales, self.zp, self.N, self.K, self.bs, out, stream)
+        return out
+
+    def gemv(self, X, Y, flags=0, stream=None):
+        mnb_gemv(X, self.packed, self.scales, self.zp, Y, X.shape[0], self.N, self.K, self.bs, flags, stream)
+
+    def gemm(self, X, Y, flags=0, stream=None):
+        mnb_gemm(X, self.packed, self.scales, self.zp, Y, X.shape[0], self.N, self.K, self.bs, flags, stream)
+
+
+class Pass:
+    """A chain of MatMulNBits calls with one X / Y buffer pair per linear.
+
+    kind = "gemv" (decode step, M <= 16) or "gemm" (prefill).  With pdl=True each
+    launch may overlap the tail of the previous one (weights stream early, X is
+    read after the previous kernel completes).  An optional int8 embedding
+    gather of M token ids runs first, as in a decode step.
+    """
+
+    def __init__(self, linears, M, kind="gemv", act_dtype=torch.float16, pdl=True, embed=None):
+        self.linears, self.M, self.kind, self.pdl = list(linears), M, kind, pdl
+        dev = self.linears[0].packed.device
+        self.X = [torch.zeros((M, l.K), dtype=act_dtype, device=dev) for l in self.linears]
+        self.Y = [torch.zeros((M, l.N), dtype=act_dtype, device=dev) for l in self.linears]
+        self.embed = embed   # (table, row_scales, ids[M], out[M, D]) or None
+        self.graph = None
+
+    @property
+    def weight_bytes(self):
+        return sum(l.nbytes for l in self.linears)
+
+    @property
+    def flops(self):
+        return sum(2 * self.M * l.N * l.K for l in self.linears)
+
+    @property
+    def launches(self):
+        return len(self.linears) + (1 if self.embed is not None else 0)
+
+    def run(self, stream=None):
+        if self.embed is not None:
+            table, rs, ids, out = self.embed
+            mnb_embed_gather(table, rs, table.shape[0], table.shape[1], ids, ids.shape[0], out,
+                             None, stream)
+        flags = MNB_FLAG_PDL if self.pdl else 0
+        for l, x, y in zip(self.linears, self.X, self.Y):
+            if self.kind == "gemv":
+                l.gemv(x, y, flags, stream)
+            else:
+                l.gemm(x, y, flags, stream)
+
+    def capture(self):
+        """Capture run() into a CUDA graph (replayed with replay())."""
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.run(s)          # warm-up outside the graph (first-use attribute setup)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            self.run(s)
+        self.graph = g
+        return g
+
+    def replay(self):
+        self.graph.replay()

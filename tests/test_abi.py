@@ -1,0 +1,116 @@
+"""Host-side checks of the C ABI: the library loads without a GPU, exports every
+entry point include/mnb.h declares, and rejects bad arguments with the
+documented codes before touching the device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mnb.h")
+
+OK, INVALID, SHAPE, ALIGN, UNSUPPORTED = 0, -1, -2, -3, -4
+F32, F16 = 0, 1
+A = 1 << 20          # a 16-byte aligned fake device address (never dereferenced)
+
+
+@pytest.fixture(scope="module")
+def mnb():
+    import int4_block_quantized_matmulnbits_b200 as m
+
+    return m
+
+
+@pytest.fixture(scope="module")
+def lib(mnb):
+    return mnb._lib
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mnb_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for f in ["mnb_packed_sizes", "mnb_quantize_rtn", "mnb_dequantize", "mnb_gemv", "mnb_gemm",
+              "mnb_embed_gather", "mnb_last_error", "mnb_device_status"]:
+        assert f in names
+
+
+def test_library_exports_every_declared_symbol(mnb):
+    raw = ctypes.CDLL(mnb.lib_path)
+    for name in declared_functions():
+        assert hasattr(raw, name), name
+
+
+def test_version_and_empty_error(mnb):
+    assert "sm_100a" in mnb.mnb_version()
+
+
+@pytest.mark.parametrize("N,K,bs,sdt,zp", [(2048, 1024, 32, F32, 1), (151936, 1024, 64, F16, 1),
+                                           (3, 96, 32, F16, 1), (5, 64, 64, F16, 0)])
+def test_packed_sizes_agree_with_oracle(lib, N, K, bs, sdt, zp):
+    p, s, z = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    assert lib.mnb_packed_sizes(N, K, bs, sdt, zp, ctypes.byref(p), ctypes.byref(s), ctypes.byref(z)) == OK
+    assert (p.value, s.value, z.value) == oracle.packed_sizes(N, K, bs, np.float16 if sdt else np.float32, bool(zp))
+
+
+def test_packed_sizes_rejects(lib):
+    p, s, z = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    args = (ctypes.byref(p), ctypes.byref(s), ctypes.byref(z))
+    assert lib.mnb_packed_sizes(4, 96, 48, F16, 1, *args) == SHAPE
+    assert lib.mnb_packed_sizes(4, 100, 32, F16, 1, *args) == SHAPE
+    assert lib.mnb_packed_sizes(-1, 64, 32, F16, 1, *args) == INVALID
+    assert lib.mnb_packed_sizes(4, 64, 32, 7, 1, *args) == INVALID
+    assert lib.mnb_packed_sizes(4, 64, 32, F16, 1, None, None, None) == INVALID
+    assert "NULL" in lib.mnb_last_error().decode()
+
+
+def test_gemv_argument_checks(lib):
+    g = lib.mnb_gemv
+    assert g(A, F16, A, A, F16, A, A, 17, 64, 64, 32, 0, None) == UNSUPPORTED
+    assert g(A, F16, A, A, F16, A, A, 1, 64, 96, 64, 0, None) == SHAPE          # K % bs
+    assert g(A, F16, A, A, F16, A, A, 1, 64, 64, 16, 0, None) == SHAPE          # bs
+    assert g(None, F16, A, A, F16, A, A, 1, 64, 64, 32, 0, None) == INVALID
+    assert g(A + 8, F16, A, A, F16, A, A, 1, 64, 64, 32, 0, None) == ALIGN
+    assert g(A, F16, A, A + 1, F16, A, A, 1, 64, 64, 32, 0, None) == ALIGN     # fp16 scales, odd address
+    assert g(A, F16, A, A, F16, A, A, -1, 64, 64, 32, 0, None) == INVALID
+    assert g(A, 5, A, A, F16, A, A, 1, 64, 64, 32, 0, None) == INVALID
+    assert g(A, F16, A, A, F16, A, A, 1, 64, 64, 32, 0x80, None) == INVALID   # unknown flag
+    assert g(A, F16, A, A, F16, A, A, 0, 64, 64, 32, 0, None) == OK            # M = 0: nothing to do
+    assert g(A, F16, A, A, F16, A, A, 1, 0, 64, 32, 0, None) == OK             # N = 0
+
+
+def test_gemm_argument_checks(lib):
+    g = lib.mnb_gemm
+    assert g(A, F32, A, A, F16, A, A, 64, 128, 64, 32, 0, None) == UNSUPPORTED   # fp32 activations
+    assert g(A, F16, A, A, F16, A, A, 64, 100, 64, 32, 0, None) == SHAPE          # N % 128
+    assert g(A, F16, A, A, F16, A, A, 64, 128, 96, 32, 0, None) == SHAPE          # K % 64
+    assert g(A, F16, A + 4, A, F16, A, A, 64, 128, 64, 32, 0, None) == ALIGN
+    assert g(A, F16, A, A, F16, A, A, 0, 128, 64, 32, 0, None) == OK
+
+
+def test_quantize_dequantize_embed_argument_checks(lib):
+    assert lib.mnb_quantize_rtn(A, 4, 96, 64, 1, A, A, F16, A, None) == SHAPE
+    assert lib.mnb_quantize_rtn(A, 4, 64, 32, 1, A, A, F16, None, None) == INVALID   # zp needed
+    assert lib.mnb_quantize_rtn(A + 4, 4, 64, 32, 1, A, A, F16, A, None) == ALIGN
+    assert lib.mnb_quantize_rtn(A, 0, 64, 32, 1, A, A, F16, A, None) == OK
+    assert lib.mnb_dequantize(A, A, F16, None, 4, 64, 32, A + 2, F16, None) == ALIGN
+    assert lib.mnb_dequantize(A, A, 3, None, 4, 64, 32, A, F16, None) == INVALID
+    assert lib.mnb_embed_gather(A, A, 10, 24, A, 4, A, F16, None, None) == SHAPE    # D % 16
+    assert lib.mnb_embed_gather(A, A, 10, 32, None, 4, A, F16, None, None) == INVALID
+    assert lib.mnb_embed_gather(A, A, 10, 32, A, 4, A + 8, F16, None, None) == ALIGN
+    assert lib.mnb_embed_gather(A, A, 10, 32, A, 0, A, F16, None, None) == OK
+    assert lib.mnb_device_status(None, 0) == INVALID
+
+
+def test_binding_raises_with_message(mnb):
+    with pytest.raises(mnb.MnbError) as e:
+        mnb.mnb_packed_sizes(4, 100, 32)
+    assert "MNB_ERR_SHAPE" in str(e.value) and "K=100" in str(e.value)

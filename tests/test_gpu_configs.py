@@ -1,0 +1,159 @@
+"""Parity at the full workload sizes, in the launch configuration bench.py times.
+
+Each workload's weights are generated and RTN-quantized on the device, then the
+whole pass (decode-step GEMVs or prefill GEMMs, every projection, PDL launches,
+captured in a CUDA graph) runs exactly as the benchmark runs it.  The oracle
+then recomputes sampled output columns one by one: for a sample of weight rows
+of every projection it re-quantizes those rows from the same fp32 weights
+(bit-exact check of packed bytes, scales and zero points) and recomputes the
+outputs in double precision (tolerance check).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from tests.parity_util import assert_close, np_of
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def step_mod(cuda_dev):
+    from int4_block_quantized_matmulnbits_b200 import step
+
+    return step
+
+
+def _sample_rows(N, count, seed):
+    if count >= N:
+        return np.arange(N)
+    rng = np.random.default_rng(seed)
+    rows = set(rng.choice(N, size=count - 2, replace=False).tolist())
+    rows.update([0, N - 1])
+    return np.array(sorted(rows))
+
+
+_MODELS = {}
+
+
+def model(step_mod, cfg_name, rows_per_proj, full_layers=()):
+    """build_model, cached per workload for the whole module."""
+    key = (cfg_name, rows_per_proj, tuple(full_layers))
+    if key not in _MODELS:
+        _MODELS.clear()
+        torch.cuda.empty_cache()
+        _MODELS[key] = build_model(step_mod, cfg_name, rows_per_proj, full_layers)
+    return _MODELS[key]
+
+
+def build_model(step_mod, cfg_name, rows_per_proj, full_layers=(), dev="cuda"):
+    """QLinears of a workload, plus the sampled fp32 weight rows for the oracle."""
+    cfg = workloads.CONFIGS[cfg_name]
+    sdt = torch.float16 if cfg["scale"] == "f16" else torch.float32
+    lins, samples = [], []
+    for lin in workloads.config_linears(cfg_name):
+        W = workloads.weight(cfg["seed"], lin.layer, lin.proj, lin.N, lin.K, cfg.get("outliers", False), device=dev)
+        q = step_mod.QLinear.quantize(W, cfg["bs"], cfg["has_zp"], sdt, name=f"{lin.name}{lin.layer}")
+        count = lin.N if lin.layer in full_layers else rows_per_proj
+        rows = _sample_rows(lin.N, count, lin.layer * 16 + lin.proj)
+        samples.append((rows, W[torch.from_numpy(rows).to(dev)].cpu().numpy()))
+        del W
+        lins.append(q)
+    torch.cuda.synchronize()
+    return cfg, lins, samples
+
+
+def check_pass(cfg, lins, samples, p, act):
+    """Bit-exact RTN on the sampled rows, then sampled outputs within tolerance."""
+    sdt = np.float16 if cfg["scale"] == "f16" else np.float32
+    for q, (rows, Wrows), X, Y in zip(lins, samples, p.X, p.Y):
+        pr, sr, zr = oracle.quantize_rtn(Wrows, cfg["bs"], cfg["has_zp"], sdt)
+        idx = torch.from_numpy(rows).to(q.packed.device)
+        assert np.array_equal(np_of(q.packed[idx]), pr), q.name
+        assert np.array_equal(np_of(q.scales[idx]).view(np.uint8), sr.view(np.uint8)), q.name
+        if cfg["has_zp"]:
+            assert np.array_equal(np_of(q.zp[idx]), zr), q.name
+        ref = oracle.matmul(np_of(X.float()), pr, sr, zr, q.K, cfg["bs"])
+        got = np_of(Y[:, idx].float())
+        assert_close(got, ref, act)
+
+
+def _fill_inputs(p, seed, act_dtype):
+    for i, x in enumerate(p.X):
+        x.copy_(workloads.activations(seed, x.shape[0], x.shape[1], act_dtype, tag=i))
+
+
+def _run_graph(p):
+    p.capture()
+    p.replay()
+    torch.cuda.synchronize()
+
+
+def test_single_gemv_fp32(step_mod, cuda_dev):
+    cfg, lins, samples = build_model(step_mod, "single_gemv", 2048)
+    p = step_mod.Pass(lins, 1, "gemv", torch.float32)
+    _fill_inputs(p, cfg["seed"], torch.float32)
+    _run_graph(p)
+    check_pass(cfg, lins, samples, p, "f32")
+
+
+def test_qwen3_0p6b_decode_step(step_mod, cuda_dev):
+    cfg, lins, samples = build_model(step_mod, "qwen3_0p6b_decode", 96, full_layers=(0,))
+    p = step_mod.Pass(lins, 1, "gemv", torch.float16)
+    _fill_inputs(p, cfg["seed"], torch.float16)
+    _run_graph(p)
+    check_pass(cfg, lins, samples, p, "f16")
+
+
+@pytest.mark.parametrize("M", [1, 2, 4, 8, 16])
+def test_qwen3_1p7b_decode_step(step_mod, cuda_dev, M):
+    cfg, lins, samples = model(step_mod, "qwen3_1p7b_decode", 48, full_layers=(27,))
+    p = step_mod.Pass(lins, M, "gemv", torch.float16)
+    _fill_inputs(p, cfg["seed"] + M, torch.float16)
+    _run_graph(p)
+    check_pass(cfg, lins, samples, p, "f16")
+
+
+@pytest.mark.parametrize("M", [64, 256, 420, 1024])
+def test_qwen3_1p7b_prefill(step_mod, cuda_dev, M):
+    cfg, lins, samples = model(step_mod, "qwen3_1p7b_prefill", 24)
+    p = step_mod.Pass(lins, M, "gemm", torch.float16)
+    _fill_inputs(p, cfg["seed"] + M, torch.float16)
+    _run_graph(p)
+    import int4_block_quantized_matmulnbits_b200 as mnb
+
+    assert mnb.mnb_device_status() == 0
+    check_pass(cfg, lins, samples, p, "f16")
+
+
+@pytest.mark.parametrize("variant", ["qwen3_0p6b_bs64", "qwen3_0p6b_nozp"])
+def test_layout_variants(step_mod, cuda_dev, variant):
+    cfg, lins, samples = build_model(step_mod, variant, 32)
+    for M in cfg["gemv_M"]:
+        p = step_mod.Pass(lins, M, "gemv", torch.float16)
+        _fill_inputs(p, cfg["seed"] + M, torch.float16)
+        _run_graph(p)
+        check_pass(cfg, lins, samples, p, "f16")
+    body = [l for l in lins if l.N != workloads.VOCAB]
+    bsamp = [s for l, s in zip(lins, samples) if l.N != workloads.VOCAB]
+    for M in cfg["gemm_M"]:
+        p = step_mod.Pass(body, M, "gemm", torch.float16)
+        _fill_inputs(p, cfg["seed"] + M, torch.float16)
+        _run_graph(p)
+        check_pass(cfg, body, bsamp, p, "f16")
+
+
+def test_embed_gather_full_table(cuda_dev):
+    import int4_block_quantized_matmulnbits_b200 as mnb
+
+    e = workloads.EMBED
+    table, scales, ids = workloads.embed_inputs(e["seed"], e["V"], e["D"], e["T"])
+    out = torch.empty((e["T"], e["D"]), dtype=torch.float16, device=cuda_dev)
+    status = torch.zeros((1,), dtype=torch.int32, device=cuda_dev)
+    mnb.mnb_embed_gather(table.to(cuda_dev), scales.to(cuda_dev), e["V"], e["D"], ids.to(cuda_dev), e["T"],
+                         out, status)
+    ref, st = oracle.embed_gather(table.numpy(), scales.numpy(), ids.numpy(), np.float16)
+    assert np.array_equal(np_of(out).view(np.uint8), ref.view(np.uint8))
+    assert int(status.item()) == st == 0

@@ -1,0 +1,283 @@
+"""GPU parity of every kernel against the CPU oracle, through the C ABI binding.
+
+Sizes are small enough for the oracle to finish in seconds while still spanning
+several tiles and a ragged tail.  Bit-exact: packing, scales, zero points,
+dequantized weights, embedding rows.  Tolerances (relative L2 over all outputs,
+max absolute error): 1e-5 / 2e-2 for fp32 activations, 2e-3 / 2e-2 for fp16.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from tests.parity_util import assert_close, np_of, random_packed, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def mnb(cuda_dev):
+    import int4_block_quantized_matmulnbits_b200 as m
+
+    m.mnb_device_status(clear=True)
+    return m
+
+
+def _quantize_dev(mnb, W, bs, has_zp, sdt, dev):
+    N, K = W.shape
+    packed = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((N, K // bs), dtype=sdt, device=dev)
+    zp = torch.empty((N, (K // bs + 1) // 2), dtype=torch.uint8, device=dev) if has_zp else None
+    mnb.mnb_quantize_rtn(W.to(dev), N, K, bs, has_zp, packed, scales, zp)
+    torch.cuda.synchronize()
+    return packed, scales, zp
+
+
+# ------------------------------------------------------------------ quantization
+
+@pytest.mark.parametrize("N,K,bs", [(1, 32, 32), (37, 96, 32), (64, 256, 64), (130, 192, 64),
+                                    (300, 1024, 32), (2048, 1024, 32)])
+@pytest.mark.parametrize("has_zp", [True, False])
+@pytest.mark.parametrize("sdt", [torch.float32, torch.float16])
+def test_quantize_rtn_bit_exact(mnb, cuda_dev, N, K, bs, has_zp, sdt):
+    g = torch.Generator().manual_seed(N * 7 + K + bs)
+    W = torch.randn((N, K), generator=g) * 0.02
+    W[::5] = W[::5] * 8.0                                   # outlier rows
+    if N > 2:
+        W[1, :bs] = 0.0                                     # an all-zero block
+        W[2, :] = W[2, :].abs() + 0.01                      # all-positive blocks
+    p_ref, s_ref, z_ref = oracle.quantize_rtn(W.numpy(), bs, has_zp,
+                                              np.float16 if sdt == torch.float16 else np.float32)
+    packed, scales, zp = _quantize_dev(mnb, W, bs, has_zp, sdt, cuda_dev)
+    assert np.array_equal(np_of(packed), p_ref)
+    assert np.array_equal(np_of(scales).view(np.uint8), s_ref.view(np.uint8))
+    if has_zp:
+        assert np.array_equal(np_of(zp), z_ref)
+
+
+def test_quantize_rtn_ties_and_constructed_block(mnb, cuda_dev):
+    W = np.zeros((3, 64), np.float32)
+    W[0, :32] = np.repeat(np.arange(-7, 9) * 0.5, 2)          # scale 0.5, zp 7, exact
+    W[1, 0], W[1, 1:16] = 15.0, np.arange(0.5, 15.0, 1.0)     # x.5 ties, scale 1
+    W[2, :4] = [-7.0, 8.0, 0.5, -0.5]                          # tie after adding zp
+    p_ref, s_ref, z_ref = oracle.quantize_rtn(W, 32)
+    packed, scales, zp = _quantize_dev(mnb, torch.from_numpy(W), 32, True, torch.float32, cuda_dev)
+    assert np.array_equal(np_of(packed), p_ref)
+    assert np.array_equal(np_of(scales), s_ref)
+    assert np.array_equal(np_of(zp), z_ref)
+
+
+# ------------------------------------------------------------------ dequantization
+
+@pytest.mark.parametrize("N,K,bs,has_zp", [(37, 96, 32, True), (64, 256, 64, True), (16, 128, 32, False)])
+@pytest.mark.parametrize("sdt", [np.float32, np.float16])
+@pytest.mark.parametrize("odt", [torch.float32, torch.float16])
+def test_dequantize_bit_exact(mnb, cuda_dev, N, K, bs, has_zp, sdt, odt):
+    rng = np.random.default_rng(N + K)
+    packed, scales, zp = random_packed(rng, N, K, bs, has_zp, sdt, 0.001, 0.5)
+    out = torch.empty((N, K), dtype=odt, device=cuda_dev)
+    mnb.mnb_dequantize(to_dev(packed, cuda_dev), to_dev(scales, cuda_dev), to_dev(zp, cuda_dev),
+                       N, K, bs, out)
+    ref = oracle.dequantize(packed, scales, zp, K, bs, np.float16 if odt == torch.float16 else np.float32)
+    assert np.array_equal(np_of(out).view(np.uint8), ref.view(np.uint8))
+
+
+# ------------------------------------------------------------------ GEMV
+
+GEMV_CASES = [
+    # M, N, K, bs, has_zp, act, scale
+    (1, 2048, 1024, 32, True, "f32", np.float32),
+    (3, 37, 96, 32, True, "f32", np.float32),
+    (16, 64, 128, 64, False, "f32", np.float16),
+    (1, 37, 96, 32, True, "f16", np.float16),
+    (1, 1024, 2048, 32, True, "f16", np.float16),
+    (2, 3000, 1024, 64, True, "f16", np.float16),
+    (5, 130, 6144, 32, True, "f16", np.float16),
+    (8, 512, 3072, 32, False, "f16", np.float16),
+    (9, 256, 2048, 64, True, "f16", np.float16),
+    (16, 2048, 2048, 32, True, "f16", np.float16),
+    (16, 48, 64, 32, True, "f16", np.float32),
+    (4, 16, 32, 32, True, "f16", np.float16),
+]
+
+
+def _run_gemv(mnb, dev, X, packed, scales, zp, M, N, K, bs, flags=0):
+    Y = torch.empty((M, N), dtype=X.dtype, device=dev)
+    mnb.mnb_gemv(X, to_dev(packed, dev), to_dev(scales, dev), to_dev(zp, dev), Y, M, N, K, bs, flags)
+    torch.cuda.synchronize()
+    return Y
+
+
+@pytest.mark.parametrize("M,N,K,bs,has_zp,act,sdt", GEMV_CASES)
+def test_gemv_parity(mnb, cuda_dev, M, N, K, bs, has_zp, act, sdt):
+    rng = np.random.default_rng(M * 1000 + N + K)
+    packed, scales, zp = random_packed(rng, N, K, bs, has_zp, sdt)
+    tdt = torch.float16 if act == "f16" else torch.float32
+    X = torch.randn((M, K), generator=torch.Generator().manual_seed(K)).to(tdt)
+    Y = _run_gemv(mnb, cuda_dev, X.to(cuda_dev), packed, scales, zp, M, N, K, bs)
+    ref = oracle.matmul(X.float().numpy(), packed, scales, zp, K, bs)
+    assert_close(np_of(Y.float()), ref, act)
+
+
+@pytest.mark.parametrize("M", [1, 2])
+def test_gemv_f16_cuda_core_variant(mnb, cuda_dev, M):
+    rng = np.random.default_rng(77 + M)
+    N, K, bs = 1000, 2048, 32
+    packed, scales, zp = random_packed(rng, N, K, bs, True, np.float16)
+    X = torch.randn((M, K), generator=torch.Generator().manual_seed(3)).half()
+    assert mnb._lib.mnb_tune_gemv_f16_cc_max_m(2) == 0
+    try:
+        Y = _run_gemv(mnb, cuda_dev, X.to(cuda_dev), packed, scales, zp, M, N, K, bs)
+    finally:
+        mnb._lib.mnb_tune_gemv_f16_cc_max_m(0)
+    ref = oracle.matmul(X.float().numpy(), packed, scales, zp, K, bs)
+    assert_close(np_of(Y.float()), ref, "f16")
+
+
+def test_gemv_q_equal_zp_gives_exact_zero(mnb, cuda_dev):
+    N, K, bs, M = 64, 256, 32, 3
+    z = np.random.default_rng(1).integers(0, 16, (N, K // bs))
+    q = np.repeat(z, bs, axis=1)
+    packed = (q[:, 0::2] | (q[:, 1::2] << 4)).astype(np.uint8)
+    zp = (z[:, 0::2] | (z[:, 1::2] << 4)).astype(np.uint8)
+    scales = np.full((N, K // bs), 0.5, np.float16)
+    for dt in (torch.float16, torch.float32):
+        X = torch.randn((M, K)).to(dt).to(cuda_dev)
+        Y = _run_gemv(mnb, cuda_dev, X, packed, scales, zp, M, N, K, bs)
+        assert torch.count_nonzero(Y).item() == 0
+
+
+def test_gemv_rtn_quantized_weights(mnb, cuda_dev):
+    # the product path end to end: RTN on the device, GEMV on the device, oracle on its own RTN
+    N, K, bs, M = 1024, 2048, 32, 1
+    W = workloads.weight(2, 0, 4, N, K, outliers=True)
+    p_ref, s_ref, z_ref = oracle.quantize_rtn(W.numpy(), bs, True, np.float16)
+    packed, scales, zp = _quantize_dev(mnb, W, bs, True, torch.float16, cuda_dev)
+    X = workloads.activations(2, M, K)
+    Y = torch.empty((M, N), dtype=torch.float16, device=cuda_dev)
+    mnb.mnb_gemv(X.to(cuda_dev), packed, scales, zp, Y, M, N, K, bs)
+    ref = oracle.matmul(X.float().numpy(), p_ref, s_ref, z_ref, K, bs)
+    assert_close(np_of(Y.float()), ref, "f16")
+
+
+def test_gemv_pdl_chain_and_graph_match_eager(mnb, cuda_dev):
+    # Y of one call is X of the next: the PDL launches must still see it
+    rng = np.random.default_rng(9)
+    K = 1024
+    layers = [random_packed(rng, K, K, 32, True, np.float16, 0.003, 0.004) for _ in range(6)]
+    dev_layers = [(to_dev(p, cuda_dev), to_dev(s, cuda_dev), to_dev(z, cuda_dev)) for p, s, z in layers]
+    x0 = torch.randn((1, K)).half().to(cuda_dev)
+
+    def chain(flags, bufs):
+        x = x0
+        for (p, s, z), y in zip(dev_layers, bufs):
+            mnb.mnb_gemv(x, p, s, z, y, 1, K, K, 32, flags)
+            x = y
+        return x
+
+    bufs_plain = [torch.empty((1, K), dtype=torch.float16, device=cuda_dev) for _ in layers]
+    bufs_pdl = [torch.empty((1, K), dtype=torch.float16, device=cuda_dev) for _ in layers]
+    ref = chain(0, bufs_plain).clone()
+    for _ in range(3):
+        got = chain(mnb.MNB_FLAG_PDL, bufs_pdl)
+    torch.cuda.synchronize()
+    assert torch.equal(got, ref)
+    # the same chain captured in a CUDA graph
+    bufs_g = [torch.zeros((1, K), dtype=torch.float16, device=cuda_dev) for _ in layers]
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        chain(mnb.MNB_FLAG_PDL, bufs_g)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(bufs_g[-1], ref)
+    # first link against the oracle
+    p, sc, z = layers[0]
+    r0 = oracle.matmul(x0.float().cpu().numpy(), p, sc, z, K, 32)
+    assert_close(np_of(bufs_plain[0].float()), r0, "f16")
+
+
+# ------------------------------------------------------------------ GEMM (tcgen05)
+
+GEMM_CASES = [
+    # M, N, K, bs, has_zp, scale
+    (1, 128, 64, 32, True, np.float16),
+    (16, 128, 128, 64, True, np.float16),
+    (63, 256, 192, 32, False, np.float16),
+    (64, 1024, 2048, 32, True, np.float16),
+    (100, 384, 1024, 64, True, np.float16),
+    (256, 512, 2048, 32, True, np.float16),
+    (300, 128, 6144, 32, True, np.float16),
+    (420, 2048, 1024, 32, True, np.float16),
+    (1024, 256, 512, 64, False, np.float16),
+    (129, 128, 256, 32, True, np.float32),
+]
+
+
+@pytest.mark.parametrize("M,N,K,bs,has_zp,sdt", GEMM_CASES)
+def test_gemm_parity(mnb, cuda_dev, M, N, K, bs, has_zp, sdt):
+    rng = np.random.default_rng(M * 31 + N + K)
+    packed, scales, zp = random_packed(rng, N, K, bs, has_zp, sdt)
+    X = torch.randn((M, K), generator=torch.Generator().manual_seed(M + K)).half()
+    Y = torch.full((M, N), float("nan"), dtype=torch.float16, device=cuda_dev)
+    mnb.mnb_gemm(X.to(cuda_dev), to_dev(packed, cuda_dev), to_dev(scales, cuda_dev), to_dev(zp, cuda_dev),
+                 Y, M, N, K, bs)
+    torch.cuda.synchronize()
+    assert mnb.mnb_device_status() == 0
+    ref = oracle.matmul(X.float().numpy(), packed, scales, zp, K, bs)
+    assert_close(np_of(Y.float()), ref, "f16")
+
+
+def test_gemm_matches_dequantized_weights_exactly_where_exact(mnb, cuda_dev):
+    # power-of-two scales and small integers: every product and sum is exact in fp32
+    N, K, M, bs = 256, 512, 80, 32
+    rng = np.random.default_rng(5)
+    packed, _, zp = random_packed(rng, N, K, bs, True, np.float16)
+    scales = (2.0 ** rng.integers(-6, -2, (N, K // bs))).astype(np.float16)
+    X = torch.from_numpy(rng.integers(-4, 5, (M, K)).astype(np.float16))
+    Y = torch.empty((M, N), dtype=torch.float16, device=cuda_dev)
+    mnb.mnb_gemm(X.to(cuda_dev), to_dev(packed, cuda_dev), to_dev(scales, cuda_dev), to_dev(zp, cuda_dev),
+                 Y, M, N, K, bs)
+    ref = oracle.matmul(X.float().numpy(), packed, scales, zp, K, bs)
+    assert np.array_equal(np_of(Y).astype(np.float64), ref.astype(np.float16).astype(np.float64))
+
+
+def test_gemm_q_equal_zp_gives_exact_zero(mnb, cuda_dev):
+    N, K, bs, M = 128, 256, 64, 70
+    z = np.random.default_rng(2).integers(0, 16, (N, K // bs))
+    q = np.repeat(z, bs, axis=1)
+    packed = (q[:, 0::2] | (q[:, 1::2] << 4)).astype(np.uint8)
+    zp = (z[:, 0::2] | (z[:, 1::2] << 4)).astype(np.uint8)
+    scales = np.full((N, K // bs), 0.25, np.float16)
+    Y = torch.ones((M, N), dtype=torch.float16, device=cuda_dev)
+    mnb.mnb_gemm(torch.randn((M, K)).half().to(cuda_dev), to_dev(packed, cuda_dev), to_dev(scales, cuda_dev),
+                 to_dev(zp, cuda_dev), Y, M, N, K, bs)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(Y).item() == 0
+
+
+# ------------------------------------------------------------------ embedding gather
+
+@pytest.mark.parametrize("V,D,T", [(1000, 1024, 4096), (50, 16, 1), (300, 80, 37)])
+@pytest.mark.parametrize("odt", [torch.float16, torch.float32])
+def test_embed_gather_bit_exact(mnb, cuda_dev, V, D, T, odt):
+    table, scales, ids = workloads.embed_inputs(7, V, D, T)
+    ids = ids.clone()
+    if T > 3:
+        ids[1], ids[2] = -5, V         # out of range -> zero rows + status bit
+    status = torch.zeros((1,), dtype=torch.int32, device=cuda_dev)
+    out = torch.full((T, D), 7.0, dtype=odt, device=cuda_dev)
+    mnb.mnb_embed_gather(table.to(cuda_dev), scales.to(cuda_dev), V, D, ids.to(cuda_dev), T, out, status)
+    ref, st = oracle.embed_gather(table.numpy(), scales.numpy(), ids.numpy(),
+                                  np.float16 if odt == torch.float16 else np.float32)
+    assert np.array_equal(np_of(out).view(np.uint8), ref.view(np.uint8))
+    assert int(status.item()) == st
+
+
+def test_no_timeouts_recorded(mnb, cuda_dev):
+    torch.cuda.synchronize()
+    assert mnb.mnb_device_status() == 0
