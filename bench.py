@@ -1,0 +1,470 @@
+"""Benchmark of the MatMulNBits hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+A step is one Qwen3-1.7B-shaped decode step at M = 1: the 28 x 7 projections
+plus the lm_head, 197 calls of mnb_gemv (int4 block-32 asymmetric weights,
+fp16 activations and scales), replayed from a CUDA graph with programmatic
+dependent launch.  `value` is the weight bytes the step streams per second
+(packed nibbles + scales + zero points), inputs already in HBM; the weights
+(995 MB) are larger than L2, so no flush is needed.  `e2e` repeats the step
+through the same calls with the inputs copied from pinned host memory and
+the outputs copied back inside the timed region.  `prefill` times the
+tensor-core path (mnb_gemm) on the same model's 196 projections at M = 1024
+(TFLOP/s).  Under torchrun every rank runs its own replica (the operator has
+no exchange step); time is the max over ranks.
+
+--impl reference times the CPU oracle (tests' reference implementation) on a
+bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "M=1 GEMV weight GB/s & prefill TFLOP/s on one B200, as % of HBM/TC roofline"
+WORKLOAD = ("qwen3-1.7b-shaped decode step, M=1: 28 layers x (q 2048->2048, k/v 2048->1024, "
+            "o 2048->2048, gate/up 2048->6144, down 6144->2048) + lm_head 2048->151936; "
+            "int4 block 32 asymmetric, fp16 activations and scales, weights N(0,0.02) with 1% outliers x8")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# --------------------------------------------------------------------------- ranks
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+class Ranks:
+    def __init__(self, world, rank, local, backend):
+        import torch
+        import torch.distributed as dist
+
+        self.world, self.rank, self.local = world, rank, local
+        self.dist = dist if world > 1 else None
+        if self.dist:
+            import datetime
+
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+
+    def barrier(self):
+        if self.dist:
+            self.dist.barrier()
+
+    def max(self, v):
+        if not self.dist:
+            return v
+        import torch
+
+        dev = "cuda" if self.dist.get_backend() == "nccl" else "cpu"
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.dist:
+            self.dist.destroy_process_group()
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML in a thread."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index, period=0.005):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self.period, self.index = period, index
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report it instead of clocks
+            self.err = repr(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def _sample(self):
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            pass
+
+    def __enter__(self):
+        if self.ok:
+            self._stop = threading.Event()
+            self._sample()
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+            self._sample()
+
+    def summary(self):
+        if not self.ok:
+            return {"error": getattr(self, "err", "nvml unavailable")}
+        names = [n for b, n in self.REASONS.items() if self.reasons & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------- workloads
+
+def build_model(cfg_name, dev, lm_head=True):
+    import torch
+
+    import workloads
+    from int4_block_quantized_matmulnbits_b200.step import QLinear
+
+    cfg = workloads.CONFIGS[cfg_name]
+    lins = []
+    linears = workloads.config_linears(cfg_name)
+    if not lm_head:
+        linears = [l for l in linears if l.name != "lm_head"]
+    for lin in linears:
+        W = workloads.weight(cfg["seed"], lin.layer, lin.proj, lin.N, lin.K, cfg.get("outliers", False), device=dev)
+        lins.append(QLinear.quantize(W, cfg["bs"], cfg["has_zp"], torch.float16, name=f"{lin.name}{lin.layer}"))
+        del W
+    torch.cuda.synchronize()
+    return cfg, lins
+
+
+def fill(p, seed):
+    import torch
+
+    import workloads
+
+    for i, x in enumerate(p.X):
+        x.copy_(workloads.activations(seed, x.shape[0], x.shape[1], torch.float16, tag=i, device=x.device))
+
+
+def timed_replays(p, steps, warmup, ranks, tag="timed"):
+    """Device time of `steps` graph replays (ms, max over ranks).  The timed
+    loop sits in an NVTX range named `tag` (for profiler filtering)."""
+    import torch
+
+    for _ in range(warmup):
+        p.replay()
+    torch.cuda.synchronize()
+    ranks.barrier()
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push(tag)
+    e0.record(s)
+    for _ in range(steps):
+        p.replay()
+    e1.record(s)
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize()
+    ranks.barrier()
+    return ranks.max(e0.elapsed_time(e1))
+
+
+def timed_e2e(p, steps, warmup, ranks):
+    """Step time with the inputs copied in from pinned host memory and the outputs
+    copied back, all inside the timed region (ms per step, max over ranks)."""
+    import torch
+
+    hx = torch.empty(p.x_flat.shape, dtype=p.x_flat.dtype, pin_memory=True)
+    hx.copy_(p.x_flat.cpu())
+    hy = torch.empty(p.y_flat.shape, dtype=p.y_flat.dtype, pin_memory=True)
+    s = torch.cuda.current_stream()
+
+    def one():
+        p.x_flat.copy_(hx, non_blocking=True)
+        p.replay()
+        hy.copy_(p.y_flat, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    ranks.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(steps):
+        one()
+    e1.record(s)
+    torch.cuda.synchronize()
+    ranks.barrier()
+    ms = ranks.max(e0.elapsed_time(e1)) / steps
+    return ms, hx.numel() * hx.element_size(), hy.numel() * hy.element_size()
+
+
+class OracleSample:
+    """The CPU oracle on a bounded sample of the decode step: the 7 projections
+    of layer 0 at M = 1, weights RTN-quantized by the oracle itself (prepared
+    once, outside any timing)."""
+
+    def __init__(self):
+        import numpy as np
+
+        import oracle
+        import workloads
+
+        self.oracle = oracle
+        cfg = workloads.CONFIGS["qwen3_1p7b_decode"]
+        self.bs = cfg["bs"]
+        self.items = []
+        for l in workloads.config_linears("qwen3_1p7b_decode"):
+            if l.layer != 0:
+                continue
+            W = workloads.weight(cfg["seed"], l.layer, l.proj, l.N, l.K, True).numpy()
+            pk, sc, zp = oracle.quantize_rtn(W, self.bs, True, np.float16)
+            X = workloads.activations(cfg["seed"], 1, l.K, tag=l.proj).float().numpy()
+            nbytes = sum(oracle.packed_sizes(l.N, l.K, self.bs, np.float16, True))
+            self.items.append((l.name, X, pk, sc, zp, l.K, nbytes))
+        self.cores = oracle.num_threads()
+
+    def run(self, i):
+        """Projection i % 7 of layer 0; returns (weight bytes, seconds)."""
+        name, X, pk, sc, zp, K, nbytes = self.items[i % len(self.items)]
+        t0 = time.perf_counter()
+        self.oracle.matmul(X, pk, sc, zp, K, self.bs)
+        return nbytes, time.perf_counter() - t0
+
+    def measure(self, reps):
+        """GB/s over `reps` passes of the whole layer."""
+        tot_b = tot_t = 0.0
+        for r in range(reps):
+            for i in range(len(self.items)):
+                b, t = self.run(i)
+                tot_b, tot_t = tot_b + b, tot_t + t
+        return tot_b / tot_t / 1e9, tot_t
+
+
+# --------------------------------------------------------------------------- arms
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    sample = OracleSample()
+    for i in range(args.warmup):
+        sample.run(i)
+    tot_b = tot_t = 0.0
+    for i in range(args.steps):
+        b, t = sample.run(args.warmup + i)
+        tot_b, tot_t = tot_b + b, tot_t + t
+    gbs = tot_b / tot_t / 1e9
+    desc = ("oracle.matmul, one projection of layer 0 of the decode step per step (cycling q, k, v, o, "
+            "gate, up, down), M=1")
+    out = {"impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1000.0 * tot_t / args.steps, 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic", "config": {"workload": WORKLOAD, "M": 1, "sample": desc},
+           "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": sample.cores, "kind": "oracle",
+                            "sample": desc},
+           "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def profile_part(args, dev, ranks):
+    """Small cases for ncu captures: the lm_head GEMV alone (180 MB of weights,
+    larger than L2) or layer 0 of the prefill at M = 1024 on the tensor cores."""
+    import torch
+
+    import workloads
+    from int4_block_quantized_matmulnbits_b200.step import Pass, QLinear
+
+    cfg = workloads.CONFIGS["qwen3_1p7b_decode"]
+    if args.only == "lmhead":
+        lin = [l for l in workloads.config_linears("qwen3_1p7b_decode") if l.name == "lm_head"]
+        M, kind = 1, "gemv"
+    else:
+        lin = [l for l in workloads.config_linears("qwen3_1p7b_prefill") if l.layer == 0]
+        M, kind = 1024, "gemm"
+    lins = []
+    for l in lin:
+        W = workloads.weight(cfg["seed"], l.layer, l.proj, l.N, l.K, True, device=dev)
+        lins.append(QLinear.quantize(W, cfg["bs"], True, torch.float16, name=l.name))
+        del W
+    p = Pass(lins, M, kind, torch.float16, pdl=False)
+    fill(p, cfg["seed"])
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        p.run()
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("profiled")
+    for _ in range(args.steps):
+        p.run()
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize()
+
+
+def run_gpu(args, world, rank, local):
+    import torch
+
+    ranks = Ranks(world, rank, local, "nccl")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    import int4_block_quantized_matmulnbits_b200 as mnb
+    from int4_block_quantized_matmulnbits_b200.step import Pass
+
+    if args.only in ("lmhead", "gemm-layer"):
+        profile_part(args, dev, ranks)
+        ranks.close()
+        return
+
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    tc_burst = float(peaks["bf16_tflops"])
+    tc_sust = float(peaks.get("bf16_tflops_sustained", tc_burst))
+
+    # ---- decode step, M = 1 (the headline)
+    cfg, lins = build_model("qwen3_1p7b_decode", dev)
+    dec = Pass(lins, 1, "gemv", torch.float16, pdl=True)
+    fill(dec, cfg["seed"])
+    dec.capture()
+    with ClockSampler(local) as clk:
+        ms_total = timed_replays(dec, args.steps, args.warmup, ranks, "decode")
+    if args.only == "decode":
+        ranks.close()
+        return
+    ms = ms_total / args.steps
+    wbytes = dec.weight_bytes
+    value = world * wbytes / (ms * 1e-3) / 1e9
+    per_launch_bytes = wbytes / len(lins)
+    per_launch_us = ms * 1000.0 / len(lins)
+    achieved = per_launch_bytes / (per_launch_us * 1e-6) / 1e9
+
+    # lm_head alone: one 180 MB launch, the kernel without launch gaps
+    lm = lins[-1]
+    lmp = Pass([lm], 1, "gemv", torch.float16, pdl=False)
+    fill(lmp, cfg["seed"] + 5)
+    lmp.capture()
+    lm_ms = timed_replays(lmp, 50, 5, ranks) / 50
+    lm_gbs = lm.nbytes / (lm_ms * 1e-3) / 1e9
+
+    e2e_ms, h2d, d2h = timed_e2e(dec, max(10, args.steps // 4), max(3, args.warmup), ranks)
+    e2e_val = world * wbytes / (e2e_ms * 1e-3) / 1e9
+
+    # decode at larger M (same weights)
+    by_m = {}
+    for M in (2, 4, 8, 16):
+        pm = Pass(lins, M, "gemv", torch.float16, pdl=True)
+        fill(pm, cfg["seed"] + M)
+        pm.capture()
+        t = timed_replays(pm, 100, 10, ranks) / 100
+        by_m[str(M)] = {"us_per_step": round(t * 1000, 2), "weight_gbs": round(wbytes / (t * 1e-3) / 1e9, 1),
+                        "frac_hbm": round(wbytes / (t * 1e-3) / 1e9 / hbm, 4)}
+        del pm
+    del dec, lmp
+    torch.cuda.empty_cache()
+
+    # ---- prefill on the tensor cores, M = 1024 (no lm_head: logits of the last position only)
+    body = [l for l in lins if l.name[:7] != "lm_head"]
+    prefill = {}
+    for M in (1024, 420, 256, 64):
+        pp = Pass(body, M, "gemm", torch.float16, pdl=True)
+        fill(pp, cfg["seed"] + M)
+        pp.capture()
+        n = 20 if M == 1024 else 10
+        with ClockSampler(local) as pclk:
+            t = timed_replays(pp, n, 3, ranks) / n
+        tflops = pp.flops / (t * 1e-3) / 1e12
+        prefill[str(M)] = {"ms_per_pass": round(t, 4), "tflops": round(tflops, 1),
+                           "frac_tc_sustained": round(tflops / tc_sust, 4),
+                           "frac_tc_burst": round(tflops / tc_burst, 4),
+                           "weight_gbs": round(pp.weight_bytes / (t * 1e-3) / 1e9, 1)}
+        if M == 1024:
+            prefill["1024"]["clocks"] = pclk.summary()
+            prefill["1024"]["gpu_launches"] = n * pp.launches
+        del pp
+        torch.cuda.empty_cache()
+    assert mnb.mnb_device_status() == 0, "a GEMM wait timed out"
+
+    cpu = None
+    if rank == 0 and world == 1:
+        sample = OracleSample()
+        gbs, dt = sample.measure(3)
+        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": sample.cores, "kind": "oracle",
+               "sample": f"oracle.matmul over the 7 projections of layer 0 of the decode step at M=1, "
+                         f"3 passes, {dt:.1f} s wall on {sample.cores} threads"}
+
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "M": 1, "launches_per_step": len(lins),
+                       "weight_bytes_per_step": wbytes, "graph": True, "pdl": True,
+                       "l2": "inputs larger than L2 (weights of one step > 126 MB)",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "hbm", "kernel": "gemv_kernel", "achieved": round(achieved, 1), "peak": hbm,
+                         "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": None,
+                         "peak_source": f"{peak_src} hbm_gbs", "bytes_per_launch": round(per_launch_bytes),
+                         "us_per_launch": round(per_launch_us, 3)},
+            "lm_head_alone": {"bytes": lm.nbytes, "us": round(lm_ms * 1000, 2), "gbs": round(lm_gbs, 1),
+                              "frac_hbm": round(lm_gbs / hbm, 4)},
+            "decode_by_M": by_m,
+            "prefill": prefill,
+            "roofline_prefill": {"bound": "tensor", "kernel": "gemm_kernel", "M": 1024,
+                                 "achieved": prefill["1024"]["tflops"], "peak": tc_sust, "unit": "TFLOP/s",
+                                 "frac": prefill["1024"]["frac_tc_sustained"], "traffic": None,
+                                 "peak_source": f"{peak_src} bf16_tflops_sustained (fp16 = bf16 nominal rate)"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(e2e_val, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
+            "gpu_launches": args.steps * len(lins),
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(out), flush=True)
+    ranks.close()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="mnb", choices=["mnb", "reference"])
+    ap.add_argument("--only", default="", choices=["", "decode", "lmhead", "gemm-layer"],
+                    help="profiling modes: run one part only and print no JSON line")
+    args = ap.parse_args()
+    world, rank, local = dist_setup()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    run_gpu(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -164,7 +164,7 @@ __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sy
 
 struct WSlot {
     uint4 p0, p1;       // k 0..31 and 32..63 of the stage
-    uint32_t s0, s1;    // raw scales of the (up to) two blocks
+    uint32_t s0, s1;    // fp16 bits of the scales of the (up to) two blocks
     uint32_t z0, z1;    // zero points
 };
 
@@ -186,9 +186,10 @@ __device__ __forceinline__ WSlot load_wslot(const GemmParams &p, int n, int it, 
         w.s0 = __ldg(s + b0);
         w.s1 = __ldg(s + b1);
     } else {
+        // fp32 scales: the tensor cores take fp16 operands, so round the scale once here
         const float *s = reinterpret_cast<const float *>(p.scales) + (int64_t)n * p.nb;
-        w.s0 = __float_as_uint(__ldg(s + b0));
-        w.s1 = __float_as_uint(__ldg(s + b1));
+        w.s0 = __half_as_ushort(__float2half_rn(__ldg(s + b0)));
+        w.s1 = __half_as_ushort(__float2half_rn(__ldg(s + b1)));
     }
     if (p.zp) {
         const uint8_t *z = p.zp + (int64_t)n * p.zpb;
@@ -201,11 +202,10 @@ __device__ __forceinline__ WSlot load_wslot(const GemmParams &p, int n, int it, 
 
 // 32 nibbles -> 32 fp16 = fp16_rn((q - zp) * s) in natural k order, written as
 // four 16-byte chunks (k 8j..8j+7) of the swizzled row.
-__device__ __forceinline__ void dq_store_half_row(const uint4 &p, uint32_t sraw, uint32_t z, int scale_f16,
-                                                  uint32_t row_addr, int r7, int j0) {
+__device__ __forceinline__ void dq_store_half_row(const uint4 &p, uint32_t s16, uint32_t z, uint32_t row_addr,
+                                                  int r7, int j0) {
     const half2 sixteenth = __floats2half2_rn(0.0625f, 0.0625f);
-    __half sh = scale_f16 ? __ushort_as_half((unsigned short)sraw) : __float2half_rn(__uint_as_float(sraw));
-    const half2 s2 = __halves2half2(sh, sh);
+    const half2 s2 = u32_as_h2(s16 | (s16 << 16));
     const uint32_t Z = 0x64006400u | (z * 0x00010001u);
     const uint32_t Zhi = 0xD400D400u + (z * 0x00100010u);
     const uint32_t words[4] = {p.x, p.y, p.z, p.w};
@@ -343,8 +343,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const WSlot cur = ring[i];
                         ring[i] = load_wslot(p, n, it + kWRing, nk);
                         const uint32_t row_addr = base + (uint32_t)s * stage_bytes + (uint32_t)r * 128;
-                        dq_store_half_row(cur.p0, cur.s0, cur.z0, p.scale_f16, row_addr, r7, 0);
-                        dq_store_half_row(cur.p1, cur.s1, cur.z1, p.scale_f16, row_addr, r7, 4);
+                        dq_store_half_row(cur.p0, cur.s0, cur.z0, row_addr, r7, 0);
+                        dq_store_half_row(cur.p1, cur.s1, cur.z1, row_addr, r7, 4);
                         fence_proxy_async_smem();
                         mbar_arrive(full_w(s));
                     }

@@ -59,8 +59,20 @@ class Pass:
     def __init__(self, linears, M, kind="gemv", act_dtype=torch.float16, pdl=True, embed=None):
         self.linears, self.M, self.kind, self.pdl = list(linears), M, kind, pdl
         dev = self.linears[0].packed.device
-        self.X = [torch.zeros((M, l.K), dtype=act_dtype, device=dev) for l in self.linears]
-        self.Y = [torch.zeros((M, l.N), dtype=act_dtype, device=dev) for l in self.linears]
+        # one flat buffer each for all inputs and all outputs (views per linear,
+        # 16-byte aligned), so a step's inputs and outputs move in one copy each
+        xs = [M * l.K for l in self.linears]
+        ys = [M * l.N for l in self.linears]
+        self.x_flat = torch.zeros((sum(xs),), dtype=act_dtype, device=dev)
+        self.y_flat = torch.zeros((sum(ys),), dtype=act_dtype, device=dev)
+        self.X, self.Y = [], []
+        ox = oy = 0
+        for l, nx, ny in zip(self.linears, xs, ys):
+            self.X.append(self.x_flat[ox:ox + nx].view(M, l.K))
+            self.Y.append(self.y_flat[oy:oy + ny].view(M, l.N))
+            ox, oy = ox + nx, oy + ny
+        for t in self.X + self.Y:
+            assert t.data_ptr() % 16 == 0
         self.embed = embed   # (table, row_scales, ids[M], out[M, D]) or None
         self.graph = None
 
