@@ -316,6 +316,7 @@ def profile_part(args, dev, ranks):
     p = Pass(lins, M, kind, torch.float16, pdl=False)
     fill(p, cfg["seed"])
     torch.cuda.synchronize()
+    torch.cuda.empty_cache()    # keep only the live buffers on the device
     for _ in range(args.warmup):
         p.run()
     torch.cuda.synchronize()
@@ -361,6 +362,22 @@ def run_gpu(args, world, rank, local):
     per_launch_bytes = wbytes / len(lins)
     per_launch_us = ms * 1000.0 / len(lins)
     achieved = per_launch_bytes / (per_launch_us * 1e-6) / 1e9
+
+    # the same step with the weights of projections that share an input stored
+    # row-concatenated (q|k|v, gate|up): 113 launches, identical bytes and math
+    from int4_block_quantized_matmulnbits_b200.step import fuse_decoder
+
+    flins = fuse_decoder(lins)
+    fdec = Pass(flins, 1, "gemv", torch.float16, pdl=True)
+    fill(fdec, cfg["seed"])
+    fdec.capture()
+    with ClockSampler(local) as fclk:
+        f_ms = timed_replays(fdec, args.steps, args.warmup, ranks, "decode_fused") / args.steps
+    assert fdec.weight_bytes == wbytes
+    fused = {"launches_per_step": len(flins), "us_per_step": round(f_ms * 1000, 2),
+             "weight_gbs": round(world * wbytes / (f_ms * 1e-3) / 1e9, 1),
+             "frac_hbm": round(wbytes / (f_ms * 1e-3) / 1e9 / hbm, 4), "clocks": fclk.summary()}
+    del fdec
 
     # lm_head alone: one 180 MB launch, the kernel without launch gaps
     lm = lins[-1]
@@ -432,6 +449,7 @@ def run_gpu(args, world, rank, local):
                          "us_per_launch": round(per_launch_us, 3)},
             "lm_head_alone": {"bytes": lm.nbytes, "us": round(lm_ms * 1000, 2), "gbs": round(lm_gbs, 1),
                               "frac_hbm": round(lm_gbs / hbm, 4)},
+            "decode_fused_qkv_gateup": fused,
             "decode_by_M": by_m,
             "prefill": prefill,
             "roofline_prefill": {"bound": "tensor", "kernel": "gemm_kernel", "M": 1024,

@@ -1,0 +1,556 @@
+// gemv_tc.cu -- decode-shaped MatMulNBits with fp16 activations (1 <= M <= 16):
+// Y[M][N] = X[M][K] . dequant(W)^T, the per-token decoder step of
+// "Qwen3-ASR-0.6B -- ONNX for the browser" ("Graph contracts": decoder_step)
+// and of "Mega-ASR -- INT4 ONNX (GPTQ-calibrated)" (decoder_step_int4).
+//
+// HBM-bound: every weight byte is read once, so the kernel is built to keep the
+// memory system full while the SM does the int4 -> fp16 work.
+//   * Weights move by TMA.  A 2D tensor map views the packed bytes as
+//     [N rows][K/2 bytes]; one box is 16 rows x 128 bytes (256 k), landing in
+//     shared memory with the 128-byte swizzle.  Each warp owns a ring of
+//     kDepth boxes with one mbarrier each; lane 0 keeps kDepth boxes in
+//     flight, so a whole SM holds tens of KB of outstanding weight traffic
+//     with a handful of instructions and no registers.
+//   * The first boxes are requested BEFORE griddepcontrol.wait: under
+//     programmatic dependent launch the weight stream of this kernel starts
+//     while the previous kernel is still finishing.  X is read after the wait.
+//   * Thread (g = lane/4, c = lane%4) owns rows g and g+8 of the warp's 16-row
+//     tile and, in every box, the 16-byte chunks 2c and 2c+1 of both rows; the
+//     swizzle makes these shared-memory reads conflict-free.
+//   * Unpack + dequant in registers: (nibble | 0x6400) is the fp16 1024+q
+//     exactly; subtracting 1024+zp leaves q-zp exactly; one multiply gives
+//     fp16_rn((q - zp) * scale).  High nibbles come out as 1024+16q and are
+//     kept at 16x scale (exact), the matching activations are staged as x/16
+//     (exact), so every nibble costs one subtract and one multiply.
+//   * mma.sync m16n8k16 (fp32 accumulation) takes the 16 rows as M and the
+//     tokens as N, so the multiply-adds leave the CUDA cores to the unpack.
+//   * Persistent CTAs of 8 warps, two per SM.  When tiles alone cannot occupy
+//     the SMs, K is split over W warps of a CTA (shared-memory reduction) and
+//     over a cluster of S CTAs (distributed shared memory): no global scratch.
+// Every mbarrier wait is bounded in time; past the limit the kernel records the
+// failure in a device status word, drains its copies and exits.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace mnb {
+
+namespace {
+
+__device__ unsigned g_gemv_status = 0;
+
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kRows = 16;
+constexpr int kBoxK = 256;                 // k per TMA box
+constexpr int kBoxBytes = kRows * 128;     // 16 rows x 128 packed bytes
+constexpr int kDepth = 4;                  // boxes in flight per warp
+constexpr int kMaxCluster = 8;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+struct TcParams {
+    const void *X;
+    const void *scales;
+    const uint8_t *zp;
+    __half *Y;
+    int M, N, K;
+    int bs_shift, nb, zpb, scale_f16, scale_pair;
+    int S;            // CTAs per cluster (K split across CTAs)
+    int W;            // warps per tile inside a CTA (K split across warps)
+    int nbx_w;        // boxes in one warp's K slice
+    int kcta;         // k covered by one CTA = W * nbx_w * kBoxK
+    int rounds;       // tile rounds per CTA (split mode)
+    int nclusters;    // gridDim.x / S
+    int xs_stride;    // bytes per token row of staged X
+    int ntiles;       // ceil(N / 16)
+    int independent;  // W == 1 && S == 1: each warp walks tiles on its own
+};
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float ld_dsmem_f32(const float *local, uint32_t rank) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void mma16816(float d[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Bounded wait on a warp-private mbarrier.  After the first timeout (*dead set)
+// it returns at once, so the warp runs to the end without waiting again.
+__device__ __forceinline__ void box_wait(uint32_t bar, uint32_t parity, bool &dead) {
+    if (dead || mbar_try_wait(bar, parity))
+        return;
+    const unsigned long long t0 = globaltimer();
+    for (uint32_t i = 1;; i++) {
+        if (mbar_try_wait(bar, parity))
+            return;
+        if ((i & 255) == 0 && globaltimer() - t0 > kWaitLimitNs) {
+            dead = true;
+            atomicOr(&g_gemv_status, 1u);
+            return;
+        }
+    }
+}
+
+// Scales (as fp16 bits, replicated into a half2) and zero points of the two
+// chunks a thread dequantizes in one box, for one row.
+struct ChunkParams {
+    uint32_t s2[2];    // half2 scale of chunk 2c and chunk 2c+1
+    uint32_t z[2];     // zero point of each chunk
+};
+
+__device__ __forceinline__ uint32_t h16_of_scale(const TcParams &p, int64_t idx) {
+    if (p.scale_f16)
+        return __ldg(reinterpret_cast<const unsigned short *>(p.scales) + idx);
+    return __half_as_ushort(__float2half_rn(__ldg(reinterpret_cast<const float *>(p.scales) + idx)));
+}
+
+__device__ __forceinline__ ChunkParams load_params(const TcParams &p, int n, int k0) {
+    ChunkParams q;
+    q.s2[0] = q.s2[1] = 0;
+    q.z[0] = q.z[1] = 8;
+    if (n >= p.N || k0 >= p.K)
+        return q;
+    const int b0 = k0 >> (5 + p.bs_shift);
+    const int64_t row = (int64_t)n * p.nb;
+    uint32_t h0, h1;
+    if (p.bs_shift == 0) {
+        // block 32: chunks 2c and 2c+1 are blocks b0, b0+1 (b0 even)
+        if (p.scale_pair) {
+            const uint32_t pair = __ldg(reinterpret_cast<const unsigned int *>(
+                reinterpret_cast<const unsigned short *>(p.scales) + row + b0));
+            h0 = pair & 0xFFFFu;
+            h1 = pair >> 16;
+        } else {
+            h0 = h16_of_scale(p, row + b0);
+            h1 = (k0 + 32 < p.K) ? h16_of_scale(p, row + b0 + 1) : 0u;
+        }
+        if (p.zp) {
+            const uint32_t zb = __ldg(p.zp + (int64_t)n * p.zpb + (b0 >> 1));
+            q.z[0] = zb & 15u;
+            q.z[1] = zb >> 4;
+        }
+    } else {
+        // block 64: both chunks lie in block b0
+        h0 = h1 = h16_of_scale(p, row + b0);
+        if (p.zp) {
+            const uint32_t zb = __ldg(p.zp + (int64_t)n * p.zpb + (b0 >> 1));
+            q.z[0] = q.z[1] = (b0 & 1) ? (zb >> 4) : (zb & 15u);
+        }
+    }
+    q.s2[0] = h0 | (h0 << 16);
+    q.s2[1] = h1 | (h1 << 16);
+    return q;
+}
+
+// 16 packed bytes (32 nibbles) -> 16 half2 A-operand words.  Word w gives
+// (e0,e4), 16*(e1,e5), (e2,e6), 16*(e3,e7) as fp16_rn((q - zp) * s) (x16 exact).
+__device__ __forceinline__ void dequant16(const uint4 &v, uint32_t z, uint32_t s2, uint32_t out[16]) {
+    const uint32_t Z = 0x64006400u | (z * 0x00010001u);      // 1024 + zp
+    const uint32_t Zhi = 0x64006400u | (z * 0x00100010u);    // 1024 + 16 zp
+    const half2 s = u32_as_h2(s2);
+    const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const uint32_t w = words[i], w8 = w >> 8;
+        out[4 * i + 0] = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(w, 0x000F000Fu, 0x64006400u)), u32_as_h2(Z)), s));
+        out[4 * i + 1] = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(w, 0x00F000F0u, 0x64006400u)), u32_as_h2(Zhi)), s));
+        out[4 * i + 2] = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(w8, 0x000F000Fu, 0x64006400u)), u32_as_h2(Z)), s));
+        out[4 * i + 3] = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(w8, 0x00F000F0u, 0x64006400u)), u32_as_h2(Zhi)), s));
+    }
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_constant__ CUtensorMap wmap,
+                                                              const TcParams p) {
+    constexpr int MP = 8 * NT;
+    extern __shared__ unsigned char smem_raw[];
+    const int tid = threadIdx.x;
+    const int lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, c = lane & 3;
+    const int W = p.W, TPC = kWarps / p.W;
+    const int slot = warp / W, wk = warp - slot * W;
+    const int rank = (p.S > 1) ? (int)cluster_ctarank() : 0;
+    const int cluster = blockIdx.x / p.S;
+    const int kcta0 = rank * p.kcta;
+    const int kw = kcta0 + wk * p.nbx_w * kBoxK;   // first k of this warp's slice
+
+    // shared memory: [kWarps][kDepth] boxes (1024-aligned) | X | red | part | barriers
+    const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    unsigned char *bp = smem_raw + (base - smem_u32(smem_raw));
+    unsigned char *xs = bp + kWarps * kDepth * kBoxBytes;
+    float *red = reinterpret_cast<float *>(xs + p.M * p.xs_stride);
+    float *part = red + kWarps * kRows * MP;
+    const uint32_t bars = smem_u32(part + kWarps * kRows * MP);
+    const uint32_t my_boxes = base + (uint32_t)(warp * kDepth * kBoxBytes);
+    const unsigned char *my_boxes_ptr = bp + warp * kDepth * kBoxBytes;
+    const uint32_t my_bars = bars + (uint32_t)(warp * kDepth * 8);
+
+    // this warp's sequence of tiles
+    int first_tile, tile_stride, units;
+    if (p.independent) {
+        const int gw = blockIdx.x * kWarps + warp, G = gridDim.x * kWarps;
+        first_tile = gw;
+        tile_stride = G;
+        units = (p.ntiles > gw) ? (p.ntiles - gw + G - 1) / G : 0;
+    } else {
+        first_tile = cluster * TPC + slot;
+        tile_stride = p.nclusters * TPC;
+        units = p.rounds;
+    }
+    const int total = units * p.nbx_w;
+
+    // ---- weights first: they do not depend on the previous kernel
+    int is_tile = first_tile, is_j = 0, is_pos = 0;   // TMA issue cursor (lane 0)
+    if (lane == 0) {
+        for (int d = 0; d < kDepth; d++)
+            mbar_init(my_bars + 8 * d, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        for (int d = 0; d < kDepth && is_pos < total; d++) {
+            mbar_expect_tx(my_bars + 8 * d, kBoxBytes);
+            tma_load_2d(my_boxes + d * kBoxBytes, &wmap, my_bars + 8 * d, (kw + is_j * kBoxK) / 2, is_tile * kRows);
+            ++is_pos;
+            if (++is_j == p.nbx_w) { is_j = 0; is_tile += tile_stride; }
+        }
+    }
+    __syncwarp();
+    pdl_launch_dependents();
+    pdl_wait();
+
+    // ---- stage X[0:M, kcta0 : kcta0 + kcta): per 256-k box qb, unit (h, w, c)
+    // holds k = qb*256 + (2c+h)*32 + 8w .. +7 as (x0,x4) (x1,x5)/16 (x2,x6) (x3,x7)/16
+    {
+        const __half *X = reinterpret_cast<const __half *>(p.X);
+        const int per_tok = (p.kcta / kBoxK) * 32;
+        const half2 sixteenth = __floats2half2_rn(0.0625f, 0.0625f);
+        for (int u = tid; u < p.M * per_tok; u += kThreads) {
+            const int m = u / per_tok;
+            const int r = u - m * per_tok;
+            const int qb = r >> 5, rem = r & 31;
+            const int h = rem >> 4, w = (rem >> 2) & 3, cc = rem & 3;
+            const int k = kcta0 + qb * kBoxK + (2 * cc + h) * 32 + w * 8;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (k < p.K)
+                v = ldg_v4(X + (int64_t)m * p.K + k);
+            uint4 o;
+            o.x = __byte_perm(v.x, v.z, 0x5410);
+            o.y = h2_as_u32(__hmul2(u32_as_h2(__byte_perm(v.x, v.z, 0x7632)), sixteenth));
+            o.z = __byte_perm(v.y, v.w, 0x5410);
+            o.w = h2_as_u32(__hmul2(u32_as_h2(__byte_perm(v.y, v.w, 0x7632)), sixteenth));
+            *reinterpret_cast<uint4 *>(xs + m * p.xs_stride + r * 16) = o;
+        }
+    }
+    __syncthreads();
+
+    float acc[NT][4];
+#pragma unroll
+    for (int t = 0; t < NT; t++)
+#pragma unroll
+        for (int e = 0; e < 4; e++) acc[t][e] = 0.f;
+
+    bool dead = false;
+    int tile = first_tile, j = 0, r = 0;
+    // scales / zero points one box ahead
+    ChunkParams pa = load_params(p, tile * kRows + g, kw + c * 64);
+    ChunkParams pb = load_params(p, tile * kRows + g + 8, kw + c * 64);
+    for (int pos = 0; pos < total; pos++) {
+        // the next box's (tile, j), for the parameter prefetch
+        int ntile = tile, nj = j + 1;
+        if (nj == p.nbx_w) { nj = 0; ntile += tile_stride; }
+        const bool more = pos + 1 < total;
+        ChunkParams na = pa, nbp = pb;
+        if (more) {
+            na = load_params(p, ntile * kRows + g, kw + nj * kBoxK + c * 64);
+            nbp = load_params(p, ntile * kRows + g + 8, kw + nj * kBoxK + c * 64);
+        }
+
+        const int d = pos % kDepth;
+        box_wait(my_bars + 8 * d, (uint32_t)((pos / kDepth) & 1), dead);
+        const unsigned char *box = my_boxes_ptr + d * kBoxBytes;
+        const int qb = (wk * p.nbx_w + j);          // box index inside the CTA's X range
+#pragma unroll
+        for (int h = 0; h < 2; h++) {
+            const int chunk = 2 * c + h;
+            const uint4 va = *reinterpret_cast<const uint4 *>(box + g * 128 + ((chunk ^ g) << 4));
+            const uint4 vb = *reinterpret_cast<const uint4 *>(box + (g + 8) * 128 + ((chunk ^ g) << 4));
+            uint32_t wa[16], wb[16];
+            dequant16(va, pa.z[h], pa.s2[h], wa);
+            dequant16(vb, pb.z[h], pb.s2[h], wb);
+#pragma unroll
+            for (int t = 0; t < NT; t++) {
+                const int tok = g + 8 * t;
+                uint32_t xb[16];
+                if (tok < p.M) {
+                    const unsigned char *xa = xs + tok * p.xs_stride + qb * 512 + h * 256 + c * 16;
+#pragma unroll
+                    for (int w = 0; w < 4; w++) {
+                        const uint4 v = *reinterpret_cast<const uint4 *>(xa + w * 64);
+                        xb[4 * w + 0] = v.x; xb[4 * w + 1] = v.y;
+                        xb[4 * w + 2] = v.z; xb[4 * w + 3] = v.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 16; e++) xb[e] = 0u;
+                }
+#pragma unroll
+                for (int q = 0; q < 8; q++)
+                    mma16816(acc[t], wa[2 * q], wb[2 * q], wa[2 * q + 1], wb[2 * q + 1], xb[2 * q], xb[2 * q + 1]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0 && is_pos < total) {
+            // box d is free again: refill it with the box kDepth positions ahead
+            fence_proxy_async_smem();
+            mbar_expect_tx(my_bars + 8 * d, kBoxBytes);
+            tma_load_2d(my_boxes + d * kBoxBytes, &wmap, my_bars + 8 * d, (kw + is_j * kBoxK) / 2, is_tile * kRows);
+            ++is_pos;
+            if (++is_j == p.nbx_w) { is_j = 0; is_tile += tile_stride; }
+        }
+        pa = na;
+        pb = nbp;
+
+        if (nj != 0) {
+            j = nj;
+            continue;
+        }
+        // ---- end of a tile (for every warp of the CTA at once in split mode)
+        const int tile_done = tile;
+        tile = ntile;
+        j = 0;
+        if (p.independent) {
+            const int n0 = tile_done * kRows + g;
+#pragma unroll
+            for (int t = 0; t < NT; t++)
+#pragma unroll
+                for (int e = 0; e < 4; e++) {
+                    const int m = 8 * t + 2 * c + (e & 1);
+                    const int n = n0 + 8 * (e >> 1);
+                    if (m < p.M && n < p.N)
+                        p.Y[(int64_t)m * p.N + n] = __float2half_rn(acc[t][e]);
+                }
+        } else {
+#pragma unroll
+            for (int t = 0; t < NT; t++) {
+                const int m0 = 8 * t + 2 * c;
+                red[(warp * kRows + g) * MP + m0] = acc[t][0];
+                red[(warp * kRows + g) * MP + m0 + 1] = acc[t][1];
+                red[(warp * kRows + g + 8) * MP + m0] = acc[t][2];
+                red[(warp * kRows + g + 8) * MP + m0 + 1] = acc[t][3];
+            }
+            __syncthreads();
+            for (int idx = tid; idx < TPC * kRows * MP; idx += kThreads) {
+                const int sl = idx / (kRows * MP), jj = idx - sl * kRows * MP;
+                float v = 0.f;
+                for (int q = 0; q < W; q++)
+                    v += red[((sl * W + q) * kRows) * MP + jj];
+                part[idx] = v;
+            }
+            if (p.S > 1) cluster_sync(); else __syncthreads();
+            if (rank == 0) {
+                for (int idx = tid; idx < TPC * kRows * MP; idx += kThreads) {
+                    const int sl = idx / (kRows * MP), jj = idx - sl * kRows * MP;
+                    const int row = jj / MP, m = jj - row * MP;
+                    const int n = ((r * p.nclusters + cluster) * TPC + sl) * kRows + row;
+                    if (m >= p.M || n >= p.N)
+                        continue;
+                    float v = part[idx];
+                    for (int q = 1; q < p.S; q++)
+                        v += ld_dsmem_f32(part + idx, (uint32_t)q);
+                    p.Y[(int64_t)m * p.N + n] = __float2half_rn(v);
+                }
+            }
+            if (p.S > 1) cluster_sync(); else __syncthreads();
+        }
+        ++r;
+#pragma unroll
+        for (int t = 0; t < NT; t++)
+#pragma unroll
+            for (int e = 0; e < 4; e++) acc[t][e] = 0.f;
+    }
+
+    // every issued box was waited for above; after a timeout, let the copies
+    // still in flight land before the CTA's shared memory is released
+    if (dead && lane == 0) {
+        for (int q = (total > kDepth ? total - kDepth : 0); q < total; q++) {
+            const uint32_t bar = my_bars + 8 * (q % kDepth);
+            const unsigned long long t0 = globaltimer();
+            while (!mbar_try_wait(bar, (uint32_t)((q / kDepth) & 1)) && globaltimer() - t0 < kWaitLimitNs) {
+            }
+        }
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+int sm_count_tc() {
+    static int count = 0;
+    if (count == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || count <= 0)
+            count = 148;
+    }
+    return count;
+}
+
+template <int NT>
+int launch_tc(const CUtensorMap &map, const TcParams &p, int grid, size_t smem, unsigned flags, cudaStream_t s) {
+    auto fn = gemv_tc_kernel<NT>;
+    static int configured = 0;
+    if ((int)smem > configured) {
+        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess)
+            return fail(MNB_ERR_CUDA, "mnb_gemv: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        configured = (int)smem;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (p.S > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = (unsigned)p.S;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        na++;
+    }
+    if (flags & MNB_FLAG_PDL) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        na++;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, fn, map, p);
+    if (e != cudaSuccess)
+        return fail(MNB_ERR_CUDA, "mnb_gemv: launch: %s", cudaGetErrorString(e));
+    return MNB_OK;
+}
+
+}  // namespace
+
+int launch_gemv_tc(const void *X, const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,
+                   void *Y, int M, int N, int K, int bs, unsigned flags, cudaStream_t s) {
+    EncodeTiledFn encode = encode_fn();
+    if (!encode)
+        return fail(MNB_ERR_CUDA, "mnb_gemv: cuTensorMapEncodeTiled unavailable");
+    const int NT = (M <= 8) ? 1 : 2;
+    const int MP = 8 * NT;
+    const int sms = sm_count_tc();
+
+    TcParams p;
+    p.X = X; p.scales = scales; p.zp = zp; p.Y = reinterpret_cast<__half *>(Y);
+    p.M = M; p.N = N; p.K = K;
+    p.bs_shift = (bs == 64) ? 1 : 0;
+    p.nb = K / bs;
+    p.zpb = (p.nb + 1) / 2;
+    p.scale_f16 = scale_f16;
+    p.scale_pair = (scale_f16 && bs == 32 && (p.nb % 2) == 0 && (reinterpret_cast<uintptr_t>(scales) % 4) == 0);
+    p.ntiles = (N + kRows - 1) / kRows;
+
+    // K slices: W warps x S CTAs per tile, enough for ~16 warps on every SM
+    const int nbx_all = (K + kBoxK - 1) / kBoxK;
+    int slices = (sms * 2 * kWarps + p.ntiles - 1) / p.ntiles;
+    if (slices > nbx_all) slices = nbx_all;
+    if (slices > kWarps * kMaxCluster) slices = kWarps * kMaxCluster;
+    if (slices < 1) slices = 1;
+    int W = 1;
+    while (W * 2 <= kWarps && W * 2 <= slices) W *= 2;
+    int S = (slices + W - 1) / W;
+    if (S > kMaxCluster) S = kMaxCluster;
+    size_t smem = 0;
+    for (;; S++) {
+        const int nbx_w = (nbx_all + W * S - 1) / (W * S);
+        p.S = S; p.W = W; p.nbx_w = nbx_w;
+        p.kcta = W * nbx_w * kBoxK;
+        p.xs_stride = (p.kcta / kBoxK) * 512 + 64;
+        smem = 1024 + (size_t)kWarps * kDepth * kBoxBytes + (size_t)M * p.xs_stride +
+               (size_t)2 * kWarps * kRows * MP * 4 + (size_t)kWarps * kDepth * 8;
+        if (smem <= 200 * 1024 || S >= kMaxCluster)
+            break;
+    }
+    if (smem > 220 * 1024)
+        return fail(MNB_ERR_SHAPE, "mnb_gemv: K=%d too large for M=%d", K, M);
+    p.independent = (p.W == 1 && p.S == 1);
+    const int per_sm = (smem <= 110 * 1024) ? 2 : 1;
+    int grid;
+    if (p.independent) {
+        const int groups = (p.ntiles + kWarps - 1) / kWarps;
+        grid = groups < sms * per_sm ? groups : sms * per_sm;
+        p.rounds = 0;
+        p.nclusters = grid;
+    } else {
+        const int tpc = kWarps / p.W;
+        const int groups = (p.ntiles + tpc - 1) / tpc;
+        int max_clusters = sms * per_sm / p.S;
+        if (max_clusters < 1) max_clusters = 1;
+        p.rounds = (groups + max_clusters - 1) / max_clusters;
+        p.nclusters = (groups + p.rounds - 1) / p.rounds;
+        grid = p.nclusters * p.S;
+    }
+
+    CUtensorMap map;
+    const cuuint64_t gdim[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N};
+    const cuuint64_t gstride[1] = {(cuuint64_t)(K / 2)};
+    const cuuint32_t box[2] = {128, (cuuint32_t)kRows};
+    const cuuint32_t estride[2] = {1, 1};
+    CUresult cr = encode(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), gdim, gstride, box,
+                         estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS)
+        return fail(MNB_ERR_CUDA, "mnb_gemv: cuTensorMapEncodeTiled failed (%d)", (int)cr);
+    if (NT == 1)
+        return launch_tc<1>(map, p, grid, smem, flags, s);
+    return launch_tc<2>(map, p, grid, smem, flags, s);
+}
+
+int read_gemv_status(unsigned *out, int clear) {
+    unsigned v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_gemv_status, sizeof(unsigned));
+    if (e == cudaSuccess && clear) {
+        const unsigned zero = 0;
+        e = cudaMemcpyToSymbol(g_gemv_status, &zero, sizeof(unsigned));
+    }
+    if (e != cudaSuccess)
+        return fail(MNB_ERR_CUDA, "mnb_device_status: %s", cudaGetErrorString(e));
+    *out |= v;
+    return MNB_OK;
+}
+
+}  // namespace mnb

@@ -17,6 +17,9 @@ int launch_gemv(const void *X, int act_f16, const uint8_t *packed, const void *s
                 int scale_f16, const uint8_t *zp, void *Y, int M, int N, int K, int bs,
                 unsigned flags, cudaStream_t s);
 
+int launch_gemv_tc(const void *X, const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,
+                   void *Y, int M, int N, int K, int bs, unsigned flags, cudaStream_t s);
+
 int launch_gemm(const void *X, const uint8_t *packed, const void *scales, int scale_f16,
                 const uint8_t *zp, void *Y, int M, int N, int K, int bs, unsigned flags,
                 cudaStream_t s);
@@ -26,5 +29,6 @@ int launch_embed_gather(const int8_t *table, const float *row_scales, int64_t V,
                         cudaStream_t s);
 
 int read_device_status(unsigned *out, int clear);
+int read_gemv_status(unsigned *out, int clear);   // ORs the decode kernel's word into *out
 
 }  // namespace mnb

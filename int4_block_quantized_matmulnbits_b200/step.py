@@ -47,6 +47,41 @@ class QLinear:
         mnb_gemm(X, self.packed, self.scales, self.zp, Y, X.shape[0], self.N, self.K, self.bs, flags, stream)
 
 
+def concat_linears(parts, name=""):
+    """One QLinear whose rows are the rows of `parts` in order.
+
+    Projections that read the same input (q, k, v; gate, up) are one
+    MatMulNBits over their row-concatenated weights: the packed rows, scales and
+    zero points are per row, so concatenation changes no stored value, and the
+    outputs come out concatenated in the same order."""
+    K, bs, has_zp = parts[0].K, parts[0].bs, parts[0].has_zp
+    assert all(p.K == K and p.bs == bs and p.has_zp == has_zp for p in parts)
+    N = sum(p.N for p in parts)
+    q = QLinear(N, K, bs, has_zp, parts[0].scales.dtype, parts[0].packed.device, name)
+    torch.cat([p.packed for p in parts], dim=0, out=q.packed)
+    torch.cat([p.scales for p in parts], dim=0, out=q.scales)
+    if has_zp:
+        torch.cat([p.zp for p in parts], dim=0, out=q.zp)
+    q.parts = [(p.name, p.N) for p in parts]
+    return q
+
+
+def fuse_decoder(linears):
+    """Per layer [q, k, v, o, gate, up, down] -> [qkv, o, gate_up, down]; others kept."""
+    out, i = [], 0
+    while i < len(linears):
+        names = [l.name.rstrip("0123456789") for l in linears[i:i + 7]]
+        if names == ["q", "k", "v", "o", "gate", "up", "down"]:
+            L = linears[i:i + 7]
+            layer = L[0].name[1:]
+            out += [concat_linears(L[0:3], f"qkv{layer}"), L[3], concat_linears(L[4:6], f"gate_up{layer}"), L[6]]
+            i += 7
+        else:
+            out.append(linears[i])
+            i += 1
+    return out
+
+
 class Pass:
     """A chain of MatMulNBits calls with one X / Y buffer pair per linear.
 

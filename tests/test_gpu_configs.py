@@ -116,6 +116,29 @@ def test_qwen3_1p7b_decode_step(step_mod, cuda_dev, M):
     check_pass(cfg, lins, samples, p, "f16")
 
 
+@pytest.mark.parametrize("M", [1, 16])
+def test_qwen3_1p7b_decode_step_fused_layout(step_mod, cuda_dev, M):
+    # q|k|v and gate|up stored row-concatenated: one GEMV per group, same outputs
+    cfg, lins, samples = model(step_mod, "qwen3_1p7b_decode", 48, full_layers=(27,))
+    fused = step_mod.fuse_decoder(lins)
+    assert len(fused) == 28 * 4 + 1
+    p = step_mod.Pass(fused, M, "gemv", torch.float16)
+    _fill_inputs(p, cfg["seed"] + M, torch.float16)
+    _run_graph(p)
+
+    class View:   # per-projection views of the fused pass, in the original order
+        X, Y = [], []
+
+    v = View()
+    for f, x, y in zip(fused, p.X, p.Y):
+        off = 0
+        for _, n in getattr(f, "parts", [(f.name, f.N)]):
+            v.X.append(x)
+            v.Y.append(y[:, off:off + n])
+            off += n
+    check_pass(cfg, lins, samples, v, "f16")
+
+
 @pytest.mark.parametrize("M", [64, 256, 420, 1024])
 def test_qwen3_1p7b_prefill(step_mod, cuda_dev, M):
     cfg, lins, samples = model(step_mod, "qwen3_1p7b_prefill", 24)
