@@ -44,8 +44,7 @@ __device__ __forceinline__ uint4 ldg_v4(const void *p) {
     uint4 r;
     asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p)
-                 : "memory");
+                 : "l"(p));
     return r;
 }
 

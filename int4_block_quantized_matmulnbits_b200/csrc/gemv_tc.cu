@@ -19,9 +19,12 @@
 //     swizzle makes these shared-memory reads conflict-free.
 //   * Unpack + dequant in registers: (nibble | 0x6400) is the fp16 1024+q
 //     exactly; subtracting 1024+zp leaves q-zp exactly; one multiply gives
-//     fp16_rn((q - zp) * scale).  High nibbles come out as 1024+16q and are
-//     kept at 16x scale (exact), the matching activations are staged as x/16
-//     (exact), so every nibble costs one subtract and one multiply.
+//     fp16_rn((q - zp) * scale), the same value the dequantizer writes.  High
+//     nibbles come out as 1024+16q and stay at 16x scale (exact); the
+//     activations they meet are staged as x/16 (exact).  So 8 weights cost one
+//     shift, four LOP3, four HSUB2 and four HMUL2.
+//   * The hot loop is compiled per configuration (block size, zero points,
+//     scale type) and carries no runtime branches.
 //   * mma.sync m16n8k16 (fp32 accumulation) takes the 16 rows as M and the
 //     tokens as N, so the multiply-adds leave the CUDA cores to the unpack.
 //   * Persistent CTAs of 8 warps, two per SM.  When tiles alone cannot occupy
@@ -110,75 +113,108 @@ __device__ __forceinline__ void box_wait(uint32_t bar, uint32_t parity, bool &de
     }
 }
 
-// Scales (as fp16 bits, replicated into a half2) and zero points of the two
-// chunks a thread dequantizes in one box, for one row.
+// Scale (fp16 bits) and zero point of the two chunks (2c, 2c+1) a thread
+// dequantizes in one box, for one row.
 struct ChunkParams {
-    uint32_t s2[2];    // half2 scale of chunk 2c and chunk 2c+1
-    uint32_t z[2];     // zero point of each chunk
+    uint32_t s[2];
+    uint32_t z[2];
 };
 
-__device__ __forceinline__ uint32_t h16_of_scale(const TcParams &p, int64_t idx) {
+// Where a thread's scales and zero points of the current tile live; moving to
+// the next box is a pointer increment.
+struct ParamCursor {
+    const uint8_t *s;     // scale of the thread's first block in this box (row g)
+    const uint8_t *z;     // its zero-point byte (row g)
+    int k0;               // k of the thread's first chunk in this box
+    bool ok0, ok1;        // rows g, g+8 inside N
+};
+
+template <class C>
+__device__ __forceinline__ void param_tile(const TcParams &p, ParamCursor &q, int tile, int g, int kfirst) {
+    const int n = tile * kRows + g;
+    const int b0 = kfirst >> (C::bs64 ? 6 : 5);
+    q.k0 = kfirst;
+    q.ok0 = n < p.N;
+    q.ok1 = n + 8 < p.N;
+    q.s = reinterpret_cast<const uint8_t *>(p.scales) + ((int64_t)n * p.nb + b0) * ((C::smode == 0) ? 2 : (p.scale_f16 ? 2 : 4));
+    q.z = C::zp ? p.zp + (int64_t)n * p.zpb + (b0 >> 1) : nullptr;
+}
+
+// Configuration of the hot loop, fixed at compile time so that it carries no
+// runtime branches: block size 64?  zero points present?  SMODE 0 = fp16 scales
+// read as aligned pairs (block 32) or singly (block 64); SMODE 1 = anything else
+// (fp32 scales, or fp16 scales an aligned pair load cannot serve).
+template <bool BS64, bool ZP, int SMODE>
+struct Cfg {
+    static constexpr bool bs64 = BS64, zp = ZP;
+    static constexpr int smode = SMODE;
+};
+
+__device__ __forceinline__ uint32_t h16_at(const TcParams &p, const uint8_t *ptr) {
     if (p.scale_f16)
-        return __ldg(reinterpret_cast<const unsigned short *>(p.scales) + idx);
-    return __half_as_ushort(__float2half_rn(__ldg(reinterpret_cast<const float *>(p.scales) + idx)));
+        return __ldg(reinterpret_cast<const unsigned short *>(ptr));
+    return __half_as_ushort(__float2half_rn(__ldg(reinterpret_cast<const float *>(ptr))));
 }
 
-__device__ __forceinline__ ChunkParams load_params(const TcParams &p, int n, int k0) {
-    ChunkParams q;
-    q.s2[0] = q.s2[1] = 0;
-    q.z[0] = q.z[1] = 8;
-    if (n >= p.N || k0 >= p.K)
-        return q;
-    const int b0 = k0 >> (5 + p.bs_shift);
-    const int64_t row = (int64_t)n * p.nb;
-    uint32_t h0, h1;
-    if (p.bs_shift == 0) {
-        // block 32: chunks 2c and 2c+1 are blocks b0, b0+1 (b0 even)
-        if (p.scale_pair) {
-            const uint32_t pair = __ldg(reinterpret_cast<const unsigned int *>(
-                reinterpret_cast<const unsigned short *>(p.scales) + row + b0));
-            h0 = pair & 0xFFFFu;
-            h1 = pair >> 16;
+// Parameters of the box at the cursor for row g (r = 0) or g+8 (r = 1).
+template <class C>
+__device__ __forceinline__ ChunkParams params_at(const TcParams &p, const ParamCursor &q, int r) {
+    ChunkParams c;
+    c.s[0] = c.s[1] = 0;
+    c.z[0] = c.z[1] = 8;
+    if (!(r ? q.ok1 : q.ok0) || q.k0 >= p.K)
+        return c;
+    const int ssz = (C::smode == 0) ? 2 : (p.scale_f16 ? 2 : 4);
+    const uint8_t *sp = q.s + (r ? (int64_t)8 * p.nb * ssz : 0);
+    if (!C::bs64) {   // block 32: chunks 2c, 2c+1 are blocks b0, b0+1 (b0 even)
+        if (C::smode == 0) {
+            const uint32_t pair = __ldg(reinterpret_cast<const unsigned int *>(sp));
+            c.s[0] = pair & 0xFFFFu;
+            c.s[1] = pair >> 16;
         } else {
-            h0 = h16_of_scale(p, row + b0);
-            h1 = (k0 + 32 < p.K) ? h16_of_scale(p, row + b0 + 1) : 0u;
+            c.s[0] = h16_at(p, sp);
+            c.s[1] = (q.k0 + 32 < p.K) ? h16_at(p, sp + ssz) : 0u;
         }
-        if (p.zp) {
-            const uint32_t zb = __ldg(p.zp + (int64_t)n * p.zpb + (b0 >> 1));
-            q.z[0] = zb & 15u;
-            q.z[1] = zb >> 4;
+        if (C::zp) {
+            const uint32_t zb = __ldg(q.z + (r ? (int64_t)8 * p.zpb : 0));
+            c.z[0] = zb & 15u;
+            c.z[1] = zb >> 4;
         }
-    } else {
-        // block 64: both chunks lie in block b0
-        h0 = h1 = h16_of_scale(p, row + b0);
-        if (p.zp) {
-            const uint32_t zb = __ldg(p.zp + (int64_t)n * p.zpb + (b0 >> 1));
-            q.z[0] = q.z[1] = (b0 & 1) ? (zb >> 4) : (zb & 15u);
+    } else {          // block 64: both chunks in one block
+        c.s[0] = c.s[1] = (C::smode == 0) ? (uint32_t)__ldg(reinterpret_cast<const unsigned short *>(sp))
+                                          : h16_at(p, sp);
+        if (C::zp) {
+            const uint32_t zb = __ldg(q.z + (r ? (int64_t)8 * p.zpb : 0));
+            c.z[0] = c.z[1] = ((q.k0 >> 6) & 1) ? (zb >> 4) : (zb & 15u);
         }
     }
-    q.s2[0] = h0 | (h0 << 16);
-    q.s2[1] = h1 | (h1 << 16);
-    return q;
+    return c;
 }
 
-// 16 packed bytes (32 nibbles) -> 16 half2 A-operand words.  Word w gives
-// (e0,e4), 16*(e1,e5), (e2,e6), 16*(e3,e7) as fp16_rn((q - zp) * s) (x16 exact).
-__device__ __forceinline__ void dequant16(const uint4 &v, uint32_t z, uint32_t s2, uint32_t out[16]) {
-    const uint32_t Z = 0x64006400u | (z * 0x00010001u);      // 1024 + zp
-    const uint32_t Zhi = 0x64006400u | (z * 0x00100010u);    // 1024 + 16 zp
+template <class C>
+__device__ __forceinline__ void param_next_box(const TcParams &p, ParamCursor &q) {
+    // one box = 256 k = 8 blocks of 32 or 4 of 64
+    constexpr int nblk = C::bs64 ? 4 : 8;
+    q.s += nblk * ((C::smode == 0) ? 2 : (p.scale_f16 ? 2 : 4));
+    if (C::zp) q.z += nblk >> 1;
+    q.k0 += kBoxK;
+}
+
+// One 32-bit word of nibbles (e0..e7) of a row -> the four A-operand half2
+// (e0,e4), 16*(e1,e5), (e2,e6), 16*(e3,e7): (1024 + q) - (1024 + zp) = q - zp
+// exactly, times the scale = fp16_rn((q - zp) * s) (x16 for the high nibbles,
+// exact).
+__device__ __forceinline__ void dq_word(uint32_t w, uint32_t s2, uint32_t Z, uint32_t Zhi, uint32_t &a0,
+                                        uint32_t &a1, uint32_t &a2, uint32_t &a3) {
+    const uint32_t w8 = w >> 8;
     const half2 s = u32_as_h2(s2);
-    const uint32_t words[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; i++) {
-        const uint32_t w = words[i], w8 = w >> 8;
-        out[4 * i + 0] = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(w, 0x000F000Fu, 0x64006400u)), u32_as_h2(Z)), s));
-        out[4 * i + 1] = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(w, 0x00F000F0u, 0x64006400u)), u32_as_h2(Zhi)), s));
-        out[4 * i + 2] = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(w8, 0x000F000Fu, 0x64006400u)), u32_as_h2(Z)), s));
-        out[4 * i + 3] = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(w8, 0x00F000F0u, 0x64006400u)), u32_as_h2(Zhi)), s));
-    }
+    a0 = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(w, 0x000F000Fu, 0x64006400u)), u32_as_h2(Z)), s));
+    a1 = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(w, 0x00F000F0u, 0x64006400u)), u32_as_h2(Zhi)), s));
+    a2 = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(w8, 0x000F000Fu, 0x64006400u)), u32_as_h2(Z)), s));
+    a3 = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(w8, 0x00F000F0u, 0x64006400u)), u32_as_h2(Zhi)), s));
 }
 
-template <int NT>
+template <int NT, class C>
 __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_constant__ CUtensorMap wmap,
                                                               const TcParams p) {
     constexpr int MP = 8 * NT;
@@ -192,19 +228,20 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
     const int cluster = blockIdx.x / p.S;
     const int kcta0 = rank * p.kcta;
     const int kw = kcta0 + wk * p.nbx_w * kBoxK;   // first k of this warp's slice
+    const int nqb = p.kcta / kBoxK;                // boxes in the CTA's X range
 
-    // shared memory: [kWarps][kDepth] boxes (1024-aligned) | X | red | part | barriers
+    // shared memory: boxes (1024-aligned) | X | zero row | red | part | barriers
     const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
     unsigned char *bp = smem_raw + (base - smem_u32(smem_raw));
     unsigned char *xs = bp + kWarps * kDepth * kBoxBytes;
-    float *red = reinterpret_cast<float *>(xs + p.M * p.xs_stride);
+    unsigned char *zrow = xs + p.M * p.xs_stride;   // 512 zero bytes: activations of absent tokens
+    float *red = reinterpret_cast<float *>(zrow + 512);
     float *part = red + kWarps * kRows * MP;
     const uint32_t bars = smem_u32(part + kWarps * kRows * MP);
     const uint32_t my_boxes = base + (uint32_t)(warp * kDepth * kBoxBytes);
     const unsigned char *my_boxes_ptr = bp + warp * kDepth * kBoxBytes;
     const uint32_t my_bars = bars + (uint32_t)(warp * kDepth * 8);
 
-    // this warp's sequence of tiles
     int first_tile, tile_stride, units;
     if (p.independent) {
         const int gw = blockIdx.x * kWarps + warp, G = gridDim.x * kWarps;
@@ -235,84 +272,88 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
     pdl_launch_dependents();
     pdl_wait();
 
-    // ---- stage X[0:M, kcta0 : kcta0 + kcta): per 256-k box qb, unit (h, w, c)
-    // holds k = qb*256 + (2c+h)*32 + 8w .. +7 as (x0,x4) (x1,x5)/16 (x2,x6) (x3,x7)/16
+    // ---- stage X[0:M, kcta0 : kcta0 + kcta).  Box qb, unit (h, w, c) holds
+    // k = qb*256 + (2c+h)*32 + 8w .. +7 as (x0,x4) (x1,x5)/16 (x2,x6) (x3,x7)/16;
+    // one thread per 32-k chunk.
     {
         const __half *X = reinterpret_cast<const __half *>(p.X);
-        const int per_tok = (p.kcta / kBoxK) * 32;
         const half2 sixteenth = __floats2half2_rn(0.0625f, 0.0625f);
+        const int per_tok = nqb * 8;   // chunks
         for (int u = tid; u < p.M * per_tok; u += kThreads) {
             const int m = u / per_tok;
             const int r = u - m * per_tok;
-            const int qb = r >> 5, rem = r & 31;
-            const int h = rem >> 4, w = (rem >> 2) & 3, cc = rem & 3;
-            const int k = kcta0 + qb * kBoxK + (2 * cc + h) * 32 + w * 8;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (k < p.K)
-                v = ldg_v4(X + (int64_t)m * p.K + k);
-            uint4 o;
-            o.x = __byte_perm(v.x, v.z, 0x5410);
-            o.y = h2_as_u32(__hmul2(u32_as_h2(__byte_perm(v.x, v.z, 0x7632)), sixteenth));
-            o.z = __byte_perm(v.y, v.w, 0x5410);
-            o.w = h2_as_u32(__hmul2(u32_as_h2(__byte_perm(v.y, v.w, 0x7632)), sixteenth));
-            *reinterpret_cast<uint4 *>(xs + m * p.xs_stride + r * 16) = o;
+            const int qb = r >> 3, chunk = r & 7;
+            const int h = chunk & 1, cc = chunk >> 1;
+            const int k = kcta0 + qb * kBoxK + chunk * 32;
+            uint4 vv[4];
+#pragma unroll
+            for (int w = 0; w < 4; w++)   // all four loads in flight before any use
+                vv[w] = (k < p.K) ? ldg_v4(X + (int64_t)m * p.K + k + 8 * w) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int w = 0; w < 4; w++) {
+                const uint4 v = vv[w];
+                uint4 o;
+                o.x = __byte_perm(v.x, v.z, 0x5410);
+                o.y = h2_as_u32(__hmul2(u32_as_h2(__byte_perm(v.x, v.z, 0x7632)), sixteenth));
+                o.z = __byte_perm(v.y, v.w, 0x5410);
+                o.w = h2_as_u32(__hmul2(u32_as_h2(__byte_perm(v.y, v.w, 0x7632)), sixteenth));
+                *reinterpret_cast<uint4 *>(xs + m * p.xs_stride + qb * 512 + h * 256 + w * 64 + cc * 16) = o;
+            }
         }
+        for (int i = tid; i < 128; i += kThreads)
+            reinterpret_cast<uint32_t *>(zrow)[i] = 0u;
     }
     __syncthreads();
 
-    float acc[NT][4];
+    float acc[NT][2][4];       // two accumulator chains (chunk 2c and 2c+1)
 #pragma unroll
     for (int t = 0; t < NT; t++)
 #pragma unroll
-        for (int e = 0; e < 4; e++) acc[t][e] = 0.f;
+        for (int e = 0; e < 8; e++) acc[t][e >> 2][e & 3] = 0.f;
 
     bool dead = false;
     int tile = first_tile, j = 0, r = 0;
-    // scales / zero points one box ahead
-    ChunkParams pa = load_params(p, tile * kRows + g, kw + c * 64);
-    ChunkParams pb = load_params(p, tile * kRows + g + 8, kw + c * 64);
+    ParamCursor pc;
+    param_tile<C>(p, pc, tile, g, kw + c * 64);
+    ChunkParams pa = params_at<C>(p, pc, 0), pb = params_at<C>(p, pc, 1);   // one box ahead
     for (int pos = 0; pos < total; pos++) {
-        // the next box's (tile, j), for the parameter prefetch
         int ntile = tile, nj = j + 1;
         if (nj == p.nbx_w) { nj = 0; ntile += tile_stride; }
-        const bool more = pos + 1 < total;
-        ChunkParams na = pa, nbp = pb;
-        if (more) {
-            na = load_params(p, ntile * kRows + g, kw + nj * kBoxK + c * 64);
-            nbp = load_params(p, ntile * kRows + g + 8, kw + nj * kBoxK + c * 64);
+        if (nj == 0) param_tile<C>(p, pc, ntile, g, kw + c * 64); else param_next_box<C>(p, pc);
+        ChunkParams na = pa, nbq = pb;
+        if (pos + 1 < total) {
+            na = params_at<C>(p, pc, 0);
+            nbq = params_at<C>(p, pc, 1);
         }
 
         const int d = pos % kDepth;
         box_wait(my_bars + 8 * d, (uint32_t)((pos / kDepth) & 1), dead);
         const unsigned char *box = my_boxes_ptr + d * kBoxBytes;
-        const int qb = (wk * p.nbx_w + j);          // box index inside the CTA's X range
+        const int qb = wk * p.nbx_w + j;      // box index inside the CTA's X range
 #pragma unroll
         for (int h = 0; h < 2; h++) {
             const int chunk = 2 * c + h;
             const uint4 va = *reinterpret_cast<const uint4 *>(box + g * 128 + ((chunk ^ g) << 4));
             const uint4 vb = *reinterpret_cast<const uint4 *>(box + (g + 8) * 128 + ((chunk ^ g) << 4));
-            uint32_t wa[16], wb[16];
-            dequant16(va, pa.z[h], pa.s2[h], wa);
-            dequant16(vb, pb.z[h], pb.s2[h], wb);
+            const uint32_t sa = pa.s[h] | (pa.s[h] << 16), sb = pb.s[h] | (pb.s[h] << 16);
+            const uint32_t Za = 0x64006400u | (pa.z[h] * 0x00010001u), Zb = 0x64006400u | (pb.z[h] * 0x00010001u);
+            const uint32_t Zha = 0x64006400u | (pa.z[h] * 0x00100010u), Zhb = 0x64006400u | (pb.z[h] * 0x00100010u);
+            const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
+            const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
             for (int t = 0; t < NT; t++) {
                 const int tok = g + 8 * t;
-                uint32_t xb[16];
-                if (tok < p.M) {
-                    const unsigned char *xa = xs + tok * p.xs_stride + qb * 512 + h * 256 + c * 16;
+                const unsigned char *xa = (tok < p.M) ? xs + tok * p.xs_stride + qb * 512 + h * 256 + c * 16
+                                                      : zrow + h * 256 + c * 16;
 #pragma unroll
-                    for (int w = 0; w < 4; w++) {
-                        const uint4 v = *reinterpret_cast<const uint4 *>(xa + w * 64);
-                        xb[4 * w + 0] = v.x; xb[4 * w + 1] = v.y;
-                        xb[4 * w + 2] = v.z; xb[4 * w + 3] = v.w;
-                    }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 16; e++) xb[e] = 0u;
+                for (int w = 0; w < 4; w++) {
+                    const uint4 xv = *reinterpret_cast<const uint4 *>(xa + w * 64);
+                    uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+                    dq_word(wa[w], sa, Za, Zha, a0, a1, a2, a3);
+                    dq_word(wb[w], sb, Zb, Zhb, b0, b1, b2, b3);
+                    mma16816(acc[t][h], a0, b0, a1, b1, xv.x, xv.y);
+                    mma16816(acc[t][h], a2, b2, a3, b3, xv.z, xv.w);
                 }
-#pragma unroll
-                for (int q = 0; q < 8; q++)
-                    mma16816(acc[t], wa[2 * q], wb[2 * q], wa[2 * q + 1], wb[2 * q + 1], xb[2 * q], xb[2 * q + 1]);
             }
         }
         __syncwarp();
@@ -325,13 +366,18 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
             if (++is_j == p.nbx_w) { is_j = 0; is_tile += tile_stride; }
         }
         pa = na;
-        pb = nbp;
-
+        pb = nbq;
         if (nj != 0) {
             j = nj;
             continue;
         }
+
         // ---- end of a tile (for every warp of the CTA at once in split mode)
+        float out[NT][4];
+#pragma unroll
+        for (int t = 0; t < NT; t++)
+#pragma unroll
+            for (int e = 0; e < 4; e++) out[t][e] = acc[t][0][e] + acc[t][1][e];
         const int tile_done = tile;
         tile = ntile;
         j = 0;
@@ -344,16 +390,16 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
                     const int m = 8 * t + 2 * c + (e & 1);
                     const int n = n0 + 8 * (e >> 1);
                     if (m < p.M && n < p.N)
-                        p.Y[(int64_t)m * p.N + n] = __float2half_rn(acc[t][e]);
+                        p.Y[(int64_t)m * p.N + n] = __float2half_rn(out[t][e]);
                 }
         } else {
 #pragma unroll
             for (int t = 0; t < NT; t++) {
                 const int m0 = 8 * t + 2 * c;
-                red[(warp * kRows + g) * MP + m0] = acc[t][0];
-                red[(warp * kRows + g) * MP + m0 + 1] = acc[t][1];
-                red[(warp * kRows + g + 8) * MP + m0] = acc[t][2];
-                red[(warp * kRows + g + 8) * MP + m0 + 1] = acc[t][3];
+                red[(warp * kRows + g) * MP + m0] = out[t][0];
+                red[(warp * kRows + g) * MP + m0 + 1] = out[t][1];
+                red[(warp * kRows + g + 8) * MP + m0] = out[t][2];
+                red[(warp * kRows + g + 8) * MP + m0 + 1] = out[t][3];
             }
             __syncthreads();
             for (int idx = tid; idx < TPC * kRows * MP; idx += kThreads) {
@@ -383,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
 #pragma unroll
         for (int t = 0; t < NT; t++)
 #pragma unroll
-            for (int e = 0; e < 4; e++) acc[t][e] = 0.f;
+            for (int e = 0; e < 8; e++) acc[t][e >> 2][e & 3] = 0.f;
     }
 
     // every issued box was waited for above; after a timeout, let the copies
@@ -426,9 +472,9 @@ int sm_count_tc() {
     return count;
 }
 
-template <int NT>
+template <int NT, class C>
 int launch_tc(const CUtensorMap &map, const TcParams &p, int grid, size_t smem, unsigned flags, cudaStream_t s) {
-    auto fn = gemv_tc_kernel<NT>;
+    auto fn = gemv_tc_kernel<NT, C>;
     static int configured = 0;
     if ((int)smem > configured) {
         cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -501,7 +547,8 @@ int launch_gemv_tc(const void *X, const uint8_t *packed, const void *scales, int
         p.kcta = W * nbx_w * kBoxK;
         p.xs_stride = (p.kcta / kBoxK) * 512 + 64;
         smem = 1024 + (size_t)kWarps * kDepth * kBoxBytes + (size_t)M * p.xs_stride +
-               (size_t)2 * kWarps * kRows * MP * 4 + (size_t)kWarps * kDepth * 8;
+               512 + (size_t)2 * kWarps * kRows * MP * 4 +
+               (size_t)kWarps * kDepth * 8;
         if (smem <= 200 * 1024 || S >= kMaxCluster)
             break;
     }
@@ -535,9 +582,22 @@ int launch_gemv_tc(const void *X, const uint8_t *packed, const void *scales, int
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (cr != CUDA_SUCCESS)
         return fail(MNB_ERR_CUDA, "mnb_gemv: cuTensorMapEncodeTiled failed (%d)", (int)cr);
-    if (NT == 1)
-        return launch_tc<1>(map, p, grid, smem, flags, s);
-    return launch_tc<2>(map, p, grid, smem, flags, s);
+    // fp16 scales read as aligned pairs (block 32) or singly (block 64)
+    const bool fast_scales = scale_f16 && (bs == 64 || p.scale_pair);
+    const bool bs64 = (bs == 64), has_zp = (zp != nullptr);
+#define MNB_TC(NT_, B_, Z_, S_) return launch_tc<NT_, Cfg<B_, Z_, S_>>(map, p, grid, smem, flags, s)
+#define MNB_TC_S(NT_, B_, Z_) \
+    if (fast_scales) MNB_TC(NT_, B_, Z_, 0); else MNB_TC(NT_, B_, Z_, 1)
+#define MNB_TC_Z(NT_, B_) \
+    if (has_zp) { MNB_TC_S(NT_, B_, true); } else { MNB_TC_S(NT_, B_, false); }
+    if (NT == 1) {
+        if (bs64) { MNB_TC_Z(1, true); } else { MNB_TC_Z(1, false); }
+    } else {
+        if (bs64) { MNB_TC_Z(2, true); } else { MNB_TC_Z(2, false); }
+    }
+#undef MNB_TC_Z
+#undef MNB_TC_S
+#undef MNB_TC
 }
 
 int read_gemv_status(unsigned *out, int clear) {
