@@ -307,7 +307,7 @@ def profile_part(args, dev, ranks):
         M, kind = 1, "gemv"
     else:
         lin = [l for l in workloads.config_linears("qwen3_1p7b_prefill") if l.layer == 0]
-        M, kind = 1024, "gemm"
+        M, kind = args.m, "gemm"
     lins = []
     for l in lin:
         W = workloads.weight(cfg["seed"], l.layer, l.proj, l.N, l.K, True, device=dev)
@@ -474,6 +474,7 @@ def main():
     ap.add_argument("--impl", default="mnb", choices=["mnb", "reference"])
     ap.add_argument("--only", default="", choices=["", "decode", "lmhead", "gemm-layer"],
                     help="profiling modes: run one part only and print no JSON line")
+    ap.add_argument("--m", type=int, default=1024, help="tokens of the gemm-layer profiling mode")
     args = ap.parse_args()
     world, rank, local = dist_setup()
     if args.warmup < 3:

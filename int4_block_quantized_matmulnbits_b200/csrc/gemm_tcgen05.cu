@@ -8,18 +8,30 @@
 // in tensor memory).  Weight rows are the MMA's M (128 per CTA) and tokens its N
 // (BN <= 256), so ragged token counts only pad N.
 //
-// Per CTA, a K loop over 64-wide stages in a ring of shared-memory buffers:
-//   warp 0     TMA producer: X tile [BN x 64] fp16, 128-byte swizzle.  Also
-//              allocates / frees the tensor-memory accumulator.
-//   warp 1     MMA issuer: one thread issues 4 x tcgen05.mma (K = 16 each) per
-//              stage and commits to the stage's "empty" barrier.
-//   warps 2-5  dequant producers, one weight row per thread: 32 packed bytes
-//              -> 64 fp16 = fp16_rn((q - zp) * scale), written in the
-//              128-byte-swizzled K-major layout the MMA descriptor reads, then
-//              fence.proxy.async + mbarrier arrive.  Their global loads run a
-//              few stages ahead in a register ring.  After the K loop the same
-//              warps are the epilogue: tcgen05.ld of their 32 TMEM lanes,
-//              fp16 conversion, coalesced stores of Y.
+// Per CTA, a K loop over 64-wide stages fed by three shared-memory rings (packed
+// weights 8 deep, X tiles up to 8 deep, fp16 weight tiles 3 deep), so the long
+// DRAM latency of the weight stream is covered without holding X or fp16 space:
+//   warp 0      TMA producer of the packed weight tile (128 rows x 32 bytes) of
+//               every stage; it never waits for the previous kernel, whose
+//               output the weights do not depend on.  Also allocates / frees the
+//               tensor-memory accumulator.
+//   warp 2      TMA producer of the X tile [BN x 64] fp16 (128-byte swizzle),
+//               after griddepcontrol.wait.
+//   warp 1      MMA issuer: one thread issues 4 x tcgen05.mma (K = 16 each) per
+//               stage and commits to the X and fp16-weight "empty" barriers.
+//   warps 3-18  dequant: four threads per weight row, 16 k each per stage: 8
+//               packed bytes from shared memory -> 16 fp16 = fp16_rn((q - zp) *
+//               scale), written in the 128-byte-swizzled K-major layout the MMA
+//               descriptor reads, then fence.proxy.async + mbarrier arrive.
+//               Sixteen warps so that the unpack's dependency chains overlap.
+//               Scales and zero points run a few stages ahead in registers.
+//               After the K loop the same warps are the epilogue: tcgen05.ld of
+//               their 32 TMEM lanes, fp16 conversion, stores of Y.
+// When rows x token tiles cannot occupy the SMs, K is split over a cluster of S
+// CTAs; each keeps its partial sum in its own tensor memory, parks it in its
+// shared memory, and every rank reduces one slice of the token columns by
+// reading the others' partials through distributed shared memory (no global
+// scratch).
 // Every mbarrier wait is bounded in time: past the limit the kernel records
 // the failure in a device status word, drains what it issued, frees tensor
 // memory and exits.
@@ -34,25 +46,31 @@ __device__ unsigned g_mnb_status = 0;
 
 namespace {
 
-constexpr int kThreads = 192;   // 6 warps
-constexpr int kBM = 128;        // weight rows per CTA
-constexpr int kBK = 64;         // k per stage (128 bytes of fp16 = one swizzle row)
-constexpr int kWRing = 3;       // dequant loads in flight per thread
+constexpr int kDqWarps = 16;
+constexpr int kThreads = 96 + kDqWarps * 32;   // 2 TMA producers, MMA, 16 dequant warps
+constexpr int kDqThreads = kDqWarps * 32;
+constexpr int kBM = 128;                       // weight rows per CTA
+constexpr int kBK = 64;                        // k per stage (128 bytes of fp16 = one swizzle row)
+constexpr int kWBytes = kBM * 128;             // fp16 weight tile per stage
+constexpr int kPBytes = kBM * 32;              // packed weight tile per stage
+constexpr int kPR = 4;                         // stages of scales / zero points prefetched
+constexpr int kWS = 3;                         // fp16 weight tiles in the ring
+constexpr int kPS = 8;                         // packed weight tiles in flight
+constexpr int kMaxCluster = 8;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
 
 struct GemmParams {
-    const uint8_t *packed;
     const void *scales;
     const uint8_t *zp;
     __half *Y;
     int M, N, K;
     int bs_shift, nb, zpb, scale_f16;
     int BN;        // tokens per CTA (multiple of 16, <= 256)
-    int stages;    // shared-memory ring depth
+    int xstages;   // depth of the X ring
     int tmem_cols; // power of two >= BN
+    int S;         // CTAs per cluster along K
+    int kslice;    // k per cluster rank (multiple of kBK)
 };
-
-// ---- mbarrier / TMA / tcgen05 wrappers -------------------------------------
 
 // Waits for the phase with the given parity; false after the time limit or,
 // unless `drain`, as soon as another role has given up (*abort set).  Drain
@@ -78,12 +96,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     }
 }
 
-__device__ __forceinline__ void tc_fence_before() {
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
 // 1024 bytes apart.
@@ -118,57 +132,63 @@ __device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t v[16]) {
 
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// ---- dequant of one stage of one weight row --------------------------------
-
-struct WSlot {
-    uint4 p0, p1;       // k 0..31 and 32..63 of the stage
-    uint32_t s0, s1;    // fp16 bits of the scales of the (up to) two blocks
-    uint32_t z0, z1;    // zero points
-};
-
-__device__ __forceinline__ WSlot load_wslot(const GemmParams &p, int n, int it, int nk) {
-    WSlot w;
-    w.p0 = w.p1 = make_uint4(0, 0, 0, 0);
-    w.s0 = w.s1 = 0;
-    w.z0 = w.z1 = 8;
-    if (it >= nk)
-        return w;
-    const int k0 = it * kBK;
-    const uint8_t *row = p.packed + (int64_t)n * (p.K / 2) + k0 / 2;
-    w.p0 = ldg_stream_v4(row);
-    w.p1 = ldg_stream_v4(row + 16);
-    const int b0 = k0 >> (5 + p.bs_shift);
-    const int b1 = (k0 + 32) >> (5 + p.bs_shift);
-    if (p.scale_f16) {
-        const unsigned short *s = reinterpret_cast<const unsigned short *>(p.scales) + (int64_t)n * p.nb;
-        w.s0 = __ldg(s + b0);
-        w.s1 = __ldg(s + b1);
-    } else {
-        // fp32 scales: the tensor cores take fp16 operands, so round the scale once here
-        const float *s = reinterpret_cast<const float *>(p.scales) + (int64_t)n * p.nb;
-        w.s0 = __half_as_ushort(__float2half_rn(__ldg(s + b0)));
-        w.s1 = __half_as_ushort(__float2half_rn(__ldg(s + b1)));
-    }
-    if (p.zp) {
-        const uint8_t *z = p.zp + (int64_t)n * p.zpb;
-        const uint32_t zb0 = __ldg(z + (b0 >> 1)), zb1 = __ldg(z + (b1 >> 1));
-        w.z0 = (b0 & 1) ? (zb0 >> 4) : (zb0 & 15);
-        w.z1 = (b1 & 1) ? (zb1 >> 4) : (zb1 & 15);
-    }
-    return w;
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
 }
 
-// 32 nibbles -> 32 fp16 = fp16_rn((q - zp) * s) in natural k order, written as
-// four 16-byte chunks (k 8j..8j+7) of the swizzled row.
-__device__ __forceinline__ void dq_store_half_row(const uint4 &p, uint32_t s16, uint32_t z, uint32_t row_addr,
-                                                  int r7, int j0) {
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float4 ld_dsmem_f4(const float *local, uint32_t rank) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(remote)
+                 : "memory");
+    return v;
+}
+
+// Scale (fp16 bits) and zero point of one thread's 16-k quarter of a stage.
+struct SZ {
+    uint32_t s, z;
+};
+
+__device__ __forceinline__ SZ load_sz(const GemmParams &p, int n, int k) {
+    SZ r;
+    r.s = 0;
+    r.z = 8;
+    if (k >= p.K)
+        return r;
+    const int b = k >> (5 + p.bs_shift);
+    if (p.scale_f16)
+        r.s = __ldg(reinterpret_cast<const unsigned short *>(p.scales) + (int64_t)n * p.nb + b);
+    else
+        r.s = __half_as_ushort(
+            __float2half_rn(__ldg(reinterpret_cast<const float *>(p.scales) + (int64_t)n * p.nb + b)));
+    if (p.zp) {
+        const uint32_t zb = __ldg(p.zp + (int64_t)n * p.zpb + (b >> 1));
+        r.z = (b & 1) ? (zb >> 4) : (zb & 15u);
+    }
+    return r;
+}
+
+// 8 packed bytes (16 k of one row) -> 16 fp16 = fp16_rn((q - zp) * s) in natural
+// k order, written as two 16-byte chunks (k 8j..8j+7, j = j0, j0+1) of the
+// row's 128-byte swizzled line.
+__device__ __forceinline__ void dq_store(const uint2 &v, uint32_t s16, uint32_t z, uint32_t row_addr, int r7,
+                                         int j0) {
     const half2 sixteenth = __floats2half2_rn(0.0625f, 0.0625f);
     const half2 s2 = u32_as_h2(s16 | (s16 << 16));
-    const uint32_t Z = 0x64006400u | (z * 0x00010001u);
-    const uint32_t Zhi = 0xD400D400u + (z * 0x00100010u);
-    const uint32_t words[4] = {p.x, p.y, p.z, p.w};
+    const uint32_t Z = 0x64006400u | (z * 0x00010001u);      // 1024 + zp
+    const uint32_t Zhi = 0xD400D400u + (z * 0x00100010u);    // -(64 + zp)
+    const uint32_t words[2] = {v.x, v.y};
 #pragma unroll
-    for (int i = 0; i < 4; i++) {
+    for (int i = 0; i < 2; i++) {
         const uint32_t w = words[i];
         const uint32_t w8 = w >> 8;
         // (e0,e4) (e1,e5) (e2,e6) (e3,e7) as exact q - zp, then times the scale
@@ -184,44 +204,60 @@ __device__ __forceinline__ void dq_store_half_row(const uint4 &p, uint32_t s16, 
         o.y = __byte_perm(c, d, 0x5410);   // (e2, e3)
         o.z = __byte_perm(a, b, 0x7632);   // (e4, e5)
         o.w = __byte_perm(c, d, 0x7632);   // (e6, e7)
-        const int j = j0 + i;
-        const uint32_t dst = row_addr + (uint32_t)(((j ^ r7) & 7) << 4);
+        const uint32_t dst = row_addr + (uint32_t)((((j0 + i) ^ r7) & 7) << 4);
         asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(o.x), "r"(o.y), "r"(o.z), "r"(o.w)
                      : "memory");
     }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap xmap, const GemmParams p) {
+    gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap wmap,
+                const GemmParams p) {
     extern __shared__ unsigned char smem_raw[];
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const int S = p.stages;
+    const int WS = kWS, PS = kPS, XS = p.xstages;
     const int BN = p.BN;
-    const int n_tile = blockIdx.x;          // weight-row tile
+    const int rank = (p.S > 1) ? (int)cluster_ctarank() : 0;
+    const int n_tile = blockIdx.x / p.S;    // weight-row tile
     const int m_tile = blockIdx.y;          // token tile
-    const int nk = p.K / kBK;
+    const int kbeg = rank * p.kslice;
+    const int kend = min(p.K, kbeg + p.kslice);
+    const int nk = (kend > kbeg) ? (kend - kbeg) / kBK : 0;
 
-    // layout: [stages][W 16 KB][X BN*128 B] (1024-aligned), then barriers
+    // layout (1024-aligned): W16 ring [WS][16 KB] | X ring [XS][BN*128 B] |
+    // packed ring [PS][4 KB] | barriers
     const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
     unsigned char *base_ptr = smem_raw + (base - smem_u32(smem_raw));
-    const uint32_t w_bytes = kBM * 128;
     const uint32_t x_bytes = (uint32_t)BN * 128;
-    const uint32_t stage_bytes = w_bytes + x_bytes;
-    const uint32_t bar_base = base + (uint32_t)S * stage_bytes;
-    // barriers: full_x[S], full_w[S], empty[S], acc_full; then tmem addr, abort flag
-    auto full_x = [&](int s) { return bar_base + 8u * (uint32_t)s; };
-    auto full_w = [&](int s) { return bar_base + 8u * (uint32_t)(S + s); };
-    auto empty = [&](int s) { return bar_base + 8u * (uint32_t)(2 * S + s); };
-    const uint32_t acc_full = bar_base + 8u * (uint32_t)(3 * S);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + (size_t)S * stage_bytes + 8 * (3 * S + 1));
+    const uint32_t x_base = base + (uint32_t)WS * kWBytes;
+    const uint32_t p_base = x_base + (uint32_t)XS * x_bytes;
+    auto w_addr = [&](int i) { return base + (uint32_t)(i % WS) * kWBytes; };
+    auto x_addr = [&](int i) { return x_base + (uint32_t)(i % XS) * x_bytes; };
+    auto p_off = [&](int i) { return (p_base - base) + (uint32_t)(i % PS) * kPBytes; };
+    const uint32_t bars = p_base + (uint32_t)PS * kPBytes;
+    auto pfull = [&](int i) { return bars + 8u * (uint32_t)(i % PS); };
+    auto pempty = [&](int i) { return bars + 8u * (uint32_t)(PS + i % PS); };
+    auto wfull = [&](int i) { return bars + 8u * (uint32_t)(2 * PS + i % WS); };
+    auto wempty = [&](int i) { return bars + 8u * (uint32_t)(2 * PS + WS + i % WS); };
+    auto xfull = [&](int i) { return bars + 8u * (uint32_t)(2 * PS + 2 * WS + i % XS); };
+    auto xempty = [&](int i) { return bars + 8u * (uint32_t)(2 * PS + 2 * WS + XS + i % XS); };
+    const uint32_t acc_full = bars + 8u * (uint32_t)(2 * PS + 2 * WS + 2 * XS);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + (acc_full + 8 - base));
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     if (tid == 0) {
-        for (int s = 0; s < S; s++) {
-            mbar_init(full_x(s), 1);
-            mbar_init(full_w(s), 128);
-            mbar_init(empty(s), 1);
+        for (int i = 0; i < PS; i++) {
+            mbar_init(pfull(i), 1);
+            mbar_init(pempty(i), kDqThreads);
+        }
+        for (int i = 0; i < WS; i++) {
+            mbar_init(wfull(i), kDqThreads);
+            mbar_init(wempty(i), 1);
+        }
+        for (int i = 0; i < XS; i++) {
+            mbar_init(xfull(i), 1);
+            mbar_init(xempty(i), 1);
         }
         mbar_init(acc_full, 1);
         *abort = 0;
@@ -241,92 +277,164 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0) {
         if (lane == 0) {
+            // ---------------- TMA producer of packed weights (independent of the
+            // previous kernel: no griddepcontrol.wait)
+            int issued = 0;
+            for (int i = 0; i < nk; i++) {
+                if (i >= PS && !mbar_wait(pempty(i), ((i / PS) - 1) & 1, abort))
+                    break;
+                mbar_expect_tx(pfull(i), kPBytes);
+                tma_load_2d(base + p_off(i), &wmap, pfull(i), (kbeg + i * kBK) / 2, n_tile * kBM);
+                issued = i + 1;
+            }
+            if (*abort)
+                for (int i = (issued > PS ? issued - PS : 0); i < issued; i++)
+                    mbar_wait(pfull(i), (i / PS) & 1, abort, true);
+        }
+    } else if (warp == 2) {
+        if (lane == 0) {
             // ---------------- TMA producer of X tiles
             pdl_wait();
             int issued = 0;
-            for (int it = 0; it < nk; it++) {
-                const int s = it % S;
-                if (it >= S && !mbar_wait(empty(s), ((it / S) - 1) & 1, abort))
+            for (int i = 0; i < nk; i++) {
+                if (i >= XS && !mbar_wait(xempty(i), ((i / XS) - 1) & 1, abort))
                     break;
-                mbar_expect_tx(full_x(s), x_bytes);
-                tma_load_2d(base + (uint32_t)s * stage_bytes + w_bytes, &xmap, full_x(s), it * kBK, m_tile * BN);
-                issued = it + 1;
+                mbar_expect_tx(xfull(i), x_bytes);
+                tma_load_2d(x_addr(i), &xmap, xfull(i), kbeg + i * kBK, m_tile * BN);
+                issued = i + 1;
             }
-            if (*abort) {
-                // drain: every issued load must land before the CTA exits
-                for (int it = (issued > S ? issued - S : 0); it < issued; it++)
-                    mbar_wait(full_x(it % S), (it / S) & 1, abort, true);
-            }
+            if (*abort)
+                for (int i = (issued > XS ? issued - XS : 0); i < issued; i++)
+                    mbar_wait(xfull(i), (i / XS) & 1, abort, true);
         }
     } else if (warp == 1) {
         if (lane == 0) {
             // ---------------- MMA issuer
             const uint32_t idesc = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
-            for (int it = 0; it < nk; it++) {
-                const int s = it % S;
-                const uint32_t par = (it / S) & 1;
-                if (!mbar_wait(full_x(s), par, abort) || !mbar_wait(full_w(s), par, abort))
+            for (int i = 0; i < nk; i++) {
+                if (!mbar_wait(xfull(i), (i / XS) & 1, abort) || !mbar_wait(wfull(i), (i / WS) & 1, abort))
                     break;
                 tc_fence_after();
-                const uint32_t wa = base + (uint32_t)s * stage_bytes;
-                const uint32_t xa = wa + w_bytes;
 #pragma unroll
                 for (int kk = 0; kk < kBK / 16; kk++)
-                    tc_mma_f16(tmem, sw128_desc(wa + kk * 32), sw128_desc(xa + kk * 32), idesc,
-                               (it > 0 || kk > 0) ? 1u : 0u);
-                tc_commit(empty(s));
+                    tc_mma_f16(tmem, sw128_desc(w_addr(i) + kk * 32), sw128_desc(x_addr(i) + kk * 32), idesc,
+                               (i > 0 || kk > 0) ? 1u : 0u);
+                tc_commit(xempty(i));
+                tc_commit(wempty(i));
             }
             tc_commit(acc_full);   // fires once every MMA issued above has completed
         }
     } else {
-        // ---------------- dequant producers (one weight row each), then epilogue
-        const int q = warp & 3;                  // TMEM lane quarter of this warp
-        const int r = q * 32 + lane;             // row within the tile
+        // ---------------- dequant: thread = (row r, quarter of the stage's 64 k)
+        const int dt = tid - 96;
+        const int r = dt >> 2, qtr = dt & 3;
         const int n = n_tile * kBM + r;
         const int r7 = r & 7;
-        WSlot ring[kWRing];
+        SZ ring[kPR];
 #pragma unroll
-        for (int i = 0; i < kWRing; i++)
-            ring[i] = load_wslot(p, n, i, nk);
+        for (int i = 0; i < kPR; i++)
+            ring[i] = (i < nk) ? load_sz(p, n, kbeg + i * kBK + qtr * 16) : SZ{0u, 8u};
         bool ok = true;
-        for (int base_it = 0; base_it < nk && ok; base_it += kWRing) {
+        for (int base_it = 0; base_it < nk && ok; base_it += kPR) {
 #pragma unroll
-            for (int i = 0; i < kWRing; i++) {
+            for (int i = 0; i < kPR; i++) {
                 const int it = base_it + i;
                 if (it < nk && ok) {
-                    const int s = it % S;
-                    if (it >= S && !mbar_wait(empty(s), ((it / S) - 1) & 1, abort)) {
+                    if (!mbar_wait(pfull(it), (it / PS) & 1, abort) ||
+                        (it >= WS && !mbar_wait(wempty(it), ((it / WS) - 1) & 1, abort))) {
                         ok = false;
                     } else {
-                        const WSlot cur = ring[i];
-                        ring[i] = load_wslot(p, n, it + kWRing, nk);
-                        const uint32_t row_addr = base + (uint32_t)s * stage_bytes + (uint32_t)r * 128;
-                        dq_store_half_row(cur.p0, cur.s0, cur.z0, row_addr, r7, 0);
-                        dq_store_half_row(cur.p1, cur.s1, cur.z1, row_addr, r7, 4);
+                        const SZ cur = ring[i];
+                        if (it + kPR < nk)
+                            ring[i] = load_sz(p, n, kbeg + (it + kPR) * kBK + qtr * 16);
+                        const uint2 v = *reinterpret_cast<const uint2 *>(base_ptr + p_off(it) + r * 32 + qtr * 8);
+                        mbar_arrive(pempty(it));   // the packed bytes are in registers now
+                        dq_store(v, cur.s, cur.z, w_addr(it) + (uint32_t)r * 128, r7, qtr * 2);
                         fence_proxy_async_smem();
-                        mbar_arrive(full_w(s));
+                        mbar_arrive(wfull(it));
                     }
                 }
             }
         }
-        // ---------------- epilogue: TMEM -> registers -> Y
-        if (mbar_wait(acc_full, 0, abort)) {
-            tc_fence_after();
-            pdl_wait();
-            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16);
-            const int m0 = m_tile * BN;
-            for (int col = 0; col < BN; col += 16) {
-                uint32_t v[16];
-                tc_ld16(taddr + (uint32_t)col, v);
-                tc_wait_ld();
+
+        // ---------------- epilogue: TMEM -> registers -> (cluster reduction) -> Y
+        const int q = warp & 3;                  // TMEM lane quarter of this warp
+        const int grp = (warp - 3) >> 2;         // 0..3: this warp's share of the column chunks
+        const int row = q * 32 + lane;
+        const int ny = n_tile * kBM + row;
+        const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16);
+        const int m0 = m_tile * BN;
+        const int nchunk = BN / 16;
+        const int red_pitch = BN + 4;            // floats per row of the partial-sum buffer
+        float *red = reinterpret_cast<float *>(base_ptr);   // reuses the ring buffers
+        const bool have = mbar_wait(acc_full, 0, abort) && nk > 0;
+        tc_fence_after();
+        pdl_wait();
+        auto store_y = [&](int col, const float *f) {
 #pragma unroll
-                for (int j = 0; j < 16; j++) {
-                    const int m = m0 + col + j;
-                    if (m < p.M)
-                        p.Y[(int64_t)m * p.N + n] = __float2half_rn(__uint_as_float(v[j]));
-                }
+            for (int j = 0; j < 16; j++) {
+                const int m = m0 + col + j;
+                if (m < p.M)
+                    p.Y[(int64_t)m * p.N + ny] = __float2half_rn(f[j]);
             }
+        };
+        if (p.S == 1) {
+            for (int c16 = grp; c16 < nchunk; c16 += 4) {
+                uint32_t v[16];
+                float f[16];
+                if (have) {
+                    tc_ld16(taddr + (uint32_t)(c16 * 16), v);
+                    tc_wait_ld();
+                }
+#pragma unroll
+                for (int j = 0; j < 16; j++) f[j] = have ? __uint_as_float(v[j]) : 0.f;
+                store_y(c16 * 16, f);
+            }
+        } else {
+            // park this rank's partial sums, then each rank reduces its own chunks
+            for (int c16 = grp; c16 < nchunk; c16 += 4) {
+                uint32_t v[16];
+                if (have) {
+                    tc_ld16(taddr + (uint32_t)(c16 * 16), v);
+                    tc_wait_ld();
+                }
+                float4 *dst = reinterpret_cast<float4 *>(red + row * red_pitch + c16 * 16);
+#pragma unroll
+                for (int j = 0; j < 4; j++)
+                    dst[j] = have ? make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                                __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]))
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            cluster_sync();
+            for (int c16 = rank + p.S * grp; c16 < nchunk; c16 += 4 * p.S) {
+                float f[16];
+                const float4 *own = reinterpret_cast<const float4 *>(red + row * red_pitch + c16 * 16);
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    const float4 o = own[j];
+                    f[4 * j] = o.x; f[4 * j + 1] = o.y; f[4 * j + 2] = o.z; f[4 * j + 3] = o.w;
+                }
+                for (int qq = 0; qq < p.S; qq++) {
+                    if (qq == rank)
+                        continue;
+                    float4 o4[4];
+#pragma unroll
+                    for (int j = 0; j < 4; j++)
+                        o4[j] = ld_dsmem_f4(red + row * red_pitch + c16 * 16 + 4 * j, (uint32_t)qq);
+#pragma unroll
+                    for (int j = 0; j < 4; j++) {
+                        f[4 * j] += o4[j].x; f[4 * j + 1] += o4[j].y; f[4 * j + 2] += o4[j].z; f[4 * j + 3] += o4[j].w;
+                    }
+                }
+                store_y(c16 * 16, f);
+            }
+            cluster_sync();   // every rank has read what it needs: the buffers may go
         }
+    }
+    if (p.S > 1 && warp < 3) {
+        // the producer and MMA warps take part in the epilogue's cluster barriers
+        cluster_sync();
+        cluster_sync();
     }
 
     // ---------------- teardown
@@ -362,32 +470,41 @@ EncodeTiledFn get_encode_fn() {
 
 }  // namespace
 
+// Tile policy knobs (tuning hooks, see mnb_tune_gemm below).
+static int g_gemm_min_bn = 128;      // smallest token tile the grid heuristic may pick
+static int g_gemm_max_split = kMaxCluster;
+
 int launch_gemm(const void *X, const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,
                 void *Y, int M, int N, int K, int bs, unsigned flags, cudaStream_t s) {
     EncodeTiledFn encode = get_encode_fn();
     if (!encode)
         return fail(MNB_ERR_CUDA, "mnb_gemm: cuTensorMapEncodeTiled unavailable");
-
-    // token tiling: as few tiles of <= 256 as possible, evenly sized
-    int mt = (M + 255) / 256;
-    int BN = ((M + mt - 1) / mt + 15) / 16 * 16;
-    const int n_tiles = N / kBM;
     int sms = 148;
     {
         int dev = 0;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     }
-    // narrower token tiles when the grid would leave most SMs idle
-    while (BN > 64 && (int64_t)n_tiles * mt * 2 <= sms) {
+
+    // token tiling: as few tiles of <= 256 as possible, evenly sized; narrower
+    // tiles (down to g_gemm_min_bn) while the grid would leave half the SMs idle
+    int mt = (M + 255) / 256;
+    int BN = ((M + mt - 1) / mt + 15) / 16 * 16;
+    const int n_tiles = N / kBM;
+    while (BN > g_gemm_min_bn && BN > 16 && (int64_t)n_tiles * mt * 4 <= sms) {
         mt = (M + BN / 2 - 1) / (BN / 2);
         BN = ((M + mt - 1) / mt + 15) / 16 * 16;
     }
     if (mt > 65535)
         return fail(MNB_ERR_SHAPE, "mnb_gemm: M too large");
+    // split K over a cluster when the tiles still leave most SMs idle
+    const int nk_all = K / kBK;
+    int S = 1;
+    while (S * 2 <= g_gemm_max_split && (int64_t)n_tiles * mt * S * 2 <= sms && nk_all / (S * 2) >= 4)
+        S *= 2;
+    const int kslice = (nk_all + S - 1) / S * kBK;
 
     GemmParams p;
-    p.packed = packed;
     p.scales = scales;
     p.zp = zp;
     p.Y = reinterpret_cast<__half *>(Y);
@@ -398,24 +515,43 @@ int launch_gemm(const void *X, const uint8_t *packed, const void *scales, int sc
     p.scale_f16 = scale_f16;
     p.BN = BN;
     p.tmem_cols = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
-    const int stage_bytes = kBM * 128 + BN * 128;
-    const int budget = 200 * 1024;
-    int stages = budget / stage_bytes;
-    if (stages > 8) stages = 8;
-    if (stages < 2) stages = 2;
-    p.stages = stages;
-    const size_t smem = 1024 + (size_t)stages * stage_bytes + 8 * (3 * stages + 1) + 16;
+    p.S = S;
+    p.kslice = kslice;
+    // rings: 3 fp16 weight tiles, 8 packed tiles, as many X tiles as fit (<= 8)
+    const int fixed = kWS * kWBytes + kPS * kPBytes;
+    int xstages = (200 * 1024 - fixed) / (BN * 128);
+    if (xstages > 8) xstages = 8;
+    if (xstages < 2) xstages = 2;
+    const size_t ring_bytes = (size_t)fixed + (size_t)xstages * BN * 128;
+    // the cluster reduction reuses the rings for [128][BN + 4] fp32
+    if (S > 1 && ring_bytes < (size_t)kBM * (BN + 4) * 4)
+        return fail(MNB_ERR_SHAPE, "mnb_gemm: reduction buffer does not fit");
+    p.xstages = xstages;
+    const size_t smem = 1024 + ring_bytes + 8 * (2 * kPS + 2 * kWS + 2 * xstages + 1) + 16;
 
-    CUtensorMap xmap;
-    const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
-    const cuuint64_t gstride[1] = {(cuuint64_t)K * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)BN};
-    const cuuint32_t estride[2] = {1, 1};
-    CUresult cr = encode(&xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(X), gdim, gstride, box,
-                         estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (cr != CUDA_SUCCESS)
-        return fail(MNB_ERR_CUDA, "mnb_gemm: cuTensorMapEncodeTiled failed (%d)", (int)cr);
+    CUtensorMap xmap, wmap;
+    {
+        const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
+        const cuuint64_t gstride[1] = {(cuuint64_t)K * 2};
+        const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)BN};
+        const cuuint32_t estride[2] = {1, 1};
+        CUresult cr = encode(&xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(X), gdim, gstride, box,
+                             estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (cr != CUDA_SUCCESS)
+            return fail(MNB_ERR_CUDA, "mnb_gemm: cuTensorMapEncodeTiled (X) failed (%d)", (int)cr);
+    }
+    {
+        const cuuint64_t gdim[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N};
+        const cuuint64_t gstride[1] = {(cuuint64_t)(K / 2)};
+        const cuuint32_t box[2] = {32, (cuuint32_t)kBM};
+        const cuuint32_t estride[2] = {1, 1};
+        CUresult cr = encode(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), gdim, gstride,
+                             box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (cr != CUDA_SUCCESS)
+            return fail(MNB_ERR_CUDA, "mnb_gemm: cuTensorMapEncodeTiled (W) failed (%d)", (int)cr);
+    }
 
     static int configured = 0;
     if ((int)smem > configured) {
@@ -425,12 +561,19 @@ int launch_gemm(const void *X, const uint8_t *packed, const void *scales, int sc
         configured = (int)smem;
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)n_tiles, (unsigned)mt, 1);
+    cfg.gridDim = dim3((unsigned)(n_tiles * S), (unsigned)mt, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     int na = 0;
+    if (S > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = (unsigned)S;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        na++;
+    }
     if (flags & MNB_FLAG_PDL) {
         attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[na].val.programmaticStreamSerializationAllowed = 1;
@@ -438,9 +581,17 @@ int launch_gemm(const void *X, const uint8_t *packed, const void *scales, int sc
     }
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel, xmap, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel, xmap, wmap, p);
     if (e != cudaSuccess)
         return fail(MNB_ERR_CUDA, "mnb_gemm: launch: %s", cudaGetErrorString(e));
+    return MNB_OK;
+}
+
+int tune_gemm(int min_bn, int max_split) {
+    if (min_bn < 16 || min_bn > 256 || max_split < 1 || max_split > kMaxCluster)
+        return MNB_ERR_INVALID_ARG;
+    g_gemm_min_bn = min_bn;
+    g_gemm_max_split = max_split;
     return MNB_OK;
 }
 
@@ -461,3 +612,7 @@ int read_device_status(unsigned *out, int clear) {
 }
 
 }  // namespace mnb
+
+// Tuning hook: smallest token tile the tile heuristic may choose (16..256) and
+// the largest cluster split along K (1..8).  Not part of the stable ABI.
+extern "C" MNB_API int mnb_tune_gemm(int min_bn, int max_split) { return mnb::tune_gemm(min_bn, max_split); }
