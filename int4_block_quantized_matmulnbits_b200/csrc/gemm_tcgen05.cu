@@ -22,7 +22,8 @@
 //   warps 3-18  dequant: four threads per weight row, 16 k each per stage: 8
 //               packed bytes from shared memory -> 16 fp16 = fp16_rn((q - zp) *
 //               scale), written in the 128-byte-swizzled K-major layout the MMA
-//               descriptor reads, then fence.proxy.async + mbarrier arrive.
+//               descriptor reads, then fence.proxy.async, __syncwarp and one
+//               mbarrier arrival per warp.
 //               Sixteen warps so that the unpack's dependency chains overlap.
 //               Scales and zero points run a few stages ahead in registers.
 //               After the K loop the same warps are the epilogue: tcgen05.ld of
@@ -48,7 +49,6 @@ namespace {
 
 constexpr int kDqWarps = 16;
 constexpr int kThreads = 96 + kDqWarps * 32;   // 2 TMA producers, MMA, 16 dequant warps
-constexpr int kDqThreads = kDqWarps * 32;
 constexpr int kBM = 128;                       // weight rows per CTA
 constexpr int kBK = 64;                        // k per stage (128 bytes of fp16 = one swizzle row)
 constexpr int kWBytes = kBM * 128;             // fp16 weight tile per stage
@@ -94,6 +94,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
             }
         }
     }
+}
+
+// mbar_wait by a whole warp with a warp-uniform result.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int *abort) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -249,10 +254,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
         for (int i = 0; i < PS; i++) {
             mbar_init(pfull(i), 1);
-            mbar_init(pempty(i), kDqThreads);
+            mbar_init(pempty(i), kDqWarps);
         }
         for (int i = 0; i < WS; i++) {
-            mbar_init(wfull(i), kDqThreads);
+            mbar_init(wfull(i), kDqWarps);
             mbar_init(wempty(i), 1);
         }
         for (int i = 0; i < XS; i++) {
@@ -275,46 +280,50 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_slot;
     pdl_launch_dependents();
 
+    // The producer and MMA warps run their loops with all 32 lanes (lane 0
+    // issues); a warp left diverged for the whole K loop runs far slower.
     if (warp == 0) {
-        if (lane == 0) {
-            // ---------------- TMA producer of packed weights (independent of the
-            // previous kernel: no griddepcontrol.wait)
-            int issued = 0;
-            for (int i = 0; i < nk; i++) {
-                if (i >= PS && !mbar_wait(pempty(i), ((i / PS) - 1) & 1, abort))
-                    break;
+        // ---------------- TMA producer of packed weights (independent of the
+        // previous kernel: no griddepcontrol.wait)
+        int issued = 0;
+        for (int i = 0; i < nk; i++) {
+            if (i >= PS && !warp_wait(pempty(i), ((i / PS) - 1) & 1, abort))
+                break;
+            if (lane == 0) {
                 mbar_expect_tx(pfull(i), kPBytes);
                 tma_load_2d(base + p_off(i), &wmap, pfull(i), (kbeg + i * kBK) / 2, n_tile * kBM);
-                issued = i + 1;
             }
-            if (*abort)
-                for (int i = (issued > PS ? issued - PS : 0); i < issued; i++)
-                    mbar_wait(pfull(i), (i / PS) & 1, abort, true);
+            __syncwarp();
+            issued = i + 1;
         }
+        if (*abort)
+            for (int i = (issued > PS ? issued - PS : 0); i < issued; i++)
+                mbar_wait(pfull(i), (i / PS) & 1, abort, true);
     } else if (warp == 2) {
-        if (lane == 0) {
-            // ---------------- TMA producer of X tiles
-            pdl_wait();
-            int issued = 0;
-            for (int i = 0; i < nk; i++) {
-                if (i >= XS && !mbar_wait(xempty(i), ((i / XS) - 1) & 1, abort))
-                    break;
+        // ---------------- TMA producer of X tiles
+        pdl_wait();
+        int issued = 0;
+        for (int i = 0; i < nk; i++) {
+            if (i >= XS && !warp_wait(xempty(i), ((i / XS) - 1) & 1, abort))
+                break;
+            if (lane == 0) {
                 mbar_expect_tx(xfull(i), x_bytes);
                 tma_load_2d(x_addr(i), &xmap, xfull(i), kbeg + i * kBK, m_tile * BN);
-                issued = i + 1;
             }
-            if (*abort)
-                for (int i = (issued > XS ? issued - XS : 0); i < issued; i++)
-                    mbar_wait(xfull(i), (i / XS) & 1, abort, true);
+            __syncwarp();
+            issued = i + 1;
         }
+        if (*abort)
+            for (int i = (issued > XS ? issued - XS : 0); i < issued; i++)
+                mbar_wait(xfull(i), (i / XS) & 1, abort, true);
     } else if (warp == 1) {
-        if (lane == 0) {
-            // ---------------- MMA issuer
-            const uint32_t idesc = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
-            for (int i = 0; i < nk; i++) {
-                if (!mbar_wait(xfull(i), (i / XS) & 1, abort) || !mbar_wait(wfull(i), (i / WS) & 1, abort))
-                    break;
-                tc_fence_after();
+        // ---------------- MMA issuer
+        const uint32_t idesc = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+        for (int i = 0; i < nk; i++) {
+            if (!warp_wait(xfull(i), (i / XS) & 1, abort) || !warp_wait(wfull(i), (i / WS) & 1, abort))
+                break;
+            tc_fence_after();
+            if (lane == 0) {
 #pragma unroll
                 for (int kk = 0; kk < kBK / 16; kk++)
                     tc_mma_f16(tmem, sw128_desc(w_addr(i) + kk * 32), sw128_desc(x_addr(i) + kk * 32), idesc,
@@ -322,8 +331,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_commit(xempty(i));
                 tc_commit(wempty(i));
             }
-            tc_commit(acc_full);   // fires once every MMA issued above has completed
+            __syncwarp();
         }
+        if (lane == 0)
+            tc_commit(acc_full);   // fires once every MMA issued above has completed
+        __syncwarp();
     } else {
         // ---------------- dequant: thread = (row r, quarter of the stage's 64 k)
         const int dt = tid - 96;
@@ -340,18 +352,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < kPR; i++) {
                 const int it = base_it + i;
                 if (it < nk && ok) {
-                    if (!mbar_wait(pfull(it), (it / PS) & 1, abort) ||
-                        (it >= WS && !mbar_wait(wempty(it), ((it / WS) - 1) & 1, abort))) {
-                        ok = false;
-                    } else {
+                    // warp-uniform outcome, so the warp stays converged for __syncwarp
+                    ok = __all_sync(0xffffffffu, mbar_wait(pfull(it), (it / PS) & 1, abort) &&
+                                                     (it < WS || mbar_wait(wempty(it), ((it / WS) - 1) & 1, abort)));
+                    if (ok) {
                         const SZ cur = ring[i];
                         if (it + kPR < nk)
                             ring[i] = load_sz(p, n, kbeg + (it + kPR) * kBK + qtr * 16);
                         const uint2 v = *reinterpret_cast<const uint2 *>(base_ptr + p_off(it) + r * 32 + qtr * 8);
-                        mbar_arrive(pempty(it));   // the packed bytes are in registers now
+                        // one arrival per warp: 512 arrivals on one mbarrier serialise
+                        __syncwarp();
+                        if (lane == 0)
+                            mbar_arrive(pempty(it));   // the warp's packed bytes are in registers now
                         dq_store(v, cur.s, cur.z, w_addr(it) + (uint32_t)r * 128, r7, qtr * 2);
                         fence_proxy_async_smem();
-                        mbar_arrive(wfull(it));
+                        __syncwarp();
+                        if (lane == 0)
+                            mbar_arrive(wfull(it));
                     }
                 }
             }
