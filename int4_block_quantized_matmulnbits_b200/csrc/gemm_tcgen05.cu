@@ -615,7 +615,9 @@ int tune_gemm(int min_bn, int max_split) {
 int read_device_status(unsigned *out, int clear) {
     cudaError_t e = cudaMemcpyFromSymbol(out, g_mnb_status, sizeof(unsigned));
     if (e == cudaSuccess) {
-        const int rc = read_gemv_status(out, clear);
+        int rc = read_gemv_status(out, clear);
+        if (!rc)
+            rc = read_stream_status(out, clear);
         if (rc)
             return rc;
     }

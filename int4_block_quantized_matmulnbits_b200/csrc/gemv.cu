@@ -548,6 +548,10 @@ int sm_count() {
 
 // Which inner product serves fp16 activations at M = 1 and 2: MMA by default.
 static int g_gemv_f16_cc_max_m = 0;
+// 1: fp16 activations go to the warp-specialized streaming kernel for the shapes
+// it serves.  Off by default: on the decoder shapes it is not yet faster than
+// the general TMA kernel.
+static int g_gemv_stream = 0;
 
 // Work decomposition: K slices = W warps x S CTAs per tile, chosen so that
 // about two CTAs of 8 warps per SM have work; rounds of tiles per CTA, with the
@@ -591,8 +595,14 @@ int plan_gemv(int M, int N, int K, int esz, int MP, int sms, Params &p, int &gri
 int launch_gemv(const void *X, int act_f16, const uint8_t *packed, const void *scales,
                 int scale_f16, const uint8_t *zp, void *Y, int M, int N, int K, int bs,
                 unsigned flags, cudaStream_t s) {
-    if (act_f16 && M > g_gemv_f16_cc_max_m)   // tensor-core path, weights streamed by TMA
+    if (act_f16 && M > g_gemv_f16_cc_max_m) {   // tensor-core paths, weights streamed by TMA
+        if (g_gemv_stream) {
+            const int rc = launch_gemv_stream(X, packed, scales, scale_f16, zp, Y, M, N, K, bs, flags, s);
+            if (rc != 1)
+                return rc;
+        }
         return launch_gemv_tc(X, packed, scales, scale_f16, zp, Y, M, N, K, bs, flags, s);
+    }
     const int mode = MODE_CC;
     int MP;
     if (mode == MODE_MMA)
@@ -638,5 +648,14 @@ extern "C" MNB_API int mnb_tune_gemv_f16_cc_max_m(int max_m) {
     if (max_m < 0 || max_m > 2)
         return MNB_ERR_INVALID_ARG;
     mnb::g_gemv_f16_cc_max_m = max_m;
+    return MNB_OK;
+}
+
+// Tuning hook: 0 (default) sends every fp16 GEMV to the general TMA kernel, 1
+// lets the streaming kernel take the shapes it serves.  Not part of the stable ABI.
+extern "C" MNB_API int mnb_tune_gemv_stream(int enable) {
+    if (enable != 0 && enable != 1)
+        return MNB_ERR_INVALID_ARG;
+    mnb::g_gemv_stream = enable;
     return MNB_OK;
 }

@@ -20,6 +20,11 @@ int launch_gemv(const void *X, int act_f16, const uint8_t *packed, const void *s
 int launch_gemv_tc(const void *X, const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,
                    void *Y, int M, int N, int K, int bs, unsigned flags, cudaStream_t s);
 
+// Warp-specialized decode kernel for the shapes it serves (M <= 8, K % 256 == 0,
+// aligned scales); returns 1 without launching anything for other shapes.
+int launch_gemv_stream(const void *X, const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,
+                       void *Y, int M, int N, int K, int bs, unsigned flags, cudaStream_t s);
+
 int launch_gemm(const void *X, const uint8_t *packed, const void *scales, int scale_f16,
                 const uint8_t *zp, void *Y, int M, int N, int K, int bs, unsigned flags,
                 cudaStream_t s);
@@ -29,6 +34,7 @@ int launch_embed_gather(const int8_t *table, const float *row_scales, int64_t V,
                         cudaStream_t s);
 
 int read_device_status(unsigned *out, int clear);
-int read_gemv_status(unsigned *out, int clear);   // ORs the decode kernel's word into *out
+int read_gemv_status(unsigned *out, int clear);     // ORs the decode kernel's word into *out
+int read_stream_status(unsigned *out, int clear);   // same for the streaming decode kernel
 
 }  // namespace mnb

@@ -101,6 +101,16 @@ GEMV_CASES = [
     (16, 2048, 2048, 32, True, "f16", np.float16),
     (16, 48, 64, 32, True, "f16", np.float32),
     (4, 16, 32, 32, True, "f16", np.float16),
+    # shapes the warp-specialized streaming kernel serves (M <= 8, K % 256 == 0)
+    (1, 4096, 2048, 32, True, "f16", np.float16),
+    (1, 2048, 6144, 32, True, "f16", np.float16),
+    (2, 1024, 3072, 32, True, "f16", np.float16),
+    (3, 1000, 1024, 64, False, "f16", np.float32),
+    (8, 777, 512, 32, True, "f16", np.float32),
+    (1, 50, 256, 32, True, "f16", np.float16),
+    (6, 2000, 2048, 64, True, "f16", np.float16),
+    (1, 300, 4096, 64, False, "f16", np.float32),
+    (4, 3333, 1024, 32, False, "f16", np.float16),
 ]
 
 
@@ -117,9 +127,15 @@ def test_gemv_parity(mnb, cuda_dev, M, N, K, bs, has_zp, act, sdt):
     packed, scales, zp = random_packed(rng, N, K, bs, has_zp, sdt)
     tdt = torch.float16 if act == "f16" else torch.float32
     X = torch.randn((M, K), generator=torch.Generator().manual_seed(K)).to(tdt)
-    Y = _run_gemv(mnb, cuda_dev, X.to(cuda_dev), packed, scales, zp, M, N, K, bs)
     ref = oracle.matmul(X.float().numpy(), packed, scales, zp, K, bs)
-    assert_close(np_of(Y.float()), ref, act)
+    # fp16 activations: the general TMA kernel, then the streaming kernel where it applies
+    for stream in ((0, 1) if act == "f16" else (0,)):
+        assert mnb._lib.mnb_tune_gemv_stream(stream) == 0
+        try:
+            Y = _run_gemv(mnb, cuda_dev, X.to(cuda_dev), packed, scales, zp, M, N, K, bs)
+        finally:
+            mnb._lib.mnb_tune_gemv_stream(0)
+        assert_close(np_of(Y.float()), ref, act)
 
 
 @pytest.mark.parametrize("M", [1, 2])
@@ -137,8 +153,32 @@ def test_gemv_f16_cuda_core_variant(mnb, cuda_dev, M):
     assert_close(np_of(Y.float()), ref, "f16")
 
 
-def test_gemv_q_equal_zp_gives_exact_zero(mnb, cuda_dev):
-    N, K, bs, M = 64, 256, 32, 3
+@pytest.mark.parametrize("M,N,K,bs,has_zp,sdt", [(1, 2048, 2048, 32, True, np.float16),
+                                                  (5, 1040, 2048, 32, True, np.float16),
+                                                  (8, 512, 1024, 64, False, np.float32),
+                                                  (1, 160, 6144, 64, False, np.float16),
+                                                  (2, 1024, 3072, 32, True, np.float16)])
+def test_gemv_streaming_and_general_kernels_agree(mnb, cuda_dev, M, N, K, bs, has_zp, sdt):
+    # the same call through the streaming decode kernel and through the general
+    # TMA decode kernel: both against the oracle, and close to each other
+    rng = np.random.default_rng(N + K + M)
+    packed, scales, zp = random_packed(rng, N, K, bs, has_zp, sdt)
+    X = torch.randn((M, K), generator=torch.Generator().manual_seed(M)).half()
+    ref = oracle.matmul(X.float().numpy(), packed, scales, zp, K, bs)
+    out = {}
+    for enable in (1, 0):
+        assert mnb._lib.mnb_tune_gemv_stream(enable) == 0
+        try:
+            out[enable] = _run_gemv(mnb, cuda_dev, X.to(cuda_dev), packed, scales, zp, M, N, K, bs)
+        finally:
+            mnb._lib.mnb_tune_gemv_stream(0)
+        assert_close(np_of(out[enable].float()), ref, "f16")
+    assert_close(np_of(out[1].float()), np_of(out[0].float()), "f16")
+
+
+@pytest.mark.parametrize("N,K", [(64, 256), (80, 1024)])
+def test_gemv_q_equal_zp_gives_exact_zero(mnb, cuda_dev, N, K):
+    bs, M = 32, 3
     z = np.random.default_rng(1).integers(0, 16, (N, K // bs))
     q = np.repeat(z, bs, axis=1)
     packed = (q[:, 0::2] | (q[:, 1::2] << 4)).astype(np.uint8)
