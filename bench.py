@@ -36,6 +36,18 @@ WORKLOAD = ("qwen3-1.7b-shaped decode step, M=1: 28 layers x (q 2048->2048, k/v 
             "int4 block 32 asymmetric, fp16 activations and scales, weights N(0,0.02) with 1% outliers x8")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# DRAM bytes (read + write) per launch from ncu captures of the current kernels
+# (dram__bytes_read.sum + dram__bytes_write.sum): the decode GEMV averaged over
+# the 197 launches of a decode step, the GEMM on the layer-0 q projection at
+# M = 1024.  Set to None when a kernel changes.
+NCU_TRAFFIC = {"gemv_tc_kernel": 5080621, "gemm_kernel": 6682624}
+
+
+def job_gbs(world, bytes_per_rank, ms_max):
+    """Whole-job throughput: every rank streams bytes_per_rank in the timed step,
+    and the step takes the slowest rank's time."""
+    return world * bytes_per_rank / (ms_max * 1e-3) / 1e9
+
 
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -258,14 +270,16 @@ class OracleSample:
         self.oracle.matmul(X, pk, sc, zp, K, self.bs)
         return nbytes, time.perf_counter() - t0
 
-    def measure(self, reps):
-        """GB/s over `reps` passes of the whole layer."""
+    def measure_for(self, seconds):
+        """GB/s over whole passes of the layer until `seconds` of oracle time."""
         tot_b = tot_t = 0.0
-        for r in range(reps):
+        reps = 0
+        while tot_t < seconds:
             for i in range(len(self.items)):
                 b, t = self.run(i)
                 tot_b, tot_t = tot_b + b, tot_t + t
-        return tot_b / tot_t / 1e9, tot_t
+            reps += 1
+        return tot_b / tot_t / 1e9, tot_t, reps
 
 
 # --------------------------------------------------------------------------- arms
@@ -358,7 +372,7 @@ def run_gpu(args, world, rank, local):
         return
     ms = ms_total / args.steps
     wbytes = dec.weight_bytes
-    value = world * wbytes / (ms * 1e-3) / 1e9
+    value = job_gbs(world, wbytes, ms)
     per_launch_bytes = wbytes / len(lins)
     per_launch_us = ms * 1000.0 / len(lins)
     achieved = per_launch_bytes / (per_launch_us * 1e-6) / 1e9
@@ -388,7 +402,7 @@ def run_gpu(args, world, rank, local):
     lm_gbs = lm.nbytes / (lm_ms * 1e-3) / 1e9
 
     e2e_ms, h2d, d2h = timed_e2e(dec, max(10, args.steps // 4), max(3, args.warmup), ranks)
-    e2e_val = world * wbytes / (e2e_ms * 1e-3) / 1e9
+    e2e_val = job_gbs(world, wbytes, e2e_ms)
 
     # decode at larger M (same weights)
     by_m = {}
@@ -428,10 +442,10 @@ def run_gpu(args, world, rank, local):
     cpu = None
     if rank == 0 and world == 1:
         sample = OracleSample()
-        gbs, dt = sample.measure(3)
+        gbs, dt, reps = sample.measure_for(10.0)
         cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": sample.cores, "kind": "oracle",
                "sample": f"oracle.matmul over the 7 projections of layer 0 of the decode step at M=1, "
-                         f"3 passes, {dt:.1f} s wall on {sample.cores} threads"}
+                         f"{reps} passes, {dt:.1f} s wall on {sample.cores} threads"}
 
     if rank == 0:
         out = {
@@ -443,8 +457,9 @@ def run_gpu(args, world, rank, local):
                        "weight_bytes_per_step": wbytes, "graph": True, "pdl": True,
                        "l2": "inputs larger than L2 (weights of one step > 126 MB)",
                        "parallelism": f"replicas x{world}"},
-            "roofline": {"bound": "hbm", "kernel": "gemv_kernel", "achieved": round(achieved, 1), "peak": hbm,
-                         "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": None,
+            "roofline": {"bound": "hbm", "kernel": "gemv_tc_kernel", "achieved": round(achieved, 1), "peak": hbm,
+                         "unit": "GB/s", "frac": round(achieved / hbm, 4),
+                         "traffic": NCU_TRAFFIC["gemv_tc_kernel"],
                          "peak_source": f"{peak_src} hbm_gbs", "bytes_per_launch": round(per_launch_bytes),
                          "us_per_launch": round(per_launch_us, 3)},
             "lm_head_alone": {"bytes": lm.nbytes, "us": round(lm_ms * 1000, 2), "gbs": round(lm_gbs, 1),
@@ -454,7 +469,8 @@ def run_gpu(args, world, rank, local):
             "prefill": prefill,
             "roofline_prefill": {"bound": "tensor", "kernel": "gemm_kernel", "M": 1024,
                                  "achieved": prefill["1024"]["tflops"], "peak": tc_sust, "unit": "TFLOP/s",
-                                 "frac": prefill["1024"]["frac_tc_sustained"], "traffic": None,
+                                 "frac": prefill["1024"]["frac_tc_sustained"],
+                                 "traffic": NCU_TRAFFIC["gemm_kernel"], "traffic_of": "layer-0 q projection",
                                  "peak_source": f"{peak_src} bf16_tflops_sustained (fp16 = bf16 nominal rate)"},
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_val, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,

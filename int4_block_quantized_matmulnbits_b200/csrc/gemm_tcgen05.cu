@@ -9,7 +9,7 @@
 // (BN <= 256), so ragged token counts only pad N.
 //
 // Per CTA, a K loop over 64-wide stages fed by three shared-memory rings (packed
-// weights 8 deep, X tiles up to 8 deep, fp16 weight tiles 3 deep), so the long
+// weights 8 deep, X tiles up to 8 deep, fp16 weight tiles 4 deep), so the long
 // DRAM latency of the weight stream is covered without holding X or fp16 space:
 //   warp 0      TMA producer of the packed weight tile (128 rows x 32 bytes) of
 //               every stage; it never waits for the previous kernel, whose
@@ -19,12 +19,12 @@
 //               after griddepcontrol.wait.
 //   warp 1      MMA issuer: one thread issues 4 x tcgen05.mma (K = 16 each) per
 //               stage and commits to the X and fp16-weight "empty" barriers.
-//   warps 3-18  dequant: four threads per weight row, 16 k each per stage: 8
-//               packed bytes from shared memory -> 16 fp16 = fp16_rn((q - zp) *
-//               scale), written in the 128-byte-swizzled K-major layout the MMA
-//               descriptor reads, then fence.proxy.async, __syncwarp and one
-//               mbarrier arrival per warp.
-//               Sixteen warps so that the unpack's dependency chains overlap.
+//   warps 3-18  dequant, in two groups of eight that take alternate stages (two
+//               stages are unpacked at once): two threads per weight row, 32 k
+//               each per stage: 16 packed bytes from shared memory -> 32 fp16 =
+//               fp16_rn((q - zp) * scale), written in the 128-byte-swizzled
+//               K-major layout the MMA descriptor reads, then fence.proxy.async,
+//               __syncwarp and one mbarrier arrival per warp.
 //               Scales and zero points run a few stages ahead in registers.
 //               After the K loop the same warps are the epilogue: tcgen05.ld of
 //               their 32 TMEM lanes, fp16 conversion, stores of Y.
@@ -54,7 +54,7 @@ constexpr int kBK = 64;                        // k per stage (128 bytes of fp16
 constexpr int kWBytes = kBM * 128;             // fp16 weight tile per stage
 constexpr int kPBytes = kBM * 32;              // packed weight tile per stage
 constexpr int kPR = 4;                         // stages of scales / zero points prefetched
-constexpr int kWS = 3;                         // fp16 weight tiles in the ring
+constexpr int kWS = 4;                         // fp16 weight tiles in the ring
 constexpr int kPS = 8;                         // packed weight tiles in flight
 constexpr int kMaxCluster = 8;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
@@ -158,7 +158,8 @@ __device__ __forceinline__ float4 ld_dsmem_f4(const float *local, uint32_t rank)
     return v;
 }
 
-// Scale (fp16 bits) and zero point of one thread's 16-k quarter of a stage.
+// Scale (fp16 bits) and zero point of one thread's 32-k half of a stage (one
+// block of 32, or half a block of 64).
 struct SZ {
     uint32_t s, z;
 };
@@ -254,10 +255,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
         for (int i = 0; i < PS; i++) {
             mbar_init(pfull(i), 1);
-            mbar_init(pempty(i), kDqWarps);
+            mbar_init(pempty(i), kDqWarps / 2);   // the 8 warps of the group that unpacks it
         }
         for (int i = 0; i < WS; i++) {
-            mbar_init(wfull(i), kDqWarps);
+            mbar_init(wfull(i), kDqWarps / 2);
             mbar_init(wempty(i), 1);
         }
         for (int i = 0; i < XS; i++) {
@@ -337,34 +338,42 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_commit(acc_full);   // fires once every MMA issued above has completed
         __syncwarp();
     } else {
-        // ---------------- dequant: thread = (row r, quarter of the stage's 64 k)
+        // ---------------- dequant: two groups of 8 warps take alternate stages, so
+        // two stages are being unpacked at once; in a group, thread = (row r,
+        // half hh of the stage's 64 k): 16 packed bytes -> 32 fp16
         const int dt = tid - 96;
-        const int r = dt >> 2, qtr = dt & 3;
+        const int dgrp = dt >> 8, t = dt & 255;
+        const int r = t >> 1, hh = t & 1;
         const int n = n_tile * kBM + r;
         const int r7 = r & 7;
         SZ ring[kPR];
 #pragma unroll
-        for (int i = 0; i < kPR; i++)
-            ring[i] = (i < nk) ? load_sz(p, n, kbeg + i * kBK + qtr * 16) : SZ{0u, 8u};
+        for (int i = 0; i < kPR; i++) {
+            const int it = dgrp + 2 * i;
+            ring[i] = (it < nk) ? load_sz(p, n, kbeg + it * kBK + hh * 32) : SZ{0u, 8u};
+        }
         bool ok = true;
-        for (int base_it = 0; base_it < nk && ok; base_it += kPR) {
+        for (int base_j = 0; dgrp + 2 * base_j < nk && ok; base_j += kPR) {
 #pragma unroll
             for (int i = 0; i < kPR; i++) {
-                const int it = base_it + i;
+                const int it = dgrp + 2 * (base_j + i);
                 if (it < nk && ok) {
                     // warp-uniform outcome, so the warp stays converged for __syncwarp
                     ok = __all_sync(0xffffffffu, mbar_wait(pfull(it), (it / PS) & 1, abort) &&
                                                      (it < WS || mbar_wait(wempty(it), ((it / WS) - 1) & 1, abort)));
                     if (ok) {
                         const SZ cur = ring[i];
-                        if (it + kPR < nk)
-                            ring[i] = load_sz(p, n, kbeg + (it + kPR) * kBK + qtr * 16);
-                        const uint2 v = *reinterpret_cast<const uint2 *>(base_ptr + p_off(it) + r * 32 + qtr * 8);
-                        // one arrival per warp: 512 arrivals on one mbarrier serialise
+                        const int nxt = it + 2 * kPR;
+                        if (nxt < nk)
+                            ring[i] = load_sz(p, n, kbeg + nxt * kBK + hh * 32);
+                        const uint4 v = *reinterpret_cast<const uint4 *>(base_ptr + p_off(it) + r * 32 + hh * 16);
+                        // one arrival per warp: hundreds of arrivals on one mbarrier serialise
                         __syncwarp();
                         if (lane == 0)
                             mbar_arrive(pempty(it));   // the warp's packed bytes are in registers now
-                        dq_store(v, cur.s, cur.z, w_addr(it) + (uint32_t)r * 128, r7, qtr * 2);
+                        const uint32_t row_addr = w_addr(it) + (uint32_t)r * 128;
+                        dq_store(make_uint2(v.x, v.y), cur.s, cur.z, row_addr, r7, hh * 4);
+                        dq_store(make_uint2(v.z, v.w), cur.s, cur.z, row_addr, r7, hh * 4 + 2);
                         fence_proxy_async_smem();
                         __syncwarp();
                         if (lane == 0)
@@ -534,9 +543,9 @@ int launch_gemm(const void *X, const uint8_t *packed, const void *scales, int sc
     p.tmem_cols = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
     p.S = S;
     p.kslice = kslice;
-    // rings: 3 fp16 weight tiles, 8 packed tiles, as many X tiles as fit (<= 8)
+    // rings: 4 fp16 weight tiles, 8 packed tiles, as many X tiles as fit (<= 8)
     const int fixed = kWS * kWBytes + kPS * kPBytes;
-    int xstages = (200 * 1024 - fixed) / (BN * 128);
+    int xstages = (224 * 1024 - fixed) / (BN * 128);
     if (xstages > 8) xstages = 8;
     if (xstages < 2) xstages = 2;
     const size_t ring_bytes = (size_t)fixed + (size_t)xstages * BN * 128;
@@ -545,6 +554,8 @@ int launch_gemm(const void *X, const uint8_t *packed, const void *scales, int sc
         return fail(MNB_ERR_SHAPE, "mnb_gemm: reduction buffer does not fit");
     p.xstages = xstages;
     const size_t smem = 1024 + ring_bytes + 8 * (2 * kPS + 2 * kWS + 2 * xstages + 1) + 16;
+    if (smem > 232448)
+        return fail(MNB_ERR_SHAPE, "mnb_gemm: shared memory plan too large");
 
     CUtensorMap xmap, wmap;
     {
