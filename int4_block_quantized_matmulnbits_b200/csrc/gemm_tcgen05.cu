@@ -498,6 +498,7 @@ EncodeTiledFn get_encode_fn() {
 
 // Tile policy knobs (tuning hooks, see mnb_tune_gemm below).
 static int g_gemm_min_bn = 128;      // smallest token tile the grid heuristic may pick
+static int g_gemm_max_bn = 256;      // largest token tile
 static int g_gemm_max_split = kMaxCluster;
 
 int launch_gemm(const void *X, const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,
@@ -514,7 +515,7 @@ int launch_gemm(const void *X, const uint8_t *packed, const void *scales, int sc
 
     // token tiling: as few tiles of <= 256 as possible, evenly sized; narrower
     // tiles (down to g_gemm_min_bn) while the grid would leave half the SMs idle
-    int mt = (M + 255) / 256;
+    int mt = (M + g_gemm_max_bn - 1) / g_gemm_max_bn;
     int BN = ((M + mt - 1) / mt + 15) / 16 * 16;
     const int n_tiles = N / kBM;
     while (BN > g_gemm_min_bn && BN > 16 && (int64_t)n_tiles * mt * 4 <= sms) {
@@ -615,10 +616,11 @@ int launch_gemm(const void *X, const uint8_t *packed, const void *scales, int sc
     return MNB_OK;
 }
 
-int tune_gemm(int min_bn, int max_split) {
-    if (min_bn < 16 || min_bn > 256 || max_split < 1 || max_split > kMaxCluster)
+int tune_gemm(int min_bn, int max_bn, int max_split) {
+    if (min_bn < 16 || max_bn > 256 || min_bn > max_bn || max_split < 1 || max_split > kMaxCluster)
         return MNB_ERR_INVALID_ARG;
     g_gemm_min_bn = min_bn;
+    g_gemm_max_bn = max_bn;
     g_gemm_max_split = max_split;
     return MNB_OK;
 }
@@ -643,6 +645,12 @@ int read_device_status(unsigned *out, int clear) {
 
 }  // namespace mnb
 
-// Tuning hook: smallest token tile the tile heuristic may choose (16..256) and
-// the largest cluster split along K (1..8).  Not part of the stable ABI.
-extern "C" MNB_API int mnb_tune_gemm(int min_bn, int max_split) { return mnb::tune_gemm(min_bn, max_split); }
+// Tuning hooks: smallest (and largest) token tile the tile heuristic may choose
+// (16..256) and the largest cluster split along K (1..8).  Not part of the
+// stable ABI.
+extern "C" MNB_API int mnb_tune_gemm(int min_bn, int max_split) {
+    return mnb::tune_gemm(min_bn, min_bn > mnb::g_gemm_max_bn ? min_bn : mnb::g_gemm_max_bn, max_split);
+}
+extern "C" MNB_API int mnb_tune_gemm_tiles(int min_bn, int max_bn, int max_split) {
+    return mnb::tune_gemm(min_bn, max_bn, max_split);
+}
