@@ -393,6 +393,17 @@ def run_gpu(args, world, rank, local):
              "frac_hbm": round(wbytes / (f_ms * 1e-3) / 1e9 / hbm, 4), "clocks": fclk.summary()}
     del fdec
 
+    # the same step ending in greedy decoding: the lm_head launch also picks the
+    # token (mnb_gemv_argmax), as a decoder's step does
+    gdec = Pass(lins, 1, "gemv", torch.float16, pdl=True, greedy=True)
+    fill(gdec, cfg["seed"])
+    gdec.capture()
+    g_ms = timed_replays(gdec, max(10, args.steps // 4), args.warmup, ranks, "decode_greedy") / max(10, args.steps // 4)
+    greedy = {"launches_per_step": len(lins), "us_per_step": round(g_ms * 1000, 2),
+              "weight_gbs": round(job_gbs(world, wbytes, g_ms), 1),
+              "frac_hbm": round(wbytes / (g_ms * 1e-3) / 1e9 / hbm, 4)}
+    del gdec
+
     # lm_head alone: one 180 MB launch, the kernel without launch gaps
     lm = lins[-1]
     lmp = Pass([lm], 1, "gemv", torch.float16, pdl=False)
@@ -400,6 +411,11 @@ def run_gpu(args, world, rank, local):
     lmp.capture()
     lm_ms = timed_replays(lmp, 50, 5, ranks) / 50
     lm_gbs = lm.nbytes / (lm_ms * 1e-3) / 1e9
+    lmg = Pass([lm], 1, "gemv", torch.float16, pdl=False, greedy=True)
+    fill(lmg, cfg["seed"] + 5)
+    lmg.capture()
+    lmg_ms = timed_replays(lmg, 50, 5, ranks) / 50
+    del lmg
 
     e2e_ms, h2d, d2h = timed_e2e(dec, max(10, args.steps // 4), max(3, args.warmup), ranks)
     e2e_val = job_gbs(world, wbytes, e2e_ms)
@@ -463,7 +479,9 @@ def run_gpu(args, world, rank, local):
                          "peak_source": f"{peak_src} hbm_gbs", "bytes_per_launch": round(per_launch_bytes),
                          "us_per_launch": round(per_launch_us, 3)},
             "lm_head_alone": {"bytes": lm.nbytes, "us": round(lm_ms * 1000, 2), "gbs": round(lm_gbs, 1),
-                              "frac_hbm": round(lm_gbs / hbm, 4)},
+                              "frac_hbm": round(lm_gbs / hbm, 4),
+                              "us_with_greedy_argmax": round(lmg_ms * 1000, 2)},
+            "decode_greedy": greedy,
             "decode_fused_qkv_gateup": fused,
             "decode_by_M": by_m,
             "prefill": prefill,

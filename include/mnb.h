@@ -129,6 +129,27 @@ MNB_API int mnb_gemv(const void *X, mnb_dtype act_t, const uint8_t *packed, cons
              mnb_dtype scale_t, const uint8_t *zp, void *Y, int64_t M, int64_t N, int64_t K,
              int bs, unsigned flags, void *stream);
 
+/* The output projection of a decode step fused with greedy decoding
+ * ("Qwen3-ASR-0.6B -- ONNX for the browser", "Building the prompt" step 5:
+ * greedy decode with decoder_step, logits [1, 1, 151936]).  Computes Y exactly
+ * as mnb_gemv (fp16 activations) and, for every token m,
+ *   ids[m]     = the smallest n with Y[m][n] = max_n' Y[m][n']  (the fp16 values
+ *                written to Y; the first maximum on ties),
+ *   max_out[m] = that maximum as fp32 (max_out may be NULL).
+ *   1 <= M <= 16, N >= 1.  ids (int32 [M]) and max_out are device pointers.
+ *   workspace: device buffer of at least mnb_gemv_argmax_workspace_bytes(M)
+ *   bytes (for the current device), 16-byte aligned, ZERO-FILLED before its
+ *   first use.  Its first bytes count the CTAs that finished; the last one
+ *   sets the count back to zero, so a workspace stays usable across calls; the
+ *   rest is scratch.  Calls that share a workspace must not run concurrently
+ *   on the GPU.
+ * Errors: MNB_ERR_INVALID_ARG (also: workspace too small), MNB_ERR_SHAPE,
+ *         MNB_ERR_ALIGN, MNB_ERR_UNSUPPORTED (M outside [1, 16]), MNB_ERR_CUDA. */
+MNB_API size_t mnb_gemv_argmax_workspace_bytes(int64_t M);   /* 0 when M is outside [1, 16] */
+MNB_API int mnb_gemv_argmax(const void *X, const uint8_t *packed, const void *scales, mnb_dtype scale_t,
+                    const uint8_t *zp, void *Y, int64_t M, int64_t N, int64_t K, int bs, int32_t *ids,
+                    float *max_out, void *workspace, size_t ws_bytes, unsigned flags, void *stream);
+
 /* Prefill-shaped MatMulNBits on the tensor cores, any M >= 1 (tuned for
  * M >= 64: the full-length prefill of "Mega-ASR -- INT4 ONNX", "What's in this
  * repo": decoder_prefill).  Y = X . dequant(W)^T with fp16 X and Y; each

@@ -22,6 +22,7 @@ __all__ = [
     "MnbError", "MNB_F32", "MNB_F16", "MNB_FLAG_PDL", "lib_path",
     "mnb_last_error", "mnb_version", "mnb_packed_sizes", "mnb_quantize_rtn", "mnb_dequantize",
     "mnb_gemv", "mnb_gemm", "mnb_embed_gather", "mnb_device_status",
+    "mnb_gemv_argmax", "mnb_gemv_argmax_workspace_bytes",
 ]
 
 MNB_F32, MNB_F16 = 0, 1
@@ -58,6 +59,8 @@ def _load():
         "mnb_gemm": ([vp, i32, vp, vp, i32, vp, vp, i64, i64, i64, i32, u32, vp], i32),
         "mnb_embed_gather": ([vp, vp, i64, i64, vp, i64, vp, i32, vp, vp], i32),
         "mnb_device_status": ([P(u32), i32], i32),
+        "mnb_gemv_argmax_workspace_bytes": ([i64], sz),
+        "mnb_gemv_argmax": ([vp, vp, vp, i32, vp, vp, i64, i64, i64, i32, vp, vp, vp, sz, u32, vp], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -133,6 +136,19 @@ def mnb_gemv(X, packed, scales, zp, Y, M, N, K, bs, flags=0, stream=None):
     _check("mnb_gemv", _lib.mnb_gemv(
         _ptr(X), _dt(X), _ptr(packed), _ptr(scales), _dt(scales), _ptr(zp), _ptr(Y),
         M, N, K, bs, flags, _stream(stream)))
+
+
+def mnb_gemv_argmax_workspace_bytes(M) -> int:
+    """Bytes of workspace mnb_gemv_argmax needs for M tokens on the current device."""
+    return _lib.mnb_gemv_argmax_workspace_bytes(M)
+
+
+def mnb_gemv_argmax(X, packed, scales, zp, Y, M, N, K, bs, ids, max_out, workspace, flags=0, stream=None):
+    """Y as mnb_gemv (fp16 X), plus ids[m] = first argmax of Y[m] and max_out[m] its value.
+    workspace: a zero-filled uint8 device tensor of mnb_gemv_argmax_workspace_bytes(M) bytes."""
+    _check("mnb_gemv_argmax", _lib.mnb_gemv_argmax(
+        _ptr(X), _ptr(packed), _ptr(scales), _dt(scales), _ptr(zp), _ptr(Y), M, N, K, bs, _ptr(ids),
+        _ptr(max_out), _ptr(workspace), workspace.numel() * workspace.element_size(), flags, _stream(stream)))
 
 
 def mnb_gemm(X, packed, scales, zp, Y, M, N, K, bs, flags=0, stream=None):

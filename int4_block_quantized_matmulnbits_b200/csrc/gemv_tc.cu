@@ -51,6 +51,13 @@ constexpr int kBoxBytes = kRows * 128;     // 16 rows x 128 packed bytes
 constexpr int kDepth = 4;                  // boxes in flight per warp
 constexpr int kMaxCluster = 8;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+constexpr size_t kArgmaxWsHeader = 256;    // the CTA counter, then the per-CTA partials
+
+struct ArgmaxArgs {
+    int32_t *ids;
+    float *max_out;
+    void *workspace;
+};
 
 struct TcParams {
     const void *X;
@@ -68,6 +75,12 @@ struct TcParams {
     int xs_stride;    // bytes per token row of staged X
     int ntiles;       // ceil(N / 16)
     int independent;  // W == 1 && S == 1: each warp walks tiles on its own
+    // greedy decoding (independent mode only): ids[m] = first n of max Y[m][n]
+    int argmax;
+    int *ids;             // [M]
+    float *max_out;       // [M] or null
+    uint2 *ws_part;       // [gridDim.x][M] (value bits, index) per CTA
+    unsigned *ws_count;   // CTAs done; the last one resets it to 0
 };
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -214,6 +227,96 @@ __device__ __forceinline__ void dq_word(uint32_t w, uint32_t s2, uint32_t Z, uin
     a3 = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(w8, 0x00F000F0u, 0x64006400u)), u32_as_h2(Zhi)), s));
 }
 
+// (value, index) pairs ordered by value, then by the SMALLER index: the greedy
+// token is the first maximum.
+__device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
+    return v > bv || (v == bv && i < bi);
+}
+
+__device__ __forceinline__ void warp_best(float &v, int &i, unsigned mask_lanes) {
+    for (unsigned o = 16; o >= 1; o >>= 1) {
+        if (!(mask_lanes & o))
+            continue;
+        const float ov = __shfl_xor_sync(0xffffffffu, v, (int)o);
+        const int oi = __shfl_xor_sync(0xffffffffu, i, (int)o);
+        if (better(ov, oi, v, i)) {
+            v = ov;
+            i = oi;
+        }
+    }
+}
+
+// Greedy decoding epilogue: the warp's best per token (lanes with one c hold
+// one token pair), then the CTA's, parked in the workspace; the last CTA to
+// finish reduces all CTAs' partials and resets the counter.
+template <int NT>
+__device__ void argmax_finish(const TcParams &p, float (&best_v)[NT][2], int (&best_i)[NT][2], uint2 *sb, int warp,
+                              int lane, int g, int c, int tid) {
+#pragma unroll
+    for (int t = 0; t < NT; t++)
+#pragma unroll
+        for (int jj = 0; jj < 2; jj++) {
+            float v = best_v[t][jj];
+            int i = best_i[t][jj];
+            warp_best(v, i, 4u | 8u | 16u);   // over g: the 8 lanes that share c
+            const int m = 8 * t + 2 * c + jj;
+            if (g == 0 && m < p.M)
+                sb[warp * 16 + m] = make_uint2(__float_as_uint(v), (unsigned)i);
+        }
+    __syncthreads();
+    __shared__ int s_last;
+    if (tid < p.M) {
+        float v = -INFINITY;
+        int i = 0x7fffffff;
+        for (int w = 0; w < kWarps; w++) {
+            const uint2 e = sb[w * 16 + tid];
+            if (better(__uint_as_float(e.x), (int)e.y, v, i)) {
+                v = __uint_as_float(e.x);
+                i = (int)e.y;
+            }
+        }
+        p.ws_part[(size_t)blockIdx.x * p.M + tid] = make_uint2(__float_as_uint(v), (unsigned)i);
+        __threadfence();
+    }
+    __syncthreads();
+    if (tid == 0)
+        s_last = (atomicAdd(p.ws_count, 1u) == gridDim.x - 1);
+    __syncthreads();
+    if (!s_last)
+        return;
+    __threadfence();
+    for (int m = 0; m < p.M; m++) {
+        float v = -INFINITY;
+        int i = 0x7fffffff;
+        for (int b = tid; b < (int)gridDim.x; b += kThreads) {
+            const uint2 e = __ldcg(p.ws_part + (size_t)b * p.M + m);
+            if (better(__uint_as_float(e.x), (int)e.y, v, i)) {
+                v = __uint_as_float(e.x);
+                i = (int)e.y;
+            }
+        }
+        warp_best(v, i, 31u);
+        __syncthreads();   // sb is reused per token
+        if (lane == 0)
+            sb[warp] = make_uint2(__float_as_uint(v), (unsigned)i);
+        __syncthreads();
+        if (tid == 0) {
+            for (int w = 1; w < kWarps; w++) {
+                const uint2 e = sb[w];
+                if (better(__uint_as_float(e.x), (int)e.y, v, i)) {
+                    v = __uint_as_float(e.x);
+                    i = (int)e.y;
+                }
+            }
+            p.ids[m] = i;
+            if (p.max_out)
+                p.max_out[m] = v;
+        }
+    }
+    if (tid == 0)
+        *p.ws_count = 0u;   // ready for the next call
+}
+
 template <int NT, class C>
 __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_constant__ CUtensorMap wmap,
                                                               const TcParams p) {
@@ -313,6 +416,15 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
 
     bool dead = false;
     int tile = first_tile, j = 0, r = 0;
+    float best_v[NT][2];   // greedy decoding: the lane's best logit so far for tokens 8t + 2c + jj
+    int best_i[NT][2];
+#pragma unroll
+    for (int t = 0; t < NT; t++)
+#pragma unroll
+        for (int jj = 0; jj < 2; jj++) {
+            best_v[t][jj] = -INFINITY;
+            best_i[t][jj] = 0x7fffffff;
+        }
     ParamCursor pc;
     param_tile<C>(p, pc, tile, g, kw + c * 64);
     ChunkParams pa = params_at<C>(p, pc, 0), pb = params_at<C>(p, pc, 1);   // one box ahead
@@ -389,8 +501,15 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
                 for (int e = 0; e < 4; e++) {
                     const int m = 8 * t + 2 * c + (e & 1);
                     const int n = n0 + 8 * (e >> 1);
-                    if (m < p.M && n < p.N)
-                        p.Y[(int64_t)m * p.N + n] = __float2half_rn(out[t][e]);
+                    if (m < p.M && n < p.N) {
+                        const __half h = __float2half_rn(out[t][e]);
+                        p.Y[(int64_t)m * p.N + n] = h;
+                        if (p.argmax)   // rows ascend within a lane: '>' keeps the first maximum
+                            if (__half2float(h) > best_v[t][e & 1]) {
+                                best_v[t][e & 1] = __half2float(h);
+                                best_i[t][e & 1] = n;
+                            }
+                    }
                 }
         } else {
 #pragma unroll
@@ -431,6 +550,9 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
 #pragma unroll
             for (int e = 0; e < 8; e++) acc[t][e >> 2][e & 3] = 0.f;
     }
+
+    if (p.argmax)
+        argmax_finish<NT>(p, best_v, best_i, reinterpret_cast<uint2 *>(red), warp, lane, g, c, tid);
 
     // every issued box was waited for above; after a timeout, let the copies
     // still in flight land before the CTA's shared memory is released
@@ -511,8 +633,10 @@ int launch_tc(const CUtensorMap &map, const TcParams &p, int grid, size_t smem, 
 
 }  // namespace
 
-int launch_gemv_tc(const void *X, const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,
-                   void *Y, int M, int N, int K, int bs, unsigned flags, cudaStream_t s) {
+// Shared by mnb_gemv (am == nullptr) and mnb_gemv_argmax.
+static int launch_tc_common(const void *X, const uint8_t *packed, const void *scales, int scale_f16,
+                            const uint8_t *zp, void *Y, int M, int N, int K, int bs, unsigned flags,
+                            cudaStream_t s, const ArgmaxArgs *am) {
     EncodeTiledFn encode = encode_fn();
     if (!encode)
         return fail(MNB_ERR_CUDA, "mnb_gemv: cuTensorMapEncodeTiled unavailable");
@@ -529,10 +653,17 @@ int launch_gemv_tc(const void *X, const uint8_t *packed, const void *scales, int
     p.scale_f16 = scale_f16;
     p.scale_pair = (scale_f16 && bs == 32 && (p.nb % 2) == 0 && (reinterpret_cast<uintptr_t>(scales) % 4) == 0);
     p.ntiles = (N + kRows - 1) / kRows;
+    p.argmax = am ? 1 : 0;
+    p.ids = am ? am->ids : nullptr;
+    p.max_out = am ? am->max_out : nullptr;
+    p.ws_part = am ? reinterpret_cast<uint2 *>(static_cast<unsigned char *>(am->workspace) + kArgmaxWsHeader) : nullptr;
+    p.ws_count = am ? static_cast<unsigned *>(am->workspace) : nullptr;
 
     // K slices: W warps x S CTAs per tile, enough for ~16 warps on every SM
     const int nbx_all = (K + kBoxK - 1) / kBoxK;
     int slices = (sms * 2 * kWarps + p.ntiles - 1) / p.ntiles;
+    if (am)
+        slices = 1;   // greedy decoding runs in independent mode: whole rows per warp
     if (slices > nbx_all) slices = nbx_all;
     if (slices > kWarps * kMaxCluster) slices = kWarps * kMaxCluster;
     if (slices < 1) slices = 1;
@@ -598,6 +729,23 @@ int launch_gemv_tc(const void *X, const uint8_t *packed, const void *scales, int
 #undef MNB_TC_Z
 #undef MNB_TC_S
 #undef MNB_TC
+}
+
+int launch_gemv_tc(const void *X, const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,
+                   void *Y, int M, int N, int K, int bs, unsigned flags, cudaStream_t s) {
+    return launch_tc_common(X, packed, scales, scale_f16, zp, Y, M, N, K, bs, flags, s, nullptr);
+}
+
+size_t gemv_argmax_workspace_bytes(int M) {
+    // one (value, index) pair per token per CTA; at most two CTAs per SM
+    return kArgmaxWsHeader + (size_t)2 * sm_count_tc() * (size_t)M * sizeof(uint2);
+}
+
+int launch_gemv_argmax(const void *X, const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,
+                       void *Y, int M, int N, int K, int bs, int32_t *ids, float *max_out, void *workspace,
+                       unsigned flags, cudaStream_t s) {
+    ArgmaxArgs am{ids, max_out, workspace};
+    return launch_tc_common(X, packed, scales, scale_f16, zp, Y, M, N, K, bs, flags, s, &am);
 }
 
 int read_gemv_status(unsigned *out, int clear) {

@@ -25,6 +25,12 @@ int launch_gemv_tc(const void *X, const uint8_t *packed, const void *scales, int
 int launch_gemv_stream(const void *X, const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,
                        void *Y, int M, int N, int K, int bs, unsigned flags, cudaStream_t s);
 
+// Decode GEMV fused with greedy decoding (first maximum of each token's fp16 logits).
+size_t gemv_argmax_workspace_bytes(int M);
+int launch_gemv_argmax(const void *X, const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,
+                       void *Y, int M, int N, int K, int bs, int32_t *ids, float *max_out, void *workspace,
+                       unsigned flags, cudaStream_t s);
+
 int launch_gemm(const void *X, const uint8_t *packed, const void *scales, int scale_f16,
                 const uint8_t *zp, void *Y, int M, int N, int K, int bs, unsigned flags,
                 cudaStream_t s);

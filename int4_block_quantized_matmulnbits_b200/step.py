@@ -12,8 +12,8 @@ from __future__ import annotations
 
 import torch
 
-from . import (MNB_FLAG_PDL, mnb_dequantize, mnb_embed_gather, mnb_gemm, mnb_gemv,
-               mnb_packed_sizes, mnb_quantize_rtn)
+from . import (MNB_FLAG_PDL, mnb_dequantize, mnb_embed_gather, mnb_gemm, mnb_gemv, mnb_gemv_argmax,
+               mnb_gemv_argmax_workspace_bytes, mnb_packed_sizes, mnb_quantize_rtn)
 
 
 class QLinear:
@@ -42,6 +42,10 @@ class QLinear:
 
     def gemv(self, X, Y, flags=0, stream=None):
         mnb_gemv(X, self.packed, self.scales, self.zp, Y, X.shape[0], self.N, self.K, self.bs, flags, stream)
+
+    def gemv_argmax(self, X, Y, ids, max_out, workspace, flags=0, stream=None):
+        mnb_gemv_argmax(X, self.packed, self.scales, self.zp, Y, X.shape[0], self.N, self.K, self.bs, ids, max_out,
+                        workspace, flags, stream)
 
     def gemm(self, X, Y, flags=0, stream=None):
         mnb_gemm(X, self.packed, self.scales, self.zp, Y, X.shape[0], self.N, self.K, self.bs, flags, stream)
@@ -91,7 +95,7 @@ class Pass:
     gather of M token ids runs first, as in a decode step.
     """
 
-    def __init__(self, linears, M, kind="gemv", act_dtype=torch.float16, pdl=True, embed=None):
+    def __init__(self, linears, M, kind="gemv", act_dtype=torch.float16, pdl=True, embed=None, greedy=False):
         self.linears, self.M, self.kind, self.pdl = list(linears), M, kind, pdl
         dev = self.linears[0].packed.device
         # one flat buffer each for all inputs and all outputs (views per linear,
@@ -110,6 +114,12 @@ class Pass:
             assert t.data_ptr() % 16 == 0
         self.embed = embed   # (table, row_scales, ids[M], out[M, D]) or None
         self.graph = None
+        # greedy=True: the last linear (the lm_head) also picks each token's id
+        self.greedy = greedy and kind == "gemv"
+        if self.greedy:
+            self.ids = torch.zeros((M,), dtype=torch.int32, device=dev)
+            self.max_out = torch.zeros((M,), dtype=torch.float32, device=dev)
+            self.ws = torch.zeros((mnb_gemv_argmax_workspace_bytes(M),), dtype=torch.uint8, device=dev)
 
     @property
     def weight_bytes(self):
@@ -129,9 +139,13 @@ class Pass:
             mnb_embed_gather(table, rs, table.shape[0], table.shape[1], ids, ids.shape[0], out,
                              None, stream)
         flags = MNB_FLAG_PDL if self.pdl else 0
-        for l, x, y in zip(self.linears, self.X, self.Y):
+        last = len(self.linears) - 1
+        for i, (l, x, y) in enumerate(zip(self.linears, self.X, self.Y)):
             if self.kind == "gemv":
-                l.gemv(x, y, flags, stream)
+                if self.greedy and i == last:
+                    l.gemv_argmax(x, y, self.ids, self.max_out, self.ws, flags, stream)
+                else:
+                    l.gemv(x, y, flags, stream)
             else:
                 l.gemm(x, y, flags, stream)
 

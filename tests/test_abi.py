@@ -114,3 +114,25 @@ def test_binding_raises_with_message(mnb):
     with pytest.raises(mnb.MnbError) as e:
         mnb.mnb_packed_sizes(4, 100, 32)
     assert "MNB_ERR_SHAPE" in str(e.value) and "K=100" in str(e.value)
+
+
+def test_gemv_argmax_argument_checks(lib):
+    fake = ctypes.c_void_p(1 << 20)   # aligned, never dereferenced: every call below fails its checks
+    ws = lib.mnb_gemv_argmax_workspace_bytes
+    ws.restype, ws.argtypes = ctypes.c_size_t, [ctypes.c_int64]
+    assert ws(0) == 0 and ws(17) == 0 and ws(1) > 0 and ws(16) > ws(1)
+    f = lib.mnb_gemv_argmax
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] + [ctypes.c_void_p] * 2 + [ctypes.c_int64] * 3 + \
+        [ctypes.c_int] + [ctypes.c_void_p] * 3 + [ctypes.c_size_t, ctypes.c_uint, ctypes.c_void_p]
+    need = ws(1)
+    # M outside [1, 16]
+    assert f(fake, fake, fake, 1, fake, fake, 17, 256, 512, 32, fake, None, fake, ws(16), 0, None) == -4
+    # NULL ids
+    assert f(fake, fake, fake, 1, fake, fake, 1, 256, 512, 32, None, None, fake, need, 0, None) == -1
+    # workspace too small
+    assert f(fake, fake, fake, 1, fake, fake, 1, 256, 512, 32, fake, None, fake, need - 1, 0, None) == -1
+    assert b"workspace" in lib.mnb_last_error()
+    # misaligned workspace
+    assert f(fake, fake, fake, 1, fake, fake, 1, 256, 512, 32, fake, None, ctypes.c_void_p((1 << 20) + 4), need, 0,
+             None) == -3

@@ -241,6 +241,67 @@ def test_gemv_pdl_chain_and_graph_match_eager(mnb, cuda_dev):
     assert_close(np_of(bufs_plain[0].float()), r0, "f16")
 
 
+# ------------------------------------------------------------------ GEMV + greedy argmax
+
+ARGMAX_CASES = [
+    # M, N, K, bs, has_zp, scale
+    (1, 151936, 2048, 32, True, np.float16),   # the 1.7B lm_head
+    (4, 5000, 1024, 64, True, np.float16),
+    (3, 777, 512, 32, False, np.float32),
+    (16, 1000, 2048, 32, True, np.float16),
+    (8, 33, 256, 32, True, np.float16),
+]
+
+
+def _run_argmax(mnb, dev, X, packed, scales, zp, M, N, K, bs, ws=None):
+    Y = torch.empty((M, N), dtype=torch.float16, device=dev)
+    ids = torch.full((M,), -1, dtype=torch.int32, device=dev)
+    mx = torch.empty((M,), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = torch.zeros(mnb.mnb_gemv_argmax_workspace_bytes(M), dtype=torch.uint8, device=dev)
+    mnb.mnb_gemv_argmax(X, to_dev(packed, dev), to_dev(scales, dev), to_dev(zp, dev), Y, M, N, K, bs, ids, mx, ws)
+    torch.cuda.synchronize()
+    return Y, ids, mx, ws
+
+
+@pytest.mark.parametrize("M,N,K,bs,has_zp,sdt", ARGMAX_CASES)
+def test_gemv_argmax(mnb, cuda_dev, M, N, K, bs, has_zp, sdt):
+    rng = np.random.default_rng(N + M)
+    packed, scales, zp = random_packed(rng, N, K, bs, has_zp, sdt)
+    X = torch.randn((M, K), generator=torch.Generator().manual_seed(N)).half()
+    Y, ids, mx, ws = _run_argmax(mnb, cuda_dev, X.to(cuda_dev), packed, scales, zp, M, N, K, bs)
+    ref = oracle.matmul(X.float().numpy(), packed, scales, zp, K, bs)
+    y = np_of(Y.float())
+    assert_close(y, ref, "f16")
+    ids_np, mx_np = np_of(ids), np_of(mx)
+    # the token is the first maximum of the logits the kernel wrote ...
+    assert np.array_equal(ids_np, np.argmax(y, axis=1))
+    assert np.array_equal(mx_np, y[np.arange(M), ids_np])
+    # ... and a valid greedy choice for the exact logits
+    assert np.all(ref[np.arange(M), ids_np] >= ref.max(axis=1) - 2e-2)
+    # the workspace counter is back at zero, so the same workspace serves again
+    assert int(np_of(ws[:4].view(torch.int32))[0]) == 0
+    Y2, ids2, mx2, _ = _run_argmax(mnb, cuda_dev, X.to(cuda_dev), packed, scales, zp, M, N, K, bs, ws)
+    assert torch.equal(ids2, ids) and torch.equal(Y2, Y) and torch.equal(mx2, mx)
+
+
+def test_gemv_argmax_ties_take_the_first_row(mnb, cuda_dev):
+    N, K, bs, M = 300, 512, 32, 2
+    rng = np.random.default_rng(5)
+    packed = np.zeros((N, K // 2), np.uint8)
+    zp = np.full((N, K // bs // 2), 0x88, np.uint8)      # zp = 8 in every block
+    packed[:] = 0x88                                     # q = zp: logit exactly 0 for rows 0..99
+    row = rng.integers(0, 256, K // 2, dtype=np.uint8)
+    packed[100:] = row                                   # rows 100..299 identical
+    scales = np.full((N, K // bs), 0.25, np.float16)
+    X = torch.randn((M, K), generator=torch.Generator().manual_seed(11)).half()
+    Y, ids, _, _ = _run_argmax(mnb, cuda_dev, X.to(cuda_dev), packed, scales, zp, M, N, K, bs)
+    y = np_of(Y.float())
+    for m in range(M):
+        assert np.all(y[m, 100:] == y[m, 100])
+        assert int(np_of(ids)[m]) == (100 if y[m, 100] > 0 else 0)
+
+
 # ------------------------------------------------------------------ GEMM (tcgen05)
 
 GEMM_CASES = [
