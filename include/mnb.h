@@ -150,6 +150,27 @@ MNB_API int mnb_gemv_argmax(const void *X, const uint8_t *packed, const void *sc
                     const uint8_t *zp, void *Y, int64_t M, int64_t N, int64_t K, int bs, int32_t *ids,
                     float *max_out, void *workspace, size_t ws_bytes, unsigned flags, void *stream);
 
+/* mnb_gemv_argmax without a workspace argument.  No counterpart on the pages:
+ * it is for callers that cannot hand this library device memory -- a plug-in
+ * whose host application owns every device allocation through its own pool,
+ * or a decode loop on a latency-critical thread that must not call the device
+ * allocator (which can block, or fail for lack of memory, between two tokens).
+ * Same arguments and results as mnb_gemv_argmax, minus workspace/ws_bytes.
+ * The scratch is a device array inside libmnb.so: 64 KiB on every GPU that
+ * loads the library, held until the process exits.  With 148 SMs that covers
+ * every M in [1, 16]; a request needing more returns MNB_ERR_SHAPE with a
+ * message.  Nothing is allocated: the first call on each device looks up the
+ * array's device address (make that first call before any stream capture),
+ * and each call clears the array's counter on `stream` before its kernel.
+ * All calls on one GPU share the one array, which keeps the last call's
+ * contents: calls that may run at the same time on the GPU (other streams,
+ * other host threads) race on it and must be serialized by the caller.
+ * Errors: MNB_ERR_INVALID_ARG, MNB_ERR_SHAPE, MNB_ERR_ALIGN,
+ *         MNB_ERR_UNSUPPORTED (M outside [1, 16]), MNB_ERR_CUDA. */
+MNB_API int mnb_gemv_argmax_noalloc(const void *X, const uint8_t *packed, const void *scales, mnb_dtype scale_t,
+                            const uint8_t *zp, void *Y, int64_t M, int64_t N, int64_t K, int bs,
+                            int32_t *ids, float *max_out, unsigned flags, void *stream);
+
 /* Prefill-shaped MatMulNBits on the tensor cores, any M >= 1 (tuned for
  * M >= 64: the full-length prefill of "Mega-ASR -- INT4 ONNX", "What's in this
  * repo": decoder_prefill).  Y = X . dequant(W)^T with fp16 X and Y; each

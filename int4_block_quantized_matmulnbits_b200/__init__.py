@@ -22,7 +22,7 @@ __all__ = [
     "MnbError", "MNB_F32", "MNB_F16", "MNB_FLAG_PDL", "lib_path",
     "mnb_last_error", "mnb_version", "mnb_packed_sizes", "mnb_quantize_rtn", "mnb_dequantize",
     "mnb_gemv", "mnb_gemm", "mnb_embed_gather", "mnb_device_status",
-    "mnb_gemv_argmax", "mnb_gemv_argmax_workspace_bytes",
+    "mnb_gemv_argmax", "mnb_gemv_argmax_workspace_bytes", "mnb_gemv_argmax_noalloc",
 ]
 
 MNB_F32, MNB_F16 = 0, 1
@@ -61,6 +61,7 @@ def _load():
         "mnb_device_status": ([P(u32), i32], i32),
         "mnb_gemv_argmax_workspace_bytes": ([i64], sz),
         "mnb_gemv_argmax": ([vp, vp, vp, i32, vp, vp, i64, i64, i64, i32, vp, vp, vp, sz, u32, vp], i32),
+        "mnb_gemv_argmax_noalloc": ([vp, vp, vp, i32, vp, vp, i64, i64, i64, i32, vp, vp, u32, vp], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -149,6 +150,15 @@ def mnb_gemv_argmax(X, packed, scales, zp, Y, M, N, K, bs, ids, max_out, workspa
     _check("mnb_gemv_argmax", _lib.mnb_gemv_argmax(
         _ptr(X), _ptr(packed), _ptr(scales), _dt(scales), _ptr(zp), _ptr(Y), M, N, K, bs, _ptr(ids),
         _ptr(max_out), _ptr(workspace), workspace.numel() * workspace.element_size(), flags, _stream(stream)))
+
+
+def mnb_gemv_argmax_noalloc(X, packed, scales, zp, Y, M, N, K, bs, ids, max_out, flags=0, stream=None):
+    """mnb_gemv_argmax with its scratch in a device array held by the library:
+    for callers that cannot provide device memory.  Calls that may overlap on
+    the GPU share that array and must be serialized."""
+    _check("mnb_gemv_argmax_noalloc", _lib.mnb_gemv_argmax_noalloc(
+        _ptr(X), _ptr(packed), _ptr(scales), _dt(scales), _ptr(zp), _ptr(Y), M, N, K, bs, _ptr(ids),
+        _ptr(max_out), flags, _stream(stream)))
 
 
 def mnb_gemm(X, packed, scales, zp, Y, M, N, K, bs, flags=0, stream=None):

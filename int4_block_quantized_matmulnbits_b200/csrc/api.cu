@@ -188,6 +188,28 @@ int mnb_gemv_argmax(const void *X, const uint8_t *packed, const void *scales, mn
                               max_out, workspace, flags, (cudaStream_t)stream);
 }
 
+int mnb_gemv_argmax_noalloc(const void *X, const uint8_t *packed, const void *scales, mnb_dtype scale_t,
+                            const uint8_t *zp, void *Y, int64_t M, int64_t N, int64_t K, int bs, int32_t *ids,
+                            float *max_out, unsigned flags, void *stream) {
+    clear_error();
+    const char *fn = "mnb_gemv_argmax_noalloc";
+    int rc = check_matmul_args(fn, X, MNB_F16, packed, scales, scale_t, Y, M, N, K, bs);
+    if (rc)
+        return rc;
+    if (M < 1 || M > 16)
+        return fail(MNB_ERR_UNSUPPORTED, "%s: M=%lld outside [1, 16]", fn, (long long)M);
+    if (N < 1)
+        return fail(MNB_ERR_SHAPE, "%s: N must be positive", fn);
+    if (flags & ~(unsigned)MNB_FLAG_PDL)
+        return fail(MNB_ERR_INVALID_ARG, "%s: unknown flags 0x%x", fn, flags);
+    if (!ids)
+        return fail(MNB_ERR_INVALID_ARG, "%s: NULL ids", fn);
+    if (!aligned(ids, 4) || !aligned(max_out, 4))
+        return fail(MNB_ERR_ALIGN, "%s: ids and max_out need 4-byte alignment", fn);
+    return launch_gemv_argmax_noalloc(X, packed, scales, scale_t == MNB_F16, zp, Y, (int)M, (int)N, (int)K, bs,
+                                      ids, max_out, flags, (cudaStream_t)stream);
+}
+
 int mnb_gemm(const void *X, mnb_dtype act_t, const uint8_t *packed, const void *scales,
              mnb_dtype scale_t, const uint8_t *zp, void *Y, int64_t M, int64_t N, int64_t K,
              int bs, unsigned flags, void *stream) {

@@ -34,6 +34,8 @@
 // failure in a device status word, drains its copies and exits.
 #include <cuda.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -745,6 +747,59 @@ int launch_gemv_argmax(const void *X, const uint8_t *packed, const void *scales,
                        void *Y, int M, int N, int K, int bs, int32_t *ids, float *max_out, void *workspace,
                        unsigned flags, cudaStream_t s) {
     ArgmaxArgs am{ids, max_out, workspace};
+    return launch_tc_common(X, packed, scales, scale_f16, zp, Y, M, N, K, bs, flags, s, &am);
+}
+
+// ---- greedy decoding without a caller-provided workspace -------------------
+//
+// The scratch of mnb_gemv_argmax_noalloc lives in this module-scope device
+// array: every GPU that loads the library holds these 64 KiB until the process
+// exits, and every call on that GPU shares them.  Host code must not hand the
+// array's name to a kernel (on the host it is only a stand-in for the symbol):
+// the first call on each device asks the runtime for the array's device
+// address, with that device current, and later calls reuse it.
+constexpr size_t kNoAllocScratchBytes = 64 * 1024;
+static __device__ __align__(256) unsigned char g_argmax_scratch[kNoAllocScratchBytes];
+
+static int noalloc_scratch_ptr(void **out) {
+    static std::mutex mu;
+    static void *ptrs[128] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return fail(MNB_ERR_CUDA, "mnb_gemv_argmax_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= 128)
+        return fail(MNB_ERR_UNSUPPORTED, "mnb_gemv_argmax_noalloc: device ordinal %d", dev);
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ptrs[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_argmax_scratch);
+        if (e != cudaSuccess || !p)
+            return fail(MNB_ERR_CUDA, "mnb_gemv_argmax_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+        ptrs[dev] = p;
+    }
+    *out = ptrs[dev];
+    return MNB_OK;
+}
+
+size_t gemv_argmax_noalloc_capacity() { return kNoAllocScratchBytes; }
+
+int launch_gemv_argmax_noalloc(const void *X, const uint8_t *packed, const void *scales, int scale_f16,
+                               const uint8_t *zp, void *Y, int M, int N, int K, int bs, int32_t *ids,
+                               float *max_out, unsigned flags, cudaStream_t s) {
+    const size_t need = gemv_argmax_workspace_bytes(M);
+    if (need > kNoAllocScratchBytes)
+        return fail(MNB_ERR_SHAPE, "mnb_gemv_argmax_noalloc: M=%d needs %zu bytes of scratch, the library holds %zu",
+                    M, need, kNoAllocScratchBytes);
+    void *scratch = nullptr;
+    int rc = noalloc_scratch_ptr(&scratch);
+    if (rc)
+        return rc;
+    // the CTA counter must start at zero; a call cut short could have left it set
+    cudaError_t e = cudaMemsetAsync(scratch, 0, kArgmaxWsHeader, s);
+    if (e != cudaSuccess)
+        return fail(MNB_ERR_CUDA, "mnb_gemv_argmax_noalloc: clearing the scratch counter: %s", cudaGetErrorString(e));
+    ArgmaxArgs am{ids, max_out, scratch};
     return launch_tc_common(X, packed, scales, scale_f16, zp, Y, M, N, K, bs, flags, s, &am);
 }
 

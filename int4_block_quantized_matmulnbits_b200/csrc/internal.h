@@ -31,6 +31,12 @@ int launch_gemv_argmax(const void *X, const uint8_t *packed, const void *scales,
                        void *Y, int M, int N, int K, int bs, int32_t *ids, float *max_out, void *workspace,
                        unsigned flags, cudaStream_t s);
 
+// The same with the scratch in a library-owned device array (no allocation).
+size_t gemv_argmax_noalloc_capacity();
+int launch_gemv_argmax_noalloc(const void *X, const uint8_t *packed, const void *scales, int scale_f16,
+                               const uint8_t *zp, void *Y, int M, int N, int K, int bs, int32_t *ids,
+                               float *max_out, unsigned flags, cudaStream_t s);
+
 int launch_gemm(const void *X, const uint8_t *packed, const void *scales, int scale_f16,
                 const uint8_t *zp, void *Y, int M, int N, int K, int bs, unsigned flags,
                 cudaStream_t s);
