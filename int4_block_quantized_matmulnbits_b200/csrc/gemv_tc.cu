@@ -635,6 +635,9 @@ int launch_tc(const CUtensorMap &map, const TcParams &p, int grid, size_t smem, 
 
 }  // namespace
 
+// Tuning hook state: a forced K split (0 = the planner decides).
+static int g_force_w = 0, g_force_s = 1;
+
 // Shared by mnb_gemv (am == nullptr) and mnb_gemv_argmax.
 static int launch_tc_common(const void *X, const uint8_t *packed, const void *scales, int scale_f16,
                             const uint8_t *zp, void *Y, int M, int N, int K, int bs, unsigned flags,
@@ -661,29 +664,75 @@ static int launch_tc_common(const void *X, const uint8_t *packed, const void *sc
     p.ws_part = am ? reinterpret_cast<uint2 *>(static_cast<unsigned char *>(am->workspace) + kArgmaxWsHeader) : nullptr;
     p.ws_count = am ? static_cast<unsigned *>(am->workspace) : nullptr;
 
-    // K slices: W warps x S CTAs per tile, enough for ~16 warps on every SM
+    // K split: W warps x S clustered CTAs per 16-row tile.  Each candidate is
+    // costed in box-times on the busiest warp: rounds of tile groups x (boxes
+    // per warp + a per-round reduction cost: none when warps own whole rows,
+    // more when the partial sums meet across a cluster).  Fitted on the
+    // decoder shapes: a cluster split rarely pays.
     const int nbx_all = (K + kBoxK - 1) / kBoxK;
-    int slices = (sms * 2 * kWarps + p.ntiles - 1) / p.ntiles;
-    if (am)
-        slices = 1;   // greedy decoding runs in independent mode: whole rows per warp
-    if (slices > nbx_all) slices = nbx_all;
-    if (slices > kWarps * kMaxCluster) slices = kWarps * kMaxCluster;
-    if (slices < 1) slices = 1;
-    int W = 1;
-    while (W * 2 <= kWarps && W * 2 <= slices) W *= 2;
-    int S = (slices + W - 1) / W;
-    if (S > kMaxCluster) S = kMaxCluster;
+    auto smem_for = [&](int W, int S, int &nbx_w, int &kcta, int &xs_stride) {
+        nbx_w = (nbx_all + W * S - 1) / (W * S);
+        kcta = W * nbx_w * kBoxK;
+        xs_stride = (kcta / kBoxK) * 512 + 64;
+        return 1024 + (size_t)kWarps * kDepth * kBoxBytes + (size_t)M * xs_stride + 512 +
+               (size_t)2 * kWarps * kRows * MP * 4 + (size_t)kWarps * kDepth * 8;
+    };
+    int W = 0, S = 1;
+    double best = 0.0;
+    for (int w = 1; w <= kWarps; w *= 2)
+        for (int sc = 1; sc <= kMaxCluster; sc *= 2) {
+            if ((w * sc > nbx_all && !(w == 1 && sc == 1)) || (am && (w != 1 || sc != 1)))
+                continue;
+            int nbx_w, kcta, xs_stride;
+            const size_t sm_ = smem_for(w, sc, nbx_w, kcta, xs_stride);
+            if (sm_ > 200 * 1024)
+                continue;
+            const int per_sm = (sm_ <= 110 * 1024) ? 2 : 1;
+            double cost;
+            if (w == 1 && sc == 1) {
+                const int warps = sms * per_sm * kWarps;
+                cost = (double)((p.ntiles + warps - 1) / warps) * nbx_all;
+            } else {
+                const int tpc = kWarps / w;
+                const int groups = (p.ntiles + tpc - 1) / tpc;
+                int maxcl = sms * per_sm / sc;
+                if (maxcl < 1) maxcl = 1;
+                const int rounds = (groups + maxcl - 1) / maxcl;
+                cost = rounds * (1.15 * nbx_w + (sc > 1 ? 1.6 : 0.5));
+            }
+            if (W == 0 || cost < best - 1e-9 || (cost < best + 1e-9 && sc < S) ||
+                (cost < best + 1e-9 && sc == S && w > W)) {
+                W = w;
+                S = sc;
+                best = cost;
+            }
+        }
+    if (M > 8 && !am) {
+        // two token groups per MMA: the model above was fitted at M <= 8; here
+        // the split aims at about 16 warps with work on every SM
+        int slices = (sms * 2 * kWarps + p.ntiles - 1) / p.ntiles;
+        if (slices > nbx_all) slices = nbx_all;
+        if (slices > kWarps * kMaxCluster) slices = kWarps * kMaxCluster;
+        if (slices < 1) slices = 1;
+        W = 1;
+        while (W * 2 <= kWarps && W * 2 <= slices) W *= 2;
+        S = (slices + W - 1) / W;
+        if (S > kMaxCluster) S = kMaxCluster;
+        int nbx_w, kcta, xs_stride;
+        while (S < kMaxCluster && smem_for(W, S, nbx_w, kcta, xs_stride) > 200 * 1024)
+            S++;
+    }
+    if (!am && g_force_w > 0) {   // tuning hook
+        W = g_force_w;
+        S = g_force_s;
+    }
+    if (W == 0)
+        return fail(MNB_ERR_SHAPE, "mnb_gemv: K=%d too large for M=%d", K, M);
     size_t smem = 0;
-    for (;; S++) {
-        const int nbx_w = (nbx_all + W * S - 1) / (W * S);
-        p.S = S; p.W = W; p.nbx_w = nbx_w;
-        p.kcta = W * nbx_w * kBoxK;
-        p.xs_stride = (p.kcta / kBoxK) * 512 + 64;
-        smem = 1024 + (size_t)kWarps * kDepth * kBoxBytes + (size_t)M * p.xs_stride +
-               512 + (size_t)2 * kWarps * kRows * MP * 4 +
-               (size_t)kWarps * kDepth * 8;
-        if (smem <= 200 * 1024 || S >= kMaxCluster)
-            break;
+    {
+        int nbx_w, kcta, xs_stride;
+        smem = smem_for(W, S, nbx_w, kcta, xs_stride);
+        p.S = S; p.W = W; p.nbx_w = nbx_w; p.kcta = kcta; p.xs_stride = xs_stride;
     }
     if (smem > 220 * 1024)
         return fail(MNB_ERR_SHAPE, "mnb_gemv: K=%d too large for M=%d", K, M);
@@ -817,3 +866,13 @@ int read_gemv_status(unsigned *out, int clear) {
 }
 
 }  // namespace mnb
+
+// Tuning hook: force the decode kernel's K split to W warps x S clustered CTAs
+// per 16-row tile (w = 0 restores the planner).  Not part of the stable ABI.
+extern "C" MNB_API int mnb_tune_gemv_split(int w, int s) {
+    if (w < 0 || w > 8 || (w & (w - 1)) != 0 || s < 1 || s > 8)
+        return MNB_ERR_INVALID_ARG;
+    mnb::g_force_w = w;
+    mnb::g_force_s = s;
+    return MNB_OK;
+}
