@@ -440,17 +440,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float4 o = own[j];
                     f[4 * j] = o.x; f[4 * j + 1] = o.y; f[4 * j + 2] = o.z; f[4 * j + 3] = o.w;
                 }
-                for (int qq = 0; qq < p.S; qq++) {
-                    if (qq == rank)
-                        continue;
-                    float4 o4[4];
+                // the peers' partials: all loads of a column quad in flight at once,
+                // then the adds (in rank order, so the sum does not depend on timing)
 #pragma unroll
-                    for (int j = 0; j < 4; j++)
-                        o4[j] = ld_dsmem_f4(red + row * red_pitch + c16 * 16 + 4 * j, (uint32_t)qq);
+                for (int j = 0; j < 4; j++) {
+                    float4 o4[kMaxCluster];
 #pragma unroll
-                    for (int j = 0; j < 4; j++) {
-                        f[4 * j] += o4[j].x; f[4 * j + 1] += o4[j].y; f[4 * j + 2] += o4[j].z; f[4 * j + 3] += o4[j].w;
-                    }
+                    for (int qq = 0; qq < kMaxCluster; qq++)
+                        if (qq < p.S && qq != rank)
+                            o4[qq] = ld_dsmem_f4(red + row * red_pitch + c16 * 16 + 4 * j, (uint32_t)qq);
+#pragma unroll
+                    for (int qq = 0; qq < kMaxCluster; qq++)
+                        if (qq < p.S && qq != rank) {
+                            f[4 * j] += o4[qq].x; f[4 * j + 1] += o4[qq].y;
+                            f[4 * j + 2] += o4[qq].z; f[4 * j + 3] += o4[qq].w;
+                        }
                 }
                 store_y(c16 * 16, f);
             }
