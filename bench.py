@@ -393,6 +393,15 @@ def run_gpu(args, world, rank, local):
              "frac_hbm": round(wbytes / (f_ms * 1e-3) / 1e9 / hbm, 4), "clocks": fclk.summary()}
     del fdec
 
+    # the fused layout with the SwiGLU activation in the gate|up launch
+    slins = fuse_decoder(lins, swiglu=True)
+    sdec = Pass(slins, 1, "gemv", torch.float16, pdl=True)
+    fill(sdec, cfg["seed"])
+    sdec.capture()
+    s_ms = timed_replays(sdec, max(10, args.steps // 4), args.warmup, ranks, "decode_swiglu") / max(10, args.steps // 4)
+    fused["with_swiglu_epilogue_us_per_step"] = round(s_ms * 1000, 2)
+    del sdec, slins
+
     # the same step ending in greedy decoding: the lm_head launch also picks the
     # token (mnb_gemv_argmax), as a decoder's step does
     gdec = Pass(lins, 1, "gemv", torch.float16, pdl=True, greedy=True)

@@ -129,6 +129,20 @@ MNB_API int mnb_gemv(const void *X, mnb_dtype act_t, const uint8_t *packed, cons
              mnb_dtype scale_t, const uint8_t *zp, void *Y, int64_t M, int64_t N, int64_t K,
              int bs, unsigned flags, void *stream);
 
+/* Gate and up projections of the decoder's SwiGLU MLP with its activation fused
+ * in ("Qwen3-ASR-1.7B ONNX", "Architecture": Qwen3 decoder with SwiGLU):
+ *   Y[m][i] = silu(G[m][i]) * U[m][i],  G = X . dequant(Wg)^T, U = X . dequant(Wu)^T,
+ *   silu(x) = x / (1 + exp(-x)), from the fp32 sums, rounded once to fp16.
+ * The weight [N][K] holds the gate and up rows interleaved in groups of 16 rows:
+ * rows 16j .. 16j+7 are gate rows 8j .. 8j+7, rows 16j+8 .. 16j+15 the up rows
+ * of the same outputs (scales and zero points follow their rows).  Y is
+ * [M][N/2].  fp16 activations, 1 <= M <= 16, N % 16 == 0.
+ * Errors: MNB_ERR_INVALID_ARG, MNB_ERR_SHAPE, MNB_ERR_ALIGN,
+ *         MNB_ERR_UNSUPPORTED (M > 16), MNB_ERR_CUDA. */
+MNB_API int mnb_gemv_swiglu(const void *X, const uint8_t *packed, const void *scales, mnb_dtype scale_t,
+                    const uint8_t *zp, void *Y, int64_t M, int64_t N, int64_t K, int bs, unsigned flags,
+                    void *stream);
+
 /* The output projection of a decode step fused with greedy decoding
  * ("Qwen3-ASR-0.6B -- ONNX for the browser", "Building the prompt" step 5:
  * greedy decode with decoder_step, logits [1, 1, 151936]).  Computes Y exactly

@@ -22,7 +22,7 @@ __all__ = [
     "MnbError", "MNB_F32", "MNB_F16", "MNB_FLAG_PDL", "lib_path",
     "mnb_last_error", "mnb_version", "mnb_packed_sizes", "mnb_quantize_rtn", "mnb_dequantize",
     "mnb_gemv", "mnb_gemm", "mnb_embed_gather", "mnb_device_status",
-    "mnb_gemv_argmax", "mnb_gemv_argmax_workspace_bytes", "mnb_gemv_argmax_noalloc",
+    "mnb_gemv_argmax", "mnb_gemv_argmax_workspace_bytes", "mnb_gemv_argmax_noalloc", "mnb_gemv_swiglu",
 ]
 
 MNB_F32, MNB_F16 = 0, 1
@@ -60,6 +60,7 @@ def _load():
         "mnb_embed_gather": ([vp, vp, i64, i64, vp, i64, vp, i32, vp, vp], i32),
         "mnb_device_status": ([P(u32), i32], i32),
         "mnb_gemv_argmax_workspace_bytes": ([i64], sz),
+        "mnb_gemv_swiglu": ([vp, vp, vp, i32, vp, vp, i64, i64, i64, i32, u32, vp], i32),
         "mnb_gemv_argmax": ([vp, vp, vp, i32, vp, vp, i64, i64, i64, i32, vp, vp, vp, sz, u32, vp], i32),
         "mnb_gemv_argmax_noalloc": ([vp, vp, vp, i32, vp, vp, i64, i64, i64, i32, vp, vp, u32, vp], i32),
     }
@@ -137,6 +138,13 @@ def mnb_gemv(X, packed, scales, zp, Y, M, N, K, bs, flags=0, stream=None):
     _check("mnb_gemv", _lib.mnb_gemv(
         _ptr(X), _dt(X), _ptr(packed), _ptr(scales), _dt(scales), _ptr(zp), _ptr(Y),
         M, N, K, bs, flags, _stream(stream)))
+
+
+def mnb_gemv_swiglu(X, packed, scales, zp, Y, M, N, K, bs, flags=0, stream=None):
+    """Y [M, N/2] = silu(gate) * up from gate/up rows interleaved in 8-row groups (fp16 X)."""
+    _check("mnb_gemv_swiglu", _lib.mnb_gemv_swiglu(
+        _ptr(X), _ptr(packed), _ptr(scales), _dt(scales), _ptr(zp), _ptr(Y), M, N, K, bs, flags,
+        _stream(stream)))
 
 
 def mnb_gemv_argmax_workspace_bytes(M) -> int:

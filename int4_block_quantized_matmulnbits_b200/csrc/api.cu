@@ -157,6 +157,27 @@ int mnb_gemv(const void *X, mnb_dtype act_t, const uint8_t *packed, const void *
                        (int)N, (int)K, bs, flags, (cudaStream_t)stream);
 }
 
+int mnb_gemv_swiglu(const void *X, const uint8_t *packed, const void *scales, mnb_dtype scale_t,
+                    const uint8_t *zp, void *Y, int64_t M, int64_t N, int64_t K, int bs, unsigned flags,
+                    void *stream) {
+    clear_error();
+    const char *fn = "mnb_gemv_swiglu";
+    int rc = check_matmul_args(fn, X, MNB_F16, packed, scales, scale_t, Y, M, N, K, bs);
+    if (rc)
+        return rc;
+    if (M > 16)
+        return fail(MNB_ERR_UNSUPPORTED, "%s: M=%lld > 16", fn, (long long)M);
+    if (N % 16 != 0)
+        return fail(MNB_ERR_SHAPE, "%s: N=%lld must be a multiple of 16 (8 gate + 8 up rows per group)", fn,
+                    (long long)N);
+    if (flags & ~(unsigned)MNB_FLAG_PDL)
+        return fail(MNB_ERR_INVALID_ARG, "%s: unknown flags 0x%x", fn, flags);
+    if (M == 0 || N == 0)
+        return MNB_OK;
+    return launch_gemv_swiglu(X, packed, scales, scale_t == MNB_F16, zp, Y, (int)M, (int)N, (int)K, bs, flags,
+                              (cudaStream_t)stream);
+}
+
 size_t mnb_gemv_argmax_workspace_bytes(int64_t M) {
     if (M < 1 || M > 16)
         return 0;

@@ -77,6 +77,9 @@ struct TcParams {
     int xs_stride;    // bytes per token row of staged X
     int ntiles;       // ceil(N / 16)
     int independent;  // W == 1 && S == 1: each warp walks tiles on its own
+    // SwiGLU epilogue: weight rows come in 16-row groups of 8 gate rows and the
+    // 8 up rows of the same outputs; Y[m][8t + i] = silu(gate) * up, N / 2 columns
+    int swiglu;
     // greedy decoding (independent mode only): ids[m] = first n of max Y[m][n]
     int argmax;
     int *ids;             // [M]
@@ -228,6 +231,9 @@ __device__ __forceinline__ void dq_word(uint32_t w, uint32_t s2, uint32_t Z, uin
     a2 = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(w8, 0x000F000Fu, 0x64006400u)), u32_as_h2(Z)), s));
     a3 = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(w8, 0x00F000F0u, 0x64006400u)), u32_as_h2(Zhi)), s));
 }
+
+// silu(x) = x * sigmoid(x), in fp32.
+__device__ __forceinline__ float silu(float x) { return x / (1.0f + __expf(-x)); }
 
 // (value, index) pairs ordered by value, then by the SMALLER index: the greedy
 // token is the first maximum.
@@ -503,6 +509,12 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
                 for (int e = 0; e < 4; e++) {
                     const int m = 8 * t + 2 * c + (e & 1);
                     const int n = n0 + 8 * (e >> 1);
+                    if (p.swiglu) {   // lane holds gate (row g) and up (row g + 8) of output 8 tile + g
+                        if (e < 2 && m < p.M && n < p.N)
+                            p.Y[(int64_t)m * (p.N / 2) + tile_done * 8 + g] =
+                                __float2half_rn(silu(out[t][e]) * out[t][e + 2]);
+                        continue;
+                    }
                     if (m < p.M && n < p.N) {
                         const __half h = __float2half_rn(out[t][e]);
                         p.Y[(int64_t)m * p.N + n] = h;
@@ -535,12 +547,20 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
                 for (int idx = tid; idx < TPC * kRows * MP; idx += kThreads) {
                     const int sl = idx / (kRows * MP), jj = idx - sl * kRows * MP;
                     const int row = jj / MP, m = jj - row * MP;
-                    const int n = ((r * p.nclusters + cluster) * TPC + sl) * kRows + row;
-                    if (m >= p.M || n >= p.N)
+                    const int tl = (r * p.nclusters + cluster) * TPC + sl;
+                    const int n = tl * kRows + row;
+                    if (m >= p.M || n >= p.N || (p.swiglu && row >= 8))
                         continue;
                     float v = part[idx];
                     for (int q = 1; q < p.S; q++)
                         v += ld_dsmem_f32(part + idx, (uint32_t)q);
+                    if (p.swiglu) {   // row < 8: the gate; row + 8: its up
+                        float u = part[idx + 8 * MP];
+                        for (int q = 1; q < p.S; q++)
+                            u += ld_dsmem_f32(part + idx + 8 * MP, (uint32_t)q);
+                        p.Y[(int64_t)m * (p.N / 2) + tl * 8 + row] = __float2half_rn(silu(v) * u);
+                        continue;
+                    }
                     p.Y[(int64_t)m * p.N + n] = __float2half_rn(v);
                 }
             }
@@ -641,7 +661,7 @@ static int g_force_w = 0, g_force_s = 1;
 // Shared by mnb_gemv (am == nullptr) and mnb_gemv_argmax.
 static int launch_tc_common(const void *X, const uint8_t *packed, const void *scales, int scale_f16,
                             const uint8_t *zp, void *Y, int M, int N, int K, int bs, unsigned flags,
-                            cudaStream_t s, const ArgmaxArgs *am) {
+                            cudaStream_t s, const ArgmaxArgs *am, int swiglu = 0) {
     EncodeTiledFn encode = encode_fn();
     if (!encode)
         return fail(MNB_ERR_CUDA, "mnb_gemv: cuTensorMapEncodeTiled unavailable");
@@ -658,6 +678,7 @@ static int launch_tc_common(const void *X, const uint8_t *packed, const void *sc
     p.scale_f16 = scale_f16;
     p.scale_pair = (scale_f16 && bs == 32 && (p.nb % 2) == 0 && (reinterpret_cast<uintptr_t>(scales) % 4) == 0);
     p.ntiles = (N + kRows - 1) / kRows;
+    p.swiglu = swiglu;
     p.argmax = am ? 1 : 0;
     p.ids = am ? am->ids : nullptr;
     p.max_out = am ? am->max_out : nullptr;
@@ -785,6 +806,11 @@ static int launch_tc_common(const void *X, const uint8_t *packed, const void *sc
 int launch_gemv_tc(const void *X, const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,
                    void *Y, int M, int N, int K, int bs, unsigned flags, cudaStream_t s) {
     return launch_tc_common(X, packed, scales, scale_f16, zp, Y, M, N, K, bs, flags, s, nullptr);
+}
+
+int launch_gemv_swiglu(const void *X, const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,
+                       void *Y, int M, int N, int K, int bs, unsigned flags, cudaStream_t s) {
+    return launch_tc_common(X, packed, scales, scale_f16, zp, Y, M, N, K, bs, flags, s, nullptr, 1);
 }
 
 size_t gemv_argmax_workspace_bytes(int M) {

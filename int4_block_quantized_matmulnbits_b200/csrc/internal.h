@@ -25,6 +25,10 @@ int launch_gemv_tc(const void *X, const uint8_t *packed, const void *scales, int
 int launch_gemv_stream(const void *X, const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,
                        void *Y, int M, int N, int K, int bs, unsigned flags, cudaStream_t s);
 
+// Decode GEMV with the SwiGLU epilogue over gate/up rows interleaved in 8-row groups.
+int launch_gemv_swiglu(const void *X, const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,
+                       void *Y, int M, int N, int K, int bs, unsigned flags, cudaStream_t s);
+
 // Decode GEMV fused with greedy decoding (first maximum of each token's fp16 logits).
 size_t gemv_argmax_workspace_bytes(int M);
 int launch_gemv_argmax(const void *X, const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,

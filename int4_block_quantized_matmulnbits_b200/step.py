@@ -13,7 +13,7 @@ from __future__ import annotations
 import torch
 
 from . import (MNB_FLAG_PDL, mnb_dequantize, mnb_embed_gather, mnb_gemm, mnb_gemv, mnb_gemv_argmax,
-               mnb_gemv_argmax_workspace_bytes, mnb_packed_sizes, mnb_quantize_rtn)
+               mnb_gemv_argmax_workspace_bytes, mnb_gemv_swiglu, mnb_packed_sizes, mnb_quantize_rtn)
 
 
 class QLinear:
@@ -43,6 +43,9 @@ class QLinear:
     def gemv(self, X, Y, flags=0, stream=None):
         mnb_gemv(X, self.packed, self.scales, self.zp, Y, X.shape[0], self.N, self.K, self.bs, flags, stream)
 
+    def gemv_swiglu(self, X, Y, flags=0, stream=None):
+        mnb_gemv_swiglu(X, self.packed, self.scales, self.zp, Y, X.shape[0], self.N, self.K, self.bs, flags, stream)
+
     def gemv_argmax(self, X, Y, ids, max_out, workspace, flags=0, stream=None):
         mnb_gemv_argmax(X, self.packed, self.scales, self.zp, Y, X.shape[0], self.N, self.K, self.bs, ids, max_out,
                         workspace, flags, stream)
@@ -70,15 +73,40 @@ def concat_linears(parts, name=""):
     return q
 
 
-def fuse_decoder(linears):
-    """Per layer [q, k, v, o, gate, up, down] -> [qkv, o, gate_up, down]; others kept."""
+def swiglu_interleave(gate, up, name=""):
+    """One QLinear [2I, K] for mnb_gemv_swiglu: rows in groups of 16, the 8 gate
+    rows 8j..8j+7 followed by the 8 up rows of the same outputs.  Every stored
+    quantity is per row, so interleaving changes no stored value."""
+    assert gate.N == up.N and gate.K == up.K and gate.bs == up.bs and gate.has_zp == up.has_zp
+    assert gate.N % 8 == 0
+    I = gate.N
+    q = QLinear(2 * I, gate.K, gate.bs, gate.has_zp, gate.scales.dtype, gate.packed.device, name)
+
+    def inter(a, b, out):
+        g = a.reshape(I // 8, 8, *a.shape[1:])
+        u = b.reshape(I // 8, 8, *b.shape[1:])
+        out.copy_(torch.stack([g, u], dim=1).reshape(2 * I, *a.shape[1:]))
+
+    inter(gate.packed, up.packed, q.packed)
+    inter(gate.scales, up.scales, q.scales)
+    if gate.has_zp:
+        inter(gate.zp, up.zp, q.zp)
+    q.swiglu = True   # a decode pass runs it through mnb_gemv_swiglu: N / 2 outputs
+    return q
+
+
+def fuse_decoder(linears, swiglu=False):
+    """Per layer [q, k, v, o, gate, up, down] -> [qkv, o, gate_up, down]; others kept.
+    swiglu=True stores gate/up interleaved for the fused SwiGLU epilogue."""
     out, i = [], 0
     while i < len(linears):
         names = [l.name.rstrip("0123456789") for l in linears[i:i + 7]]
         if names == ["q", "k", "v", "o", "gate", "up", "down"]:
             L = linears[i:i + 7]
             layer = L[0].name[1:]
-            out += [concat_linears(L[0:3], f"qkv{layer}"), L[3], concat_linears(L[4:6], f"gate_up{layer}"), L[6]]
+            gu = swiglu_interleave(L[4], L[5], f"gate_up{layer}") if swiglu else \
+                concat_linears(L[4:6], f"gate_up{layer}")
+            out += [concat_linears(L[0:3], f"qkv{layer}"), L[3], gu, L[6]]
             i += 7
         else:
             out.append(linears[i])
@@ -101,14 +129,14 @@ class Pass:
         # one flat buffer each for all inputs and all outputs (views per linear,
         # 16-byte aligned), so a step's inputs and outputs move in one copy each
         xs = [M * l.K for l in self.linears]
-        ys = [M * l.N for l in self.linears]
+        ys = [M * (l.N // 2 if getattr(l, "swiglu", False) else l.N) for l in self.linears]
         self.x_flat = torch.zeros((sum(xs),), dtype=act_dtype, device=dev)
         self.y_flat = torch.zeros((sum(ys),), dtype=act_dtype, device=dev)
         self.X, self.Y = [], []
         ox = oy = 0
         for l, nx, ny in zip(self.linears, xs, ys):
             self.X.append(self.x_flat[ox:ox + nx].view(M, l.K))
-            self.Y.append(self.y_flat[oy:oy + ny].view(M, l.N))
+            self.Y.append(self.y_flat[oy:oy + ny].view(M, ny // M))
             ox, oy = ox + nx, oy + ny
         for t in self.X + self.Y:
             assert t.data_ptr() % 16 == 0
@@ -144,6 +172,8 @@ class Pass:
             if self.kind == "gemv":
                 if self.greedy and i == last:
                     l.gemv_argmax(x, y, self.ids, self.max_out, self.ws, flags, stream)
+                elif getattr(l, "swiglu", False):
+                    l.gemv_swiglu(x, y, flags, stream)
                 else:
                     l.gemv(x, y, flags, stream)
             else:

@@ -20,6 +20,8 @@ Parity status of each function (what pins it, in ``tests/test_oracle.py``):
   matmul         pinned: exact rational brute force, zero-contribution blocks,
                  block-64 == paired block-32.
   embed_gather   pinned: exact power-of-two scales, bad-id rows, table sizes.
+  swiglu         pinned: closed forms (silu(0) = 0, silu(1) = 1/(1 + 1/e),
+                 silu(x) - silu(-x) = x, the large-|x| limits).
 """
 from __future__ import annotations
 
@@ -135,6 +137,15 @@ def matmul(X, packed, scales, zp, K, bs, cols=None):
     if rc != 0:
         raise ValueError("bad shape or column index")
     return Y
+
+
+def swiglu(gate, up):
+    """silu(gate) * up in float64 (the SwiGLU activation of a Qwen3 MLP:
+    "Qwen3-ASR-1.7B ONNX", "Architecture"), silu(x) = x / (1 + exp(-x))."""
+    g = np.asarray(gate, np.float64)
+    u = np.asarray(up, np.float64)
+    with np.errstate(over="ignore"):
+        return g / (1.0 + np.exp(-g)) * u
 
 
 def embed_gather(table, row_scales, ids, out_dtype=np.float16):

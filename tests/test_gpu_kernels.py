@@ -241,6 +241,57 @@ def test_gemv_pdl_chain_and_graph_match_eager(mnb, cuda_dev):
     assert_close(np_of(bufs_plain[0].float()), r0, "f16")
 
 
+# ------------------------------------------------------------------ GEMV + SwiGLU epilogue
+
+def _interleave8(g, u):
+    """Rows in groups of 16: 8 gate rows, then the 8 up rows of the same outputs."""
+    I = g.shape[0]
+    return np.stack([g.reshape(I // 8, 8, *g.shape[1:]), u.reshape(I // 8, 8, *u.shape[1:])],
+                    axis=1).reshape(2 * I, *g.shape[1:])
+
+
+@pytest.mark.parametrize("M,I,K,bs,has_zp,sdt", [(1, 6144, 2048, 32, True, np.float16),
+                                                 (4, 3072, 1024, 32, True, np.float16),
+                                                 (16, 1000, 1024, 64, True, np.float32),
+                                                 (3, 8, 256, 32, False, np.float16),
+                                                 (2, 1024, 6144, 32, True, np.float16)])
+def test_gemv_swiglu(mnb, cuda_dev, M, I, K, bs, has_zp, sdt):
+    rng = np.random.default_rng(I + K + M)
+    pg, sg, zg = random_packed(rng, I, K, bs, has_zp, sdt)
+    pu, su, zu = random_packed(rng, I, K, bs, has_zp, sdt)
+    X = torch.randn((M, K), generator=torch.Generator().manual_seed(I)).half()
+    ref = oracle.swiglu(oracle.matmul(X.float().numpy(), pg, sg, zg, K, bs),
+                        oracle.matmul(X.float().numpy(), pu, su, zu, K, bs))
+    packed, scales = _interleave8(pg, pu), _interleave8(sg, su)
+    zp = _interleave8(zg, zu) if has_zp else None
+    Y = torch.empty((M, I), dtype=torch.float16, device=cuda_dev)
+    mnb.mnb_gemv_swiglu(X.to(cuda_dev), to_dev(packed, cuda_dev), to_dev(scales, cuda_dev), to_dev(zp, cuda_dev), Y,
+                        M, 2 * I, K, bs)
+    torch.cuda.synchronize()
+    assert_close(np_of(Y.float()), ref, "f16")
+
+
+def test_gemv_swiglu_layout_helper(mnb, cuda_dev):
+    from int4_block_quantized_matmulnbits_b200.step import QLinear, swiglu_interleave
+
+    K, I, M = 2048, 6144, 1
+    g = QLinear.quantize(workloads.weight(2, 0, 4, I, K, outliers=True).to(cuda_dev), 32)
+    u = QLinear.quantize(workloads.weight(2, 0, 5, I, K, outliers=True).to(cuda_dev), 32)
+    gu = swiglu_interleave(g, u)
+    X = workloads.activations(2, M, K).to(cuda_dev)
+    Y = torch.empty((M, I), dtype=torch.float16, device=cuda_dev)
+    gu.gemv_swiglu(X, Y)
+    yg = torch.empty((M, I), dtype=torch.float16, device=cuda_dev)
+    yu = torch.empty((M, I), dtype=torch.float16, device=cuda_dev)
+    g.gemv(X, yg)
+    u.gemv(X, yu)
+    torch.cuda.synchronize()
+    ref = oracle.swiglu(oracle.matmul(X.float().cpu().numpy(), np_of(g.packed), np_of(g.scales), np_of(g.zp), K, 32),
+                        oracle.matmul(X.float().cpu().numpy(), np_of(u.packed), np_of(u.scales), np_of(u.zp), K, 32))
+    assert_close(np_of(Y.float()), ref, "f16")
+    assert_close(np_of(Y.float()), oracle.swiglu(np_of(yg.float()), np_of(yu.float())), "f16")
+
+
 # ------------------------------------------------------------------ GEMV + greedy argmax
 
 ARGMAX_CASES = [

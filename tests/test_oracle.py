@@ -381,3 +381,17 @@ def test_embed_fp16_is_rounded_from_the_fp32_product():
     prod = table[ids].astype(np.float32) * scales[ids][:, None]      # numpy's fp32 product
     assert np.array_equal(o32, prod)
     assert np.array_equal(o16, prod.astype(np.float16))
+
+
+def test_swiglu_closed_forms():
+    # silu(x) = x * sigmoid(x): zero at 0, 1/(1 + 1/e) at 1, odd part x, limits x and 0
+    x = np.array([0.0, 1.0, -1.0, 2.5, -2.5, 40.0, -40.0])
+    ones = np.ones_like(x)
+    s = oracle.swiglu(x, ones)
+    assert s[0] == 0.0
+    assert abs(s[1] - 1.0 / (1.0 + np.exp(-1.0))) < 1e-15
+    assert abs(s[1] - 0.7310585786300049) < 1e-15
+    assert np.allclose(s[1::2][:3] - s[2::2][:3], x[1::2][:3], rtol=0, atol=1e-14)
+    assert abs(s[5] - 40.0) < 1e-15 and abs(s[6]) < 1e-15
+    # the up factor multiplies
+    assert np.allclose(oracle.swiglu(x, 3.0 * ones), 3.0 * s, rtol=1e-15, atol=0)
