@@ -503,7 +503,9 @@ EncodeTiledFn get_encode_fn() {
 // Tile policy knobs (tuning hooks, see mnb_tune_gemm below).
 static int g_gemm_min_bn = 128;      // smallest token tile the grid heuristic may pick
 static int g_gemm_max_bn = 256;      // largest token tile
-static int g_gemm_max_split = kMaxCluster;
+// at most 4 CTAs per cluster: 8-CTA clusters of ~200 KB each wait for 8 free
+// SMs of one GPC and measured up to 2x slower, never faster
+static int g_gemm_max_split = 4;
 
 int launch_gemm(const void *X, const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,
                 void *Y, int M, int N, int K, int bs, unsigned flags, cudaStream_t s) {
