@@ -380,6 +380,11 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
         }
     }
     __syncwarp();
+    // the first box's scales and zero points are weights too: fetch them before
+    // waiting for the previous kernel, so their latency overlaps the wait
+    ParamCursor pc;
+    param_tile<C>(p, pc, first_tile, g, kw + c * 64);
+    ChunkParams pa = params_at<C>(p, pc, 0), pb = params_at<C>(p, pc, 1);   // one box ahead
     pdl_launch_dependents();
     pdl_wait();
 
@@ -433,9 +438,6 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
             best_v[t][jj] = -INFINITY;
             best_i[t][jj] = 0x7fffffff;
         }
-    ParamCursor pc;
-    param_tile<C>(p, pc, tile, g, kw + c * 64);
-    ChunkParams pa = params_at<C>(p, pc, 0), pb = params_at<C>(p, pc, 1);   // one box ahead
     for (int pos = 0; pos < total; pos++) {
         int ntile = tile, nj = j + 1;
         if (nj == p.nbx_w) { nj = 0; ntile += tile_stride; }
