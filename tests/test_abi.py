@@ -136,3 +136,12 @@ def test_gemv_argmax_argument_checks(lib):
     # misaligned workspace
     assert f(fake, fake, fake, 1, fake, fake, 1, 256, 512, 32, fake, None, ctypes.c_void_p((1 << 20) + 4), need, 0,
              None) == -3
+
+
+def test_gemv_swiglu_argument_checks(lib):
+    f = lib.mnb_gemv_swiglu
+    assert f(A, A, A, F16, A, A, 17, 64, 64, 32, 0, None) == UNSUPPORTED      # M > 16
+    assert f(A, A, A, F16, A, A, 1, 72, 64, 32, 0, None) == SHAPE            # N % 16
+    assert f(A, A, A, F16, A, A, 1, 64, 96, 64, 0, None) == SHAPE            # K % bs
+    assert f(A, A, A, F16, A, A, 1, 64, 64, 32, 0x80, None) == INVALID       # unknown flag
+    assert f(A, A, A, F16, A, A, 0, 64, 64, 32, 0, None) == OK               # M = 0
