@@ -527,6 +527,40 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
                             }
                     }
                 }
+        } else if (p.S == 1) {
+            // one CTA per tile group: the W partial sums of each output meet in a
+            // shared buffer that alternates between rounds (red, part), so one
+            // barrier per round suffices
+            float *rb = (r & 1) ? part : red;
+#pragma unroll
+            for (int t = 0; t < NT; t++) {
+                const int m0 = 8 * t + 2 * c;
+                rb[(warp * kRows + g) * MP + m0] = out[t][0];
+                rb[(warp * kRows + g) * MP + m0 + 1] = out[t][1];
+                rb[(warp * kRows + g + 8) * MP + m0] = out[t][2];
+                rb[(warp * kRows + g + 8) * MP + m0 + 1] = out[t][3];
+            }
+            __syncthreads();
+            for (int idx = tid; idx < TPC * kRows * MP; idx += kThreads) {
+                const int sl = idx / (kRows * MP), jj = idx - sl * kRows * MP;
+                const int row = jj / MP, m = jj - row * MP;
+                const int tl = (r * p.nclusters + cluster) * TPC + sl;
+                const int n = tl * kRows + row;
+                if (m >= p.M || n >= p.N || (p.swiglu && row >= 8))
+                    continue;
+                const float *src = rb + (sl * W * kRows) * MP + jj;
+                float v = 0.f;
+                for (int q = 0; q < W; q++)
+                    v += src[q * kRows * MP];
+                if (p.swiglu) {   // row < 8: the gate; row + 8: its up
+                    float u = 0.f;
+                    for (int q = 0; q < W; q++)
+                        u += src[q * kRows * MP + 8 * MP];
+                    p.Y[(int64_t)m * (p.N / 2) + tl * 8 + row] = __float2half_rn(silu(v) * u);
+                    continue;
+                }
+                p.Y[(int64_t)m * p.N + n] = __float2half_rn(v);
+            }
         } else {
 #pragma unroll
             for (int t = 0; t < NT; t++) {
