@@ -462,6 +462,19 @@ def run_gpu(args, world, rank, local):
             prefill["1024"]["gpu_launches"] = n * pp.launches
         del pp
         torch.cuda.empty_cache()
+    # the same GEMM on a 24-layer audio encoder's linears over one clip's audio tokens
+    ecfg, elins = build_model("audio_encoder_prefill", dev)
+    encoder = {}
+    for M in ecfg["gemm_M"]:
+        ep = Pass(elins, M, "gemm", torch.float16, pdl=True)
+        fill(ep, ecfg["seed"] + M)
+        ep.capture()
+        t = timed_replays(ep, 10, 3, ranks) / 10
+        encoder[str(M)] = {"ms_per_pass": round(t, 4), "tflops": round(ep.flops / (t * 1e-3) / 1e12, 1),
+                           "weight_gbs": round(ep.weight_bytes / (t * 1e-3) / 1e9, 1)}
+        del ep
+    del elins
+    torch.cuda.empty_cache()
     assert mnb.mnb_device_status() == 0, "a GEMM wait timed out"
 
     cpu = None
@@ -494,6 +507,7 @@ def run_gpu(args, world, rank, local):
             "decode_fused_qkv_gateup": fused,
             "decode_by_M": by_m,
             "prefill": prefill,
+            "audio_encoder_prefill": encoder,
             "roofline_prefill": {"bound": "tensor", "kernel": "gemm_kernel", "M": 1024,
                                  "achieved": prefill["1024"]["tflops"], "peak": tc_sust, "unit": "TFLOP/s",
                                  "frac": prefill["1024"]["frac_tc_sustained"],

@@ -151,6 +151,15 @@ def test_qwen3_1p7b_prefill(step_mod, cuda_dev, M):
     check_pass(cfg, lins, samples, p, "f16")
 
 
+@pytest.mark.parametrize("M", [42, 390])
+def test_audio_encoder_prefill(step_mod, cuda_dev, M):
+    cfg, lins, samples = model(step_mod, "audio_encoder_prefill", 24)
+    p = step_mod.Pass(lins, M, "gemm", torch.float16)
+    _fill_inputs(p, cfg["seed"] + M, torch.float16)
+    _run_graph(p)
+    check_pass(cfg, lins, samples, p, "f16")
+
+
 @pytest.mark.parametrize("variant", ["qwen3_0p6b_bs64", "qwen3_0p6b_nozp"])
 def test_layout_variants(step_mod, cuda_dev, variant):
     cfg, lins, samples = build_model(step_mod, variant, 32)

@@ -56,6 +56,13 @@ def decoder_linears(hidden: int, q_out: int, kv_out: int, inter: int,
     return out
 
 
+def audio_encoder(layers=24, d=1024, ffn=4096):
+    """A Whisper-style audio encoder's linears: per layer q, k, v, o (d -> d),
+    fc1 (d -> ffn), fc2 (ffn -> d)."""
+    per_layer = [("q", d, d), ("k", d, d), ("v", d, d), ("o", d, d), ("fc1", ffn, d), ("fc2", d, ffn)]
+    return [Linear(name, layer, p, n, k) for layer in range(layers) for p, (name, n, k) in enumerate(per_layer)]
+
+
 def qwen3_0p6b(lm_head=True, layers=N_LAYERS):
     """Qwen3-0.6B-shaped decoder: hidden 1024, q 2048, kv 1024, MLP 3072."""
     return decoder_linears(1024, 2048, 1024, 3072, lm_head, layers)
@@ -87,6 +94,11 @@ CONFIGS = {
     "qwen3_0p6b_nozp": dict(desc="Qwen3-0.6B shapes, block 32 without zero points (zp = 8)",
                             seed=4, bs=32, has_zp=False, act="f16", scale="f16",
                             model="0.6b", gemv_M=[1, 4, 16], gemm_M=[64, 390]),
+    # the encoder's linears over one clip's audio tokens: 42 for a 3.2 s command,
+    # 390 for a 30 s clip (the audio-token count of "Building the prompt", step 2)
+    "audio_encoder_prefill": dict(desc="24-layer Whisper-style audio encoder linears (d 1024, FFN 4096), fp16, bs32 zp",
+                                  seed=5, bs=32, has_zp=True, act="f16", scale="f16",
+                                  model="encoder", lm_head=False, gemv_M=[], gemm_M=[42, 390]),
 }
 
 EMBED = dict(seed=4, V=VOCAB, D=1024, T=4096)
@@ -96,6 +108,8 @@ def config_linears(name: str):
     c = CONFIGS[name]
     if "linears" in c:
         return list(c["linears"])
+    if c["model"] == "encoder":
+        return audio_encoder()
     f = qwen3_0p6b if c["model"] == "0.6b" else qwen3_1p7b
     return f(lm_head=c.get("lm_head", True))
 
