@@ -377,6 +377,51 @@ def run_gpu(args, world, rank, local):
     per_launch_us = ms * 1000.0 / len(lins)
     achieved = per_launch_bytes / (per_launch_us * 1e-6) / 1e9
 
+    # the same 197 GEMVs as ONE persistent launch (mnb_gemv_chain): each GEMV
+    # waits for the previous one, as the separate launches do; then with the
+    # decoder's own dependencies (k, v read q's input; up reads gate's)
+    cdec = Pass(lins, 1, "gemv", torch.float16, pdl=True, chain=True)
+    fill(cdec, cfg["seed"])
+    cdec.capture()
+    with ClockSampler(local) as cclk:
+        c_ms = timed_replays(cdec, args.steps, args.warmup, ranks, "decode_chain") / args.steps
+    del cdec
+    waits = [0 if l.name.rstrip("0123456789") in ("k", "v", "up") else 1 for l in lins]
+    gcdec = Pass(lins, 1, "gemv", torch.float16, pdl=True, chain=True, waits=waits)
+    fill(gcdec, cfg["seed"])
+    gcdec.capture()
+    gc_ms = timed_replays(gcdec, args.steps, args.warmup, ranks, "decode_chain_grouped") / args.steps
+    del gcdec
+    # without a CUDA graph (eager, one host call per launch): the one-launch
+    # step against 197 launches issued from Python
+    def eager_us(p, n=20):
+        for _ in range(3):
+            p.run()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(True), torch.cuda.Event(True)
+        a.record()
+        for _ in range(n):
+            p.run()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n * 1000.0
+
+    esep = Pass(lins, 1, "gemv", torch.float16, pdl=True)
+    fill(esep, cfg["seed"])
+    e_sep_us = eager_us(esep)
+    del esep
+    echain = Pass(lins, 1, "gemv", torch.float16, pdl=True, chain=True)
+    fill(echain, cfg["seed"])
+    e_chain_us = eager_us(echain)
+    del echain
+    one_launch = {"launches_per_step": 1, "us_per_step": round(c_ms * 1000, 2),
+                  "eager_us_per_step": round(e_chain_us, 2), "eager_us_per_step_197_launches": round(e_sep_us, 2),
+                  "weight_gbs": round(world * wbytes / (c_ms * 1e-3) / 1e9, 1),
+                  "frac_hbm": round(wbytes / (c_ms * 1e-3) / 1e9 / hbm, 4), "clocks": cclk.summary(),
+                  "waits_per_step": len(lins) - 1,
+                  "grouped_us_per_step": round(gc_ms * 1000, 2), "grouped_waits_per_step": sum(waits) - 1,
+                  "grouped_weight_gbs": round(world * wbytes / (gc_ms * 1e-3) / 1e9, 1)}
+
     # the same step with the weights of projections that share an input stored
     # row-concatenated (q|k|v, gate|up): 113 launches, identical bytes and math
     from int4_block_quantized_matmulnbits_b200.step import fuse_decoder
@@ -505,6 +550,7 @@ def run_gpu(args, world, rank, local):
                               "us_with_greedy_argmax": round(lmg_ms * 1000, 2)},
             "decode_greedy": greedy,
             "decode_fused_qkv_gateup": fused,
+            "decode_one_launch": one_launch,
             "decode_by_M": by_m,
             "prefill": prefill,
             "audio_encoder_prefill": encoder,

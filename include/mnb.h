@@ -214,6 +214,63 @@ MNB_API int mnb_embed_gather(const int8_t *table, const float *row_scales, int64
                      const int32_t *ids, int64_t T, void *out, mnb_dtype out_t, int *status,
                      void *stream);
 
+/* ---- a whole decode step in one launch ----------------------------------
+ * The decoder step of "Qwen3-ASR-0.6B -- ONNX for the browser" ("Graph
+ * contracts": decoder_step) and of "Mega-ASR -- INT4 ONNX (GPTQ-calibrated)"
+ * is a sequence of MatMulNBits calls, 28 layers x 7 projections plus the
+ * lm_head, each small enough that a launch per call costs more than its
+ * weight traffic.  mnb_gemv_chain runs such a sequence ("tasks") as one
+ * persistent kernel: per task the same Y = X . dequant(W)^T as mnb_gemv with
+ * fp16 activations, fp16 scales and fp32 accumulation.
+ *
+ * Task j with wait != 0 reads its X only after tasks 0..j-1 have completed,
+ * so X may be (part of) an earlier task's Y; with wait == 0 its X must not be
+ * written by any task of the chain.  Task 0's X is read after the stream's
+ * earlier work (and, with MNB_FLAG_PDL, after the previous kernel completes).
+ * Tasks may share X; Y buffers must not overlap any task's X, W or another Y.
+ *
+ * Two steps.  mnb_gemv_chain_plan (host only, no device work) checks every
+ * task, encodes its tensor map and writes a plan of
+ * mnb_gemv_chain_plan_bytes(ntasks) bytes into caller memory.  The caller
+ * copies those bytes unchanged to device memory (64-byte aligned) and calls
+ * mnb_gemv_chain with both copies: the host copy for the launch shape, the
+ * device copy for the kernel.  A plan holds device addresses and is valid for
+ * the device that was current when it was made, for as long as every buffer
+ * it names stays allocated; the same plan may be launched any number of
+ * times (and captured in a CUDA graph).
+ *
+ * Requirements per task: N % 16 == 0, K % 256 == 0 (K % 512 == 0 for block
+ * 64 with zero points); X and packed 16-byte aligned; scales 16-byte (block
+ * 32) or 8-byte (block 64) aligned; zp 4-byte aligned; Y 2-byte aligned.
+ * All tasks share M (1..8), the block size and the presence of zero points.
+ *
+ * workspace: mnb_gemv_chain_workspace_bytes(ntasks) bytes of device memory,
+ * zero-filled before the first call; every call that completes leaves it
+ * zero-filled again.  Calls sharing a workspace must be stream-ordered.
+ * Failure: a wait inside the kernel that exceeds 2 s sets bit 1 (a weight
+ * copy) or bit 2 (a task's inputs) of the status word read by
+ * mnb_device_status; the kernel then exits early, Y is undefined and the
+ * workspace must be zero-filled again.
+ * Errors: MNB_ERR_INVALID_ARG, MNB_ERR_SHAPE, MNB_ERR_ALIGN,
+ *         MNB_ERR_UNSUPPORTED (M > 8, mixed layouts), MNB_ERR_CUDA. */
+typedef struct mnb_gemv_task {
+    const void *X;          /* fp16 [M][K] */
+    const uint8_t *packed;  /* [N][K/2] */
+    const void *scales;     /* fp16 [N][K/bs] */
+    const uint8_t *zp;      /* [N][ceil(K/bs/2)] or NULL (zero point 8) */
+    void *Y;                /* fp16 [M][N] */
+    int64_t N, K;
+    int32_t wait;           /* != 0: X is read after tasks 0..j-1 complete */
+    int32_t reserved;       /* 0 */
+} mnb_gemv_task;
+
+MNB_API size_t mnb_gemv_chain_plan_bytes(int ntasks);        /* 0 when ntasks is outside [1, 65536] */
+MNB_API size_t mnb_gemv_chain_workspace_bytes(int ntasks);   /* 0 when ntasks is outside [1, 65536] */
+MNB_API int mnb_gemv_chain_plan(const mnb_gemv_task *tasks, int ntasks, int64_t M, int bs, void *plan,
+                                size_t plan_bytes);
+MNB_API int mnb_gemv_chain(const void *plan, const void *plan_device, void *workspace, size_t ws_bytes,
+                           unsigned flags, void *stream);
+
 /* Reads (and, if clear != 0, zeroes) the library's device status word on the
  * current device: bit 0 = a GEMM mbarrier wait timed out.  Synchronizes the
  * device.  Errors: MNB_ERR_INVALID_ARG (NULL), MNB_ERR_CUDA. */

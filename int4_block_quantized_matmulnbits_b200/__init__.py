@@ -23,6 +23,8 @@ __all__ = [
     "mnb_last_error", "mnb_version", "mnb_packed_sizes", "mnb_quantize_rtn", "mnb_dequantize",
     "mnb_gemv", "mnb_gemm", "mnb_embed_gather", "mnb_device_status",
     "mnb_gemv_argmax", "mnb_gemv_argmax_workspace_bytes", "mnb_gemv_argmax_noalloc", "mnb_gemv_swiglu",
+    "mnb_gemv_task", "mnb_gemv_chain_plan_bytes", "mnb_gemv_chain_workspace_bytes", "mnb_gemv_chain_plan",
+    "mnb_gemv_chain",
 ]
 
 MNB_F32, MNB_F16 = 0, 1
@@ -38,6 +40,13 @@ class MnbError(RuntimeError):
     def __init__(self, fn, code, msg):
         super().__init__(f"{fn} -> {_ERRORS.get(code, code)}: {msg}")
         self.code = code
+
+
+class mnb_gemv_task(ctypes.Structure):
+    """One GEMV of mnb_gemv_chain (the C struct of the same name)."""
+    _fields_ = [("X", ctypes.c_void_p), ("packed", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("zp", ctypes.c_void_p), ("Y", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("wait", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 def _load():
@@ -63,6 +72,10 @@ def _load():
         "mnb_gemv_swiglu": ([vp, vp, vp, i32, vp, vp, i64, i64, i64, i32, u32, vp], i32),
         "mnb_gemv_argmax": ([vp, vp, vp, i32, vp, vp, i64, i64, i64, i32, vp, vp, vp, sz, u32, vp], i32),
         "mnb_gemv_argmax_noalloc": ([vp, vp, vp, i32, vp, vp, i64, i64, i64, i32, vp, vp, u32, vp], i32),
+        "mnb_gemv_chain_plan_bytes": ([i32], sz),
+        "mnb_gemv_chain_workspace_bytes": ([i32], sz),
+        "mnb_gemv_chain_plan": ([P(mnb_gemv_task), i32, i64, i32, vp, sz], i32),
+        "mnb_gemv_chain": ([vp, vp, vp, sz, u32, vp], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -169,6 +182,44 @@ def mnb_gemv_argmax_noalloc(X, packed, scales, zp, Y, M, N, K, bs, ids, max_out,
         _ptr(max_out), flags, _stream(stream)))
 
 
+def mnb_gemv_chain_plan_bytes(ntasks) -> int:
+    return _lib.mnb_gemv_chain_plan_bytes(ntasks)
+
+
+def mnb_gemv_chain_workspace_bytes(ntasks) -> int:
+    """Bytes of the (zero-filled) device workspace of a chain of ntasks GEMVs."""
+    return _lib.mnb_gemv_chain_workspace_bytes(ntasks)
+
+
+def mnb_gemv_chain_plan(tasks, M, bs):
+    """Plan a chain of decode GEMVs for mnb_gemv_chain (host only).
+
+    tasks: sequence of (X, packed, scales, zp, Y, N, K, wait) with device
+    tensors (zp may be None).  Returns the plan as a 64-byte aligned uint8 CPU
+    tensor; copy it unchanged to the device (e.g. ``plan.cuda()``) and pass both."""
+    n = len(tasks)
+    arr = (mnb_gemv_task * n)()
+    for i, (X, packed, scales, zp, Y, N, K, wait) in enumerate(tasks):
+        arr[i] = mnb_gemv_task(_ptr(X), _ptr(packed), _ptr(scales), _ptr(zp), _ptr(Y), N, K, int(wait), 0)
+    nbytes = mnb_gemv_chain_plan_bytes(n)
+    if nbytes == 0:
+        raise MnbError("mnb_gemv_chain_plan", -1, f"ntasks={n} outside [1, 65536]")
+    buf = torch.empty(nbytes + 64, dtype=torch.uint8)
+    off = (-buf.data_ptr()) % 64
+    plan = buf[off:off + nbytes]
+    _check("mnb_gemv_chain_plan", _lib.mnb_gemv_chain_plan(arr, n, M, bs, plan.data_ptr(), nbytes))
+    return plan
+
+
+def mnb_gemv_chain(plan, plan_device, workspace, flags=0, stream=None):
+    """Run a planned chain of decode GEMVs as one launch (plan: the host tensor
+    from mnb_gemv_chain_plan; plan_device: its device copy; workspace:
+    zero-filled uint8 device tensor of mnb_gemv_chain_workspace_bytes bytes)."""
+    _check("mnb_gemv_chain", _lib.mnb_gemv_chain(
+        _ptr(plan), _ptr(plan_device), _ptr(workspace), workspace.numel() * workspace.element_size(), flags,
+        _stream(stream)))
+
+
 def mnb_gemm(X, packed, scales, zp, Y, M, N, K, bs, flags=0, stream=None):
     """Y [M, N] = X [M, K] . dequant(W)^T on the tensor cores (fp16 X and Y)."""
     _check("mnb_gemm", _lib.mnb_gemm(
@@ -184,7 +235,8 @@ def mnb_embed_gather(table, row_scales, V, D, ids, T, out, status=None, stream=N
 
 
 def mnb_device_status(clear=False) -> int:
-    """The library's device status word (bit 0: a GEMM wait timed out); synchronizes."""
+    """The library's device status word (bit 0: a GEMM or GEMV wait timed out;
+    bits 1-2: mnb_gemv_chain); synchronizes."""
     v = ctypes.c_uint()
     _check("mnb_device_status", _lib.mnb_device_status(ctypes.byref(v), int(bool(clear))))
     return v.value

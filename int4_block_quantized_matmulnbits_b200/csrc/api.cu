@@ -4,6 +4,8 @@
 #include <stdarg.h>
 #include <stdio.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -26,6 +28,34 @@ int check_launch(const char *what) {
     if (e != cudaSuccess)
         return fail(MNB_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
     return MNB_OK;
+}
+
+EncodeTiledFn tensor_map_encoder() {
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+int device_sm_count() {
+    static int counts[128] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128)
+        return 148;
+    if (counts[dev] <= 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        counts[dev] = n;
+    }
+    return counts[dev];
 }
 
 // Limits: sizes fit comfortably in 32-bit element indices of one row and in
@@ -273,6 +303,44 @@ int mnb_embed_gather(const int8_t *table, const float *row_scales, int64_t V, in
         return fail(MNB_ERR_ALIGN, "%s: table and out must be 16-byte aligned", fn);
     return launch_embed_gather(table, row_scales, V, D, ids, T, out, out_t == MNB_F16, status,
                                (cudaStream_t)stream);
+}
+
+size_t mnb_gemv_chain_plan_bytes(int ntasks) { return gemv_chain_plan_bytes(ntasks); }
+
+size_t mnb_gemv_chain_workspace_bytes(int ntasks) { return gemv_chain_workspace_bytes(ntasks); }
+
+int mnb_gemv_chain_plan(const mnb_gemv_task *tasks, int ntasks, int64_t M, int bs, void *plan, size_t plan_bytes) {
+    clear_error();
+    static const char *fn = "mnb_gemv_chain_plan";
+    if (!tasks || !plan)
+        return fail(MNB_ERR_INVALID_ARG, "%s: NULL tasks or plan", fn);
+    if (ntasks < 1 || ntasks > 65536)
+        return fail(MNB_ERR_INVALID_ARG, "%s: ntasks=%d outside [1, 65536]", fn, ntasks);
+    if (plan_bytes < gemv_chain_plan_bytes(ntasks))
+        return fail(MNB_ERR_INVALID_ARG, "%s: plan buffer of %zu bytes, %zu needed", fn, plan_bytes,
+                    gemv_chain_plan_bytes(ntasks));
+    if (!aligned(plan, 64))
+        return fail(MNB_ERR_ALIGN, "%s: plan buffer not 64-byte aligned", fn);
+    if (bs != 32 && bs != 64)
+        return fail(MNB_ERR_SHAPE, "%s: block size %d not in {32, 64}", fn, bs);
+    if (M < 1)
+        return fail(MNB_ERR_INVALID_ARG, "%s: M=%lld", fn, (long long)M);
+    if (M > 8)
+        return fail(MNB_ERR_UNSUPPORTED, "%s: M=%lld above 8", fn, (long long)M);
+    return gemv_chain_plan(tasks, ntasks, (int)M, bs, plan, plan_bytes);
+}
+
+int mnb_gemv_chain(const void *plan, const void *plan_device, void *workspace, size_t ws_bytes, unsigned flags,
+                   void *stream) {
+    clear_error();
+    static const char *fn = "mnb_gemv_chain";
+    if (!plan || !plan_device || !workspace)
+        return fail(MNB_ERR_INVALID_ARG, "%s: NULL plan, device plan or workspace", fn);
+    if (!aligned(plan, 64) || !aligned(plan_device, 64) || !aligned(workspace, 4))
+        return fail(MNB_ERR_ALIGN, "%s: plans must be 64-byte aligned, the workspace 4-byte aligned", fn);
+    if (flags & ~(unsigned)MNB_FLAG_PDL)
+        return fail(MNB_ERR_INVALID_ARG, "%s: unknown flags 0x%x", fn, flags);
+    return launch_gemv_chain(plan, plan_device, workspace, ws_bytes, flags, (cudaStream_t)stream);
 }
 
 int mnb_device_status(unsigned *status_out, int clear) {

@@ -1,6 +1,7 @@
 // common.cuh -- shared host/device helpers of libmnb (the CUDA side only).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -18,6 +19,15 @@ void clear_error();
 int check_launch(const char *what);
 
 inline bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// cuTensorMapEncodeTiled from the driver, or null when it is unavailable.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn tensor_map_encoder();
+
+// Streaming multiprocessors of the current device (cached per device).
+int device_sm_count();
 
 // ---------------------------------------------------------------- device PTX
 

@@ -481,23 +481,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---- host side ----------------------------------------------------------------
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-    return fn;
-}
-
 }  // namespace
 
 // Tile policy knobs (tuning hooks, see mnb_tune_gemm below).
@@ -509,15 +492,10 @@ static int g_gemm_max_split = 4;
 
 int launch_gemm(const void *X, const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,
                 void *Y, int M, int N, int K, int bs, unsigned flags, cudaStream_t s) {
-    EncodeTiledFn encode = get_encode_fn();
+    EncodeTiledFn encode = tensor_map_encoder();
     if (!encode)
         return fail(MNB_ERR_CUDA, "mnb_gemm: cuTensorMapEncodeTiled unavailable");
-    int sms = 148;
-    {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    }
+    const int sms = device_sm_count();
 
     // token tiling: as few tiles of <= 256 as possible, evenly sized; narrower
     // tiles (down to g_gemm_min_bn) while the grid would leave half the SMs idle
@@ -637,6 +615,8 @@ int read_device_status(unsigned *out, int clear) {
         int rc = read_gemv_status(out, clear);
         if (!rc)
             rc = read_stream_status(out, clear);
+        if (!rc)
+            rc = read_chain_status(out, clear);
         if (rc)
             return rc;
     }

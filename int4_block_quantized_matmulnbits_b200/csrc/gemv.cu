@@ -533,16 +533,6 @@ int launch_one(const Params &p, int grid, size_t smem, unsigned flags, cudaStrea
     return MNB_OK;
 }
 
-int sm_count() {
-    static int count = 0;
-    if (count == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || count <= 0)
-            count = 148;
-    }
-    return count;
-}
 
 }  // namespace
 
@@ -619,7 +609,7 @@ int launch_gemv(const void *X, int act_f16, const uint8_t *packed, const void *s
     p.scale_f16 = scale_f16;
     int grid = 0;
     size_t smem = 0;
-    int rc = plan_gemv(M, N, K, act_f16 ? 2 : 4, MP, sm_count(), p, grid, smem);
+    int rc = plan_gemv(M, N, K, act_f16 ? 2 : 4, MP, device_sm_count(), p, grid, smem);
     if (rc)
         return rc;
 

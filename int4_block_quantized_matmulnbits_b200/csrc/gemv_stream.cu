@@ -408,34 +408,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncthreads();   // pairs with the producer's: it drains after a timeout
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn stream_encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-    return fn;
-}
-
-int stream_sm_count() {
-    static int count = 0;
-    if (count == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || count <= 0)
-            count = 148;
-    }
-    return count;
-}
-
 constexpr size_t kSmemCap = 110 * 1024;   // under half an SM: the next call's CTA fits beside this one
 
 template <bool BS64, bool ZP, bool SF32>
@@ -481,10 +453,10 @@ int launch_gemv_stream(const void *X, const uint8_t *packed, const void *scales,
         return 1;
     if (has_zp && (!aligned(zp, 16) || zpb % 16 != 0))
         return 1;
-    EncodeTiledFn encode = stream_encode_fn();
+    EncodeTiledFn encode = tensor_map_encoder();
     if (!encode)
         return fail(MNB_ERR_CUDA, "mnb_gemv: cuTensorMapEncodeTiled unavailable");
-    const int sms = stream_sm_count();
+    const int sms = device_sm_count();
 
     StreamParams p;
     p.X = reinterpret_cast<const __half *>(X);

@@ -624,34 +624,6 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
     }
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-    return fn;
-}
-
-int sm_count_tc() {
-    static int count = 0;
-    if (count == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || count <= 0)
-            count = 148;
-    }
-    return count;
-}
-
 template <int NT, class C>
 int launch_tc(const CUtensorMap &map, const TcParams &p, int grid, size_t smem, unsigned flags, cudaStream_t s) {
     auto fn = gemv_tc_kernel<NT, C>;
@@ -698,12 +670,12 @@ static int g_force_w = 0, g_force_s = 1;
 static int launch_tc_common(const void *X, const uint8_t *packed, const void *scales, int scale_f16,
                             const uint8_t *zp, void *Y, int M, int N, int K, int bs, unsigned flags,
                             cudaStream_t s, const ArgmaxArgs *am, int swiglu = 0) {
-    EncodeTiledFn encode = encode_fn();
+    EncodeTiledFn encode = tensor_map_encoder();
     if (!encode)
         return fail(MNB_ERR_CUDA, "mnb_gemv: cuTensorMapEncodeTiled unavailable");
     const int NT = (M <= 8) ? 1 : 2;
     const int MP = 8 * NT;
-    const int sms = sm_count_tc();
+    const int sms = device_sm_count();
 
     TcParams p;
     p.X = X; p.scales = scales; p.zp = zp; p.Y = reinterpret_cast<__half *>(Y);
@@ -851,7 +823,7 @@ int launch_gemv_swiglu(const void *X, const uint8_t *packed, const void *scales,
 
 size_t gemv_argmax_workspace_bytes(int M) {
     // one (value, index) pair per token per CTA; at most two CTAs per SM
-    return kArgmaxWsHeader + (size_t)2 * sm_count_tc() * (size_t)M * sizeof(uint2);
+    return kArgmaxWsHeader + (size_t)2 * device_sm_count() * (size_t)M * sizeof(uint2);
 }
 
 int launch_gemv_argmax(const void *X, const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,

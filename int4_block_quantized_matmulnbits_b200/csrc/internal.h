@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "mnb.h"
+
 namespace mnb {
 
 int launch_quantize_rtn(const float *W, int64_t N, int64_t K, int bs, int has_zp, uint8_t *packed,
@@ -49,8 +51,16 @@ int launch_embed_gather(const int8_t *table, const float *row_scales, int64_t V,
                         const int32_t *ids, int64_t T, void *out, int out_f16, int *status,
                         cudaStream_t s);
 
+// A sequence of decode GEMVs as one persistent launch (plan on the host first).
+size_t gemv_chain_plan_bytes(int ntasks);
+size_t gemv_chain_workspace_bytes(int ntasks);
+int gemv_chain_plan(const mnb_gemv_task *tasks, int ntasks, int M, int bs, void *plan, size_t plan_bytes);
+int launch_gemv_chain(const void *plan, const void *plan_device, void *workspace, size_t ws_bytes, unsigned flags,
+                      cudaStream_t s);
+
 int read_device_status(unsigned *out, int clear);
 int read_gemv_status(unsigned *out, int clear);     // ORs the decode kernel's word into *out
 int read_stream_status(unsigned *out, int clear);   // same for the streaming decode kernel
+int read_chain_status(unsigned *out, int clear);    // the chain kernel's bits, shifted to bits 1-2
 
 }  // namespace mnb

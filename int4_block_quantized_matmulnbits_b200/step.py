@@ -13,7 +13,8 @@ from __future__ import annotations
 import torch
 
 from . import (MNB_FLAG_PDL, mnb_dequantize, mnb_embed_gather, mnb_gemm, mnb_gemv, mnb_gemv_argmax,
-               mnb_gemv_argmax_workspace_bytes, mnb_gemv_swiglu, mnb_packed_sizes, mnb_quantize_rtn)
+               mnb_gemv_argmax_workspace_bytes, mnb_gemv_chain, mnb_gemv_chain_plan, mnb_gemv_chain_workspace_bytes,
+               mnb_gemv_swiglu, mnb_packed_sizes, mnb_quantize_rtn)
 
 
 class QLinear:
@@ -123,7 +124,8 @@ class Pass:
     gather of M token ids runs first, as in a decode step.
     """
 
-    def __init__(self, linears, M, kind="gemv", act_dtype=torch.float16, pdl=True, embed=None, greedy=False):
+    def __init__(self, linears, M, kind="gemv", act_dtype=torch.float16, pdl=True, embed=None, greedy=False,
+                 chain=False, waits=None):
         self.linears, self.M, self.kind, self.pdl = list(linears), M, kind, pdl
         dev = self.linears[0].packed.device
         # one flat buffer each for all inputs and all outputs (views per linear,
@@ -148,6 +150,20 @@ class Pass:
             self.ids = torch.zeros((M,), dtype=torch.int32, device=dev)
             self.max_out = torch.zeros((M,), dtype=torch.float32, device=dev)
             self.ws = torch.zeros((mnb_gemv_argmax_workspace_bytes(M),), dtype=torch.uint8, device=dev)
+        # chain=True: all GEMVs in one persistent launch (mnb_gemv_chain).  waits[i]
+        # = 1 makes linear i read its X only after linears 0..i-1 are complete
+        # (default: every linear waits, the dependencies of separate launches)
+        self.chain = None
+        if chain:
+            assert kind == "gemv" and not self.greedy
+            assert not any(getattr(l, "swiglu", False) for l in self.linears)
+            n = len(self.linears)
+            waits = [1] * n if waits is None else list(waits)
+            tasks = [(x, l.packed, l.scales, l.zp, y, l.N, l.K, w)
+                     for l, x, y, w in zip(self.linears, self.X, self.Y, waits)]
+            plan = mnb_gemv_chain_plan(tasks, M, self.linears[0].bs)
+            self.chain = (plan, plan.to(dev),
+                          torch.zeros((mnb_gemv_chain_workspace_bytes(n),), dtype=torch.uint8, device=dev))
 
     @property
     def weight_bytes(self):
@@ -159,7 +175,8 @@ class Pass:
 
     @property
     def launches(self):
-        return len(self.linears) + (1 if self.embed is not None else 0)
+        n = 1 if self.chain is not None else len(self.linears)
+        return n + (1 if self.embed is not None else 0)
 
     def run(self, stream=None):
         if self.embed is not None:
@@ -167,6 +184,9 @@ class Pass:
             mnb_embed_gather(table, rs, table.shape[0], table.shape[1], ids, ids.shape[0], out,
                              None, stream)
         flags = MNB_FLAG_PDL if self.pdl else 0
+        if self.chain is not None:
+            mnb_gemv_chain(*self.chain, flags, stream)
+            return
         last = len(self.linears) - 1
         for i, (l, x, y) in enumerate(zip(self.linears, self.X, self.Y)):
             if self.kind == "gemv":

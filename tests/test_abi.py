@@ -145,3 +145,46 @@ def test_gemv_swiglu_argument_checks(lib):
     assert f(A, A, A, F16, A, A, 1, 64, 96, 64, 0, None) == SHAPE            # K % bs
     assert f(A, A, A, F16, A, A, 1, 64, 64, 32, 0x80, None) == INVALID       # unknown flag
     assert f(A, A, A, F16, A, A, 0, 64, 64, 32, 0, None) == OK               # M = 0
+
+
+def test_gemv_chain_argument_checks(mnb, lib):
+    T = mnb.mnb_gemv_task
+    assert mnb.mnb_gemv_chain_plan_bytes(0) == 0 and mnb.mnb_gemv_chain_plan_bytes(65537) == 0
+    assert mnb.mnb_gemv_chain_plan_bytes(3) == 64 + 3 * 256
+    assert mnb.mnb_gemv_chain_workspace_bytes(0) == 0 and mnb.mnb_gemv_chain_workspace_bytes(197) >= 198 * 4
+
+    def task(N=2048, K=2048, X=A, packed=A, scales=A, zp=A, Y=A, wait=1, reserved=0):
+        return T(X, packed, scales, zp, Y, N, K, wait, reserved)
+
+    nbytes = mnb.mnb_gemv_chain_plan_bytes(2)
+    buf = ctypes.create_string_buffer(nbytes + 128)
+    plan = ctypes.addressof(buf) + (-ctypes.addressof(buf)) % 64
+
+    def rc(tasks, M=1, bs=32, size=nbytes, ptr=plan):
+        arr = (T * len(tasks))(*tasks)
+        return lib.mnb_gemv_chain_plan(arr, len(tasks), M, bs, ptr, size)
+
+    assert rc([task(), task(N=72)]) == SHAPE                  # N % 16
+    assert rc([task(), task(K=320)]) == SHAPE                 # K % 256
+    assert rc([task(K=768)], bs=64) == SHAPE                  # block 64 with zero points: K % 512
+    assert rc([task(), task(X=A + 8)]) == ALIGN               # X not 16-byte aligned
+    assert rc([task(scales=A + 8)]) == ALIGN                  # block-32 scales not 16-byte aligned
+    assert rc([task(zp=A + 2)]) == ALIGN
+    assert rc([task(), task(zp=None)]) == UNSUPPORTED         # zero points in some tasks only
+    assert rc([task()], M=9) == UNSUPPORTED
+    assert rc([task()], M=0) == INVALID
+    assert rc([task()], bs=48) == SHAPE
+    assert rc([task(reserved=1)]) == INVALID
+    assert rc([task(Y=None)]) == INVALID
+    assert rc([task(), task()], size=nbytes - 1) == INVALID   # plan buffer too small
+    assert rc([task()], ptr=plan + 16) == ALIGN               # plan buffer not 64-byte aligned
+    assert rc([task(K=65536)], M=8) == SHAPE                  # X does not fit in shared memory
+    # launch: the plan's header is checked before anything touches the device
+    f = lib.mnb_gemv_chain
+    ctypes.memset(plan, 0, nbytes)
+    ws = mnb.mnb_gemv_chain_workspace_bytes(2)
+    assert f(plan, A, A, ws, 0, None) == INVALID              # not a plan
+    assert b"not a plan" in lib.mnb_last_error()
+    assert f(None, A, A, ws, 0, None) == INVALID
+    assert f(plan, A + 32, A, ws, 0, None) == ALIGN           # device plan not 64-byte aligned
+    assert f(plan, A, A, ws, 0x80, None) == INVALID           # unknown flag

@@ -116,6 +116,17 @@ def test_qwen3_1p7b_decode_step(step_mod, cuda_dev, M):
     check_pass(cfg, lins, samples, p, "f16")
 
 
+@pytest.mark.parametrize("M", [1, 2, 4, 8])
+def test_qwen3_1p7b_decode_step_one_launch(step_mod, cuda_dev, M):
+    # the same 197 GEMVs as one mnb_gemv_chain launch, each waiting for the previous
+    cfg, lins, samples = model(step_mod, "qwen3_1p7b_decode", 48, full_layers=(27,))
+    p = step_mod.Pass(lins, M, "gemv", torch.float16, chain=True)
+    assert p.launches == 1
+    _fill_inputs(p, cfg["seed"] + M, torch.float16)
+    _run_graph(p)
+    check_pass(cfg, lins, samples, p, "f16")
+
+
 @pytest.mark.parametrize("M", [1, 16])
 def test_qwen3_1p7b_decode_step_fused_layout(step_mod, cuda_dev, M):
     # q|k|v and gate|up stored row-concatenated: one GEMV per group, same outputs
@@ -158,6 +169,24 @@ def test_audio_encoder_prefill(step_mod, cuda_dev, M):
     _fill_inputs(p, cfg["seed"] + M, torch.float16)
     _run_graph(p)
     check_pass(cfg, lins, samples, p, "f16")
+
+
+def test_qwen3_0p6b_decode_step_one_launch(step_mod, cuda_dev):
+    cfg, lins, samples = build_model(step_mod, "qwen3_0p6b_decode", 96, full_layers=(0,))
+    p = step_mod.Pass(lins, 1, "gemv", torch.float16, chain=True)
+    _fill_inputs(p, cfg["seed"], torch.float16)
+    _run_graph(p)
+    check_pass(cfg, lins, samples, p, "f16")
+
+
+@pytest.mark.parametrize("variant", ["qwen3_0p6b_bs64", "qwen3_0p6b_nozp"])
+def test_layout_variants_one_launch(step_mod, cuda_dev, variant):
+    cfg, lins, samples = build_model(step_mod, variant, 32)
+    for M in [m for m in cfg["gemv_M"] if m <= 8]:
+        p = step_mod.Pass(lins, M, "gemv", torch.float16, chain=True)
+        _fill_inputs(p, cfg["seed"] + M, torch.float16)
+        _run_graph(p)
+        check_pass(cfg, lins, samples, p, "f16")
 
 
 @pytest.mark.parametrize("variant", ["qwen3_0p6b_bs64", "qwen3_0p6b_nozp"])
