@@ -507,6 +507,23 @@ def run_gpu(args, world, rank, local):
             prefill["1024"]["gpu_launches"] = n * pp.launches
         del pp
         torch.cuda.empty_cache()
+    # the same prefill with q|k|v and gate|up stored row-concatenated (one GEMM
+    # per group, 113 launches): identical weights, bytes and FLOPs, larger GEMMs
+    fbody = fuse_decoder(body)
+    prefill_fused = {}
+    for M in (1024, 420, 256, 64):
+        pf = Pass(fbody, M, "gemm", torch.float16, pdl=True)
+        fill(pf, cfg["seed"] + M)
+        pf.capture()
+        n = 20 if M == 1024 else 10
+        t = timed_replays(pf, n, 3, ranks) / n
+        assert pf.flops == sum(2 * M * l.N * l.K for l in body)
+        tflops = pf.flops / (t * 1e-3) / 1e12
+        prefill_fused[str(M)] = {"launches_per_pass": len(fbody), "ms_per_pass": round(t, 4),
+                                 "tflops": round(tflops, 1), "frac_tc_sustained": round(tflops / tc_sust, 4)}
+        del pf
+        torch.cuda.empty_cache()
+    del fbody
     # the same GEMM on a 24-layer audio encoder's linears over one clip's audio tokens
     ecfg, elins = build_model("audio_encoder_prefill", dev)
     encoder = {}
@@ -553,6 +570,7 @@ def run_gpu(args, world, rank, local):
             "decode_one_launch": one_launch,
             "decode_by_M": by_m,
             "prefill": prefill,
+            "prefill_fused_qkv_gateup": prefill_fused,
             "audio_encoder_prefill": encoder,
             "roofline_prefill": {"bound": "tensor", "kernel": "gemm_kernel", "M": 1024,
                                  "achieved": prefill["1024"]["tflops"], "peak": tc_sust, "unit": "TFLOP/s",

@@ -162,6 +162,29 @@ def test_qwen3_1p7b_prefill(step_mod, cuda_dev, M):
     check_pass(cfg, lins, samples, p, "f16")
 
 
+def test_qwen3_1p7b_prefill_fused_layout(step_mod, cuda_dev):
+    # q|k|v and gate|up row-concatenated: one GEMM per group, the same outputs
+    cfg, lins, samples = model(step_mod, "qwen3_1p7b_prefill", 24)
+    fused = step_mod.fuse_decoder(lins)
+    assert len(fused) == 28 * 4
+    M = 420
+    p = step_mod.Pass(fused, M, "gemm", torch.float16)
+    _fill_inputs(p, cfg["seed"] + M, torch.float16)
+    _run_graph(p)
+
+    class View:   # per-projection views of the fused pass, in the original order
+        X, Y = [], []
+
+    v = View()
+    for f, x, y in zip(fused, p.X, p.Y):
+        off = 0
+        for _, n in getattr(f, "parts", [(f.name, f.N)]):
+            v.X.append(x)
+            v.Y.append(y[:, off:off + n])
+            off += n
+    check_pass(cfg, lins, samples, v, "f16")
+
+
 @pytest.mark.parametrize("M", [42, 390])
 def test_audio_encoder_prefill(step_mod, cuda_dev, M):
     cfg, lins, samples = model(step_mod, "audio_encoder_prefill", 24)
