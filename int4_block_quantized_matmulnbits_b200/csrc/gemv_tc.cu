@@ -697,7 +697,9 @@ static int launch_tc_common(const void *X, const uint8_t *packed, const void *sc
     // costed in box-times on the busiest warp: rounds of tile groups x (boxes
     // per warp + a per-round reduction cost: none when warps own whole rows,
     // more when the partial sums meet across a cluster).  Fitted on the
-    // decoder shapes: a cluster split rarely pays.
+    // decoder shapes at M <= 8 (one MMA column group); at 9 <= M <= 16 a box
+    // costs twice as much (two column groups) and a cluster reduction grows
+    // with the cluster (measured: 3 box-times per CTA of the cluster).
     const int nbx_all = (K + kBoxK - 1) / kBoxK;
     auto smem_for = [&](int W, int S, int &nbx_w, int &kcta, int &xs_stride) {
         nbx_w = (nbx_all + W * S - 1) / (W * S);
@@ -706,6 +708,7 @@ static int launch_tc_common(const void *X, const uint8_t *packed, const void *sc
         return 1024 + (size_t)kWarps * kDepth * kBoxBytes + (size_t)M * xs_stride + 512 +
                (size_t)2 * kWarps * kRows * MP * 4 + (size_t)kWarps * kDepth * 8;
     };
+    const double groups_f = (double)NT;   // MMA column groups of 8 tokens
     int W = 0, S = 1;
     double best = 0.0;
     for (int w = 1; w <= kWarps; w *= 2)
@@ -720,14 +723,15 @@ static int launch_tc_common(const void *X, const uint8_t *packed, const void *sc
             double cost;
             if (w == 1 && sc == 1) {
                 const int warps = sms * per_sm * kWarps;
-                cost = (double)((p.ntiles + warps - 1) / warps) * nbx_all;
+                cost = (double)((p.ntiles + warps - 1) / warps) * nbx_all * groups_f;
             } else {
                 const int tpc = kWarps / w;
                 const int groups = (p.ntiles + tpc - 1) / tpc;
                 int maxcl = sms * per_sm / sc;
                 if (maxcl < 1) maxcl = 1;
                 const int rounds = (groups + maxcl - 1) / maxcl;
-                cost = rounds * (1.15 * nbx_w + (sc > 1 ? 1.6 : 0.5));
+                const double red = (sc == 1) ? 0.5 * groups_f : (NT == 1 ? 1.6 : 3.0 * sc);
+                cost = rounds * (1.15 * groups_f * nbx_w + red);
             }
             if (W == 0 || cost < best - 1e-9 || (cost < best + 1e-9 && sc < S) ||
                 (cost < best + 1e-9 && sc == S && w > W)) {
@@ -736,21 +740,6 @@ static int launch_tc_common(const void *X, const uint8_t *packed, const void *sc
                 best = cost;
             }
         }
-    if (M > 8 && !am) {
-        // two token groups per MMA: the model above was fitted at M <= 8; here
-        // the split aims at about 16 warps with work on every SM
-        int slices = (sms * 2 * kWarps + p.ntiles - 1) / p.ntiles;
-        if (slices > nbx_all) slices = nbx_all;
-        if (slices > kWarps * kMaxCluster) slices = kWarps * kMaxCluster;
-        if (slices < 1) slices = 1;
-        W = 1;
-        while (W * 2 <= kWarps && W * 2 <= slices) W *= 2;
-        S = (slices + W - 1) / W;
-        if (S > kMaxCluster) S = kMaxCluster;
-        int nbx_w, kcta, xs_stride;
-        while (S < kMaxCluster && smem_for(W, S, nbx_w, kcta, xs_stride) > 200 * 1024)
-            S++;
-    }
     if (!am && g_force_w > 0) {   // tuning hook
         W = g_force_w;
         S = g_force_s;
