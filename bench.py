@@ -524,6 +524,22 @@ def run_gpu(args, world, rank, local):
         del pf
         torch.cuda.empty_cache()
     del fbody
+    # a prompt appended to a cached one: 17-63 new tokens through mnb_matmul,
+    # which runs GEMV launches of 16 tokens up to M = 20 and the GEMM above
+    # (same shapes as the prefill pass; its weights)
+    cached = {}
+    for M in (17, 20, 24, 32, 48, 63):
+        pc = Pass(body, M, "matmul", torch.float16, pdl=True)
+        fill(pc, cfg["seed"] + M)
+        pc.capture()
+        t = timed_replays(pc, 10, 3, ranks) / 10
+        tflops = pc.flops / (t * 1e-3) / 1e12
+        cached[str(M)] = {"ms_per_pass": round(t, 4), "tflops": round(tflops, 1),
+                          "weight_gbs": round(pc.weight_bytes / (t * 1e-3) / 1e9, 1),
+                          "frac_hbm": round(pc.weight_bytes / (t * 1e-3) / 1e9 / hbm, 4),
+                          "path": "gemv, 2 launches per projection" if M <= 20 else "gemm"}
+        del pc
+        torch.cuda.empty_cache()
     # the same GEMM on a 24-layer audio encoder's linears over one clip's audio tokens
     ecfg, elins = build_model("audio_encoder_prefill", dev)
     encoder = {}
@@ -571,6 +587,7 @@ def run_gpu(args, world, rank, local):
             "decode_by_M": by_m,
             "prefill": prefill,
             "prefill_fused_qkv_gateup": prefill_fused,
+            "cached_prefill": cached,
             "audio_encoder_prefill": encoder,
             "roofline_prefill": {"bound": "tensor", "kernel": "gemm_kernel", "M": 1024,
                                  "achieved": prefill["1024"]["tflops"], "peak": tc_sust, "unit": "TFLOP/s",

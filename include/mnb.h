@@ -200,6 +200,24 @@ MNB_API int mnb_gemm(const void *X, mnb_dtype act_t, const uint8_t *packed, cons
              mnb_dtype scale_t, const uint8_t *zp, void *Y, int64_t M, int64_t N, int64_t K,
              int bs, unsigned flags, void *stream);
 
+/* The MatMulNBits operator for any number of tokens: the same
+ * Y = X . dequant(W)^T (layouts, tolerances and errors as mnb_gemv/mnb_gemm)
+ * on the kernel that serves M best.  Decode ("Graph contracts":
+ * decoder_step), prefill of a prompt appended to a cached one (a few to a few
+ * dozen new tokens) and full prefill (decoder_init / decoder_prefill) all take
+ * this one call:
+ *   M <= 16: mnb_gemv;
+ *   17 <= M <= 20, fp16 X: mnb_gemv launches of 16 tokens and the rest
+ *     (measured faster than the tensor-core GEMM there);
+ *   M >= 21 with fp16 X, N % 128 == 0, K % 64 == 0: mnb_gemm;
+ *   otherwise (fp32 X, or shapes the GEMM does not take): mnb_gemv launches
+ *     of up to 16 tokens.
+ * Requires X, packed and Y 16-byte aligned.
+ * Errors: MNB_ERR_INVALID_ARG, MNB_ERR_SHAPE, MNB_ERR_ALIGN, MNB_ERR_CUDA. */
+MNB_API int mnb_matmul(const void *X, mnb_dtype act_t, const uint8_t *packed, const void *scales, mnb_dtype scale_t,
+                       const uint8_t *zp, void *Y, int64_t M, int64_t N, int64_t K, int bs, unsigned flags,
+                       void *stream);
+
 /* int8 embedding lookup ("Qwen3-ASR-0.6B -- ONNX for the browser",
  * "Building the prompt" step 4 and "Pick a variant": embed_tokens.int8.bin +
  * embed_scales.f32.bin):

@@ -24,7 +24,7 @@ __all__ = [
     "mnb_gemv", "mnb_gemm", "mnb_embed_gather", "mnb_device_status",
     "mnb_gemv_argmax", "mnb_gemv_argmax_workspace_bytes", "mnb_gemv_argmax_noalloc", "mnb_gemv_swiglu",
     "mnb_gemv_task", "mnb_gemv_chain_plan_bytes", "mnb_gemv_chain_workspace_bytes", "mnb_gemv_chain_plan",
-    "mnb_gemv_chain",
+    "mnb_gemv_chain", "mnb_matmul",
 ]
 
 MNB_F32, MNB_F16 = 0, 1
@@ -66,6 +66,7 @@ def _load():
         "mnb_dequantize": ([vp, vp, i32, vp, i64, i64, i32, vp, i32, vp], i32),
         "mnb_gemv": ([vp, i32, vp, vp, i32, vp, vp, i64, i64, i64, i32, u32, vp], i32),
         "mnb_gemm": ([vp, i32, vp, vp, i32, vp, vp, i64, i64, i64, i32, u32, vp], i32),
+        "mnb_matmul": ([vp, i32, vp, vp, i32, vp, vp, i64, i64, i64, i32, u32, vp], i32),
         "mnb_embed_gather": ([vp, vp, i64, i64, vp, i64, vp, i32, vp, vp], i32),
         "mnb_device_status": ([P(u32), i32], i32),
         "mnb_gemv_argmax_workspace_bytes": ([i64], sz),
@@ -223,6 +224,13 @@ def mnb_gemv_chain(plan, plan_device, workspace, flags=0, stream=None):
 def mnb_gemm(X, packed, scales, zp, Y, M, N, K, bs, flags=0, stream=None):
     """Y [M, N] = X [M, K] . dequant(W)^T on the tensor cores (fp16 X and Y)."""
     _check("mnb_gemm", _lib.mnb_gemm(
+        _ptr(X), _dt(X), _ptr(packed), _ptr(scales), _dt(scales), _ptr(zp), _ptr(Y),
+        M, N, K, bs, flags, _stream(stream)))
+
+
+def mnb_matmul(X, packed, scales, zp, Y, M, N, K, bs, flags=0, stream=None):
+    """Y [M, N] = X [M, K] . dequant(W)^T for any M, on the kernel that serves M best."""
+    _check("mnb_matmul", _lib.mnb_matmul(
         _ptr(X), _dt(X), _ptr(packed), _ptr(scales), _dt(scales), _ptr(zp), _ptr(Y),
         M, N, K, bs, flags, _stream(stream)))
 

@@ -14,7 +14,7 @@ import torch
 
 from . import (MNB_FLAG_PDL, mnb_dequantize, mnb_embed_gather, mnb_gemm, mnb_gemv, mnb_gemv_argmax,
                mnb_gemv_argmax_workspace_bytes, mnb_gemv_chain, mnb_gemv_chain_plan, mnb_gemv_chain_workspace_bytes,
-               mnb_gemv_swiglu, mnb_packed_sizes, mnb_quantize_rtn)
+               mnb_gemv_swiglu, mnb_matmul, mnb_packed_sizes, mnb_quantize_rtn)
 
 
 class QLinear:
@@ -53,6 +53,9 @@ class QLinear:
 
     def gemm(self, X, Y, flags=0, stream=None):
         mnb_gemm(X, self.packed, self.scales, self.zp, Y, X.shape[0], self.N, self.K, self.bs, flags, stream)
+
+    def matmul(self, X, Y, flags=0, stream=None):
+        mnb_matmul(X, self.packed, self.scales, self.zp, Y, X.shape[0], self.N, self.K, self.bs, flags, stream)
 
 
 def concat_linears(parts, name=""):
@@ -118,7 +121,8 @@ def fuse_decoder(linears, swiglu=False):
 class Pass:
     """A chain of MatMulNBits calls with one X / Y buffer pair per linear.
 
-    kind = "gemv" (decode step, M <= 16) or "gemm" (prefill).  With pdl=True each
+    kind = "gemv" (decode step, M <= 16), "gemm" (prefill) or "matmul" (any M:
+    mnb_matmul picks the kernel).  With pdl=True each
     launch may overlap the tail of the previous one (weights stream early, X is
     read after the previous kernel completes).  An optional int8 embedding
     gather of M token ids runs first, as in a decode step.
@@ -196,6 +200,8 @@ class Pass:
                     l.gemv_swiglu(x, y, flags, stream)
                 else:
                     l.gemv(x, y, flags, stream)
+            elif self.kind == "matmul":
+                l.matmul(x, y, flags, stream)
             else:
                 l.gemm(x, y, flags, stream)
 

@@ -188,3 +188,13 @@ def test_gemv_chain_argument_checks(mnb, lib):
     assert f(None, A, A, ws, 0, None) == INVALID
     assert f(plan, A + 32, A, ws, 0, None) == ALIGN           # device plan not 64-byte aligned
     assert f(plan, A, A, ws, 0x80, None) == INVALID           # unknown flag
+
+
+def test_matmul_argument_checks(lib):
+    f = lib.mnb_matmul
+    assert f(A, F16, A, A, F16, A, A, 17, 128, 96, 64, 0, None) == SHAPE        # K % bs
+    assert f(A, F16, A, A, F16, A, A, 17, 128, 64, 48, 0, None) == SHAPE        # bs
+    assert f(A + 8, F16, A, A, F16, A, A, 17, 128, 64, 32, 0, None) == ALIGN    # X not 16-byte aligned
+    assert f(A, F16, A, A, F16, A, A, 17, 128, 64, 32, 0x80, None) == INVALID   # unknown flag
+    assert f(A, 7, A, A, F16, A, A, 17, 128, 64, 32, 0, None) == INVALID        # dtype
+    assert f(A, F16, A, A, F16, A, A, 0, 128, 64, 32, 0, None) == OK            # M = 0: nothing to do

@@ -185,6 +185,16 @@ def test_qwen3_1p7b_prefill_fused_layout(step_mod, cuda_dev):
     check_pass(cfg, lins, samples, v, "f16")
 
 
+@pytest.mark.parametrize("M", [17, 20, 32, 63])
+def test_qwen3_1p7b_cached_prefill(step_mod, cuda_dev, M):
+    # mnb_matmul: GEMV launches of 16 tokens up to M = 20, the tensor-core GEMM above
+    cfg, lins, samples = model(step_mod, "qwen3_1p7b_cached_prefill", 24)
+    p = step_mod.Pass(lins, M, "matmul", torch.float16)
+    _fill_inputs(p, cfg["seed"] + M, torch.float16)
+    _run_graph(p)
+    check_pass(cfg, lins, samples, p, "f16")
+
+
 @pytest.mark.parametrize("M", [42, 390])
 def test_audio_encoder_prefill(step_mod, cuda_dev, M):
     cfg, lins, samples = model(step_mod, "audio_encoder_prefill", 24)

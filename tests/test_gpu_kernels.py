@@ -414,6 +414,24 @@ def test_gemm_q_equal_zp_gives_exact_zero(mnb, cuda_dev):
 
 # ------------------------------------------------------------------ embedding gather
 
+@pytest.mark.parametrize("M,N,K,bs,has_zp,act", [
+    (1, 256, 512, 32, True, "f16"), (16, 384, 1024, 32, True, "f16"), (17, 384, 1024, 32, True, "f16"),
+    (20, 256, 2048, 64, True, "f16"), (21, 256, 512, 32, False, "f16"), (33, 1024, 256, 32, True, "f16"),
+    (64, 128, 1024, 32, True, "f16"), (130, 384, 512, 64, False, "f16"), (40, 200, 512, 32, True, "f16"),
+    (17, 256, 512, 32, True, "f32"), (40, 130, 256, 64, True, "f32")])
+def test_matmul_dispatch(mnb, cuda_dev, M, N, K, bs, has_zp, act):
+    # one entry point for any M: GEMV launches of up to 16 tokens or the GEMM
+    rng = np.random.default_rng(M * 7 + N + K)
+    packed, scales, zp = random_packed(rng, N, K, bs, has_zp, np.float16)
+    tdt = torch.float16 if act == "f16" else torch.float32
+    X = torch.randn((M, K), generator=torch.Generator().manual_seed(M + K)).to(tdt)
+    Y = torch.full((M, N), float("nan"), dtype=tdt, device=cuda_dev)
+    mnb.mnb_matmul(X.to(cuda_dev), to_dev(packed, cuda_dev), to_dev(scales, cuda_dev), to_dev(zp, cuda_dev), Y,
+                   M, N, K, bs)
+    torch.cuda.synchronize()
+    assert_close(np_of(Y.float()), oracle.matmul(X.float().numpy(), packed, scales, zp, K, bs), act)
+
+
 @pytest.mark.parametrize("V,D,T", [(1000, 1024, 4096), (50, 16, 1), (300, 80, 37)])
 @pytest.mark.parametrize("odt", [torch.float16, torch.float32])
 def test_embed_gather_bit_exact(mnb, cuda_dev, V, D, T, odt):

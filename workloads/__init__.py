@@ -73,8 +73,9 @@ def qwen3_1p7b(lm_head=True, layers=N_LAYERS):
     return decoder_linears(2048, 2048, 1024, 6144, lm_head, layers)
 
 
-# The five workloads.  'gemv_M' lists go to the decode kernel, 'gemm_M' to the
-# tensor-core kernel.
+# The five workloads, and three more shapes of the same decoders.  'gemv_M'
+# lists go to the decode kernel, 'gemm_M' to the tensor-core kernel, 'matmul_M'
+# to mnb_matmul (which picks one).
 CONFIGS = {
     "single_gemv": dict(desc="single GEMV M=1 K=1024 N=2048 bs32 zp, fp32 activations",
                         seed=0, bs=32, has_zp=True, act="f32", scale="f32",
@@ -94,6 +95,12 @@ CONFIGS = {
     "qwen3_0p6b_nozp": dict(desc="Qwen3-0.6B shapes, block 32 without zero points (zp = 8)",
                             seed=4, bs=32, has_zp=False, act="f16", scale="f16",
                             model="0.6b", gemv_M=[1, 4, 16], gemm_M=[64, 390]),
+    # a prompt appended to a cached one: a few to a few dozen new tokens through
+    # the 1.7B decoder's projections, between the decode and prefill regimes
+    "qwen3_1p7b_cached_prefill": dict(desc="Qwen3-1.7B-shaped prefill of 17-63 new tokens, fp16, bs32 zp, no lm_head",
+                                      seed=6, bs=32, has_zp=True, act="f16", scale="f16",
+                                      model="1.7b", lm_head=False, gemv_M=[], gemm_M=[],
+                                      matmul_M=[17, 20, 24, 32, 48, 63]),
     # the encoder's linears over one clip's audio tokens: 42 for a 3.2 s command,
     # 390 for a 30 s clip (the audio-token count of "Building the prompt", step 2)
     "audio_encoder_prefill": dict(desc="24-layer Whisper-style audio encoder linears (d 1024, FFN 4096), fp16, bs32 zp",
