@@ -525,8 +525,8 @@ def run_gpu(args, world, rank, local):
         torch.cuda.empty_cache()
     del fbody
     # a prompt appended to a cached one: 17-63 new tokens through mnb_matmul,
-    # which runs GEMV launches of 16 tokens up to M = 20 and the GEMM above
-    # (same shapes as the prefill pass; its weights)
+    # which runs the decode GEMV up to M = 24 and the GEMM above (same shapes as
+    # the prefill pass; its weights)
     cached = {}
     for M in (17, 20, 24, 32, 48, 63):
         pc = Pass(body, M, "matmul", torch.float16, pdl=True)
@@ -537,7 +537,7 @@ def run_gpu(args, world, rank, local):
         cached[str(M)] = {"ms_per_pass": round(t, 4), "tflops": round(tflops, 1),
                           "weight_gbs": round(pc.weight_bytes / (t * 1e-3) / 1e9, 1),
                           "frac_hbm": round(pc.weight_bytes / (t * 1e-3) / 1e9 / hbm, 4),
-                          "path": "gemv, 2 launches per projection" if M <= 20 else "gemm"}
+                          "path": "gemv" if M <= 24 else "gemm"}
         del pc
         torch.cuda.empty_cache()
     # the same GEMM on a 24-layer audio encoder's linears over one clip's audio tokens

@@ -118,13 +118,15 @@ MNB_API int mnb_dequantize(const uint8_t *packed, const void *scales, mnb_dtype 
                    const uint8_t *zp, int64_t N, int64_t K, int bs, void *W_out,
                    mnb_dtype out_t, void *stream);
 
-/* Decode-shaped MatMulNBits, 1 <= M <= 16 (the autoregressive step of
+/* Decode-shaped MatMulNBits, 1 <= M <= 16 with fp32 activations and
+ * 1 <= M <= 32 with fp16 activations (the autoregressive step of
  * "Qwen3-ASR-0.6B -- ONNX for the browser", "Graph contracts": decoder_step,
- * input_embeds [1, 1, 1024]).  Y = X . dequant(W)^T.
+ * input_embeds [1, 1, 1024], batched or over a few appended prompt tokens).
+ * Y = X . dequant(W)^T.
  *   act_t  = dtype of X and Y (fp32 or fp16); scale_t = dtype of scales.
  *   Accumulation is fp32.  Bandwidth-bound: streams the packed weights once.
  * Errors: MNB_ERR_INVALID_ARG, MNB_ERR_SHAPE, MNB_ERR_ALIGN,
- *         MNB_ERR_UNSUPPORTED (M > 16), MNB_ERR_CUDA. */
+ *         MNB_ERR_UNSUPPORTED (M above the limit), MNB_ERR_CUDA. */
 MNB_API int mnb_gemv(const void *X, mnb_dtype act_t, const uint8_t *packed, const void *scales,
              mnb_dtype scale_t, const uint8_t *zp, void *Y, int64_t M, int64_t N, int64_t K,
              int bs, unsigned flags, void *stream);
@@ -206,12 +208,11 @@ MNB_API int mnb_gemm(const void *X, mnb_dtype act_t, const uint8_t *packed, cons
  * decoder_step), prefill of a prompt appended to a cached one (a few to a few
  * dozen new tokens) and full prefill (decoder_init / decoder_prefill) all take
  * this one call:
- *   M <= 16: mnb_gemv;
- *   17 <= M <= 20, fp16 X: mnb_gemv launches of 16 tokens and the rest
- *     (measured faster than the tensor-core GEMM there);
- *   M >= 21 with fp16 X, N % 128 == 0, K % 64 == 0: mnb_gemm;
+ *   M <= 24 with fp16 X (M <= 16 with fp32 X): one mnb_gemv (measured faster
+ *     than the tensor-core GEMM up to 24 tokens);
+ *   M >= 25 with fp16 X, N % 128 == 0, K % 64 == 0: mnb_gemm;
  *   otherwise (fp32 X, or shapes the GEMM does not take): mnb_gemv launches
- *     of up to 16 tokens.
+ *     of up to 24 (fp16) or 16 (fp32) tokens.
  * Requires X, packed and Y 16-byte aligned.
  * Errors: MNB_ERR_INVALID_ARG, MNB_ERR_SHAPE, MNB_ERR_ALIGN, MNB_ERR_CUDA. */
 MNB_API int mnb_matmul(const void *X, mnb_dtype act_t, const uint8_t *packed, const void *scales, mnb_dtype scale_t,

@@ -177,8 +177,9 @@ int mnb_gemv(const void *X, mnb_dtype act_t, const uint8_t *packed, const void *
     int rc = check_matmul_args(fn, X, act_t, packed, scales, scale_t, Y, M, N, K, bs);
     if (rc)
         return rc;
-    if (M > 16)
-        return fail(MNB_ERR_UNSUPPORTED, "%s: M=%lld > 16 (use mnb_gemm)", fn, (long long)M);
+    if (M > 32 || (M > 16 && act_t != MNB_F16))
+        return fail(MNB_ERR_UNSUPPORTED, "%s: M=%lld above %d for %s activations (use mnb_gemm or mnb_matmul)", fn,
+                    (long long)M, act_t == MNB_F16 ? 32 : 16, act_t == MNB_F16 ? "fp16" : "fp32");
     if (flags & ~(unsigned)MNB_FLAG_PDL)
         return fail(MNB_ERR_INVALID_ARG, "%s: unknown flags 0x%x", fn, flags);
     if (M == 0 || N == 0)
@@ -282,11 +283,11 @@ int mnb_gemm(const void *X, mnb_dtype act_t, const uint8_t *packed, const void *
                        flags, (cudaStream_t)stream);
 }
 
-// Largest M the dispatcher serves with decode GEMV launches of up to 16 tokens
-// each before switching to the tensor-core GEMM (measured on the 1.7B decoder
-// projections: two GEMV launches beat the GEMM up to 20 tokens, the GEMM wins
-// from 24).
-static const int64_t kGemvChunksMaxM = 20;
+// Largest M the dispatcher serves with one decode GEMV launch before switching
+// to the tensor-core GEMM (measured on the 1.7B decoder projections, per
+// 196-projection pass: GEMV 1.84 / 2.16 / 2.53 ms against GEMM 2.51 / 2.51 /
+// 2.51 ms at M = 17 / 24 / 28).
+static const int64_t kGemvMaxM = 24;
 
 int mnb_matmul(const void *X, mnb_dtype act_t, const uint8_t *packed, const void *scales, mnb_dtype scale_t,
                const uint8_t *zp, void *Y, int64_t M, int64_t N, int64_t K, int bs, unsigned flags, void *stream) {
@@ -300,14 +301,16 @@ int mnb_matmul(const void *X, mnb_dtype act_t, const uint8_t *packed, const void
     if (M == 0 || N == 0)
         return MNB_OK;
     const bool gemm_ok = act_t == MNB_F16 && N % 128 == 0 && K % 64 == 0;
-    if (gemm_ok && M > kGemvChunksMaxM)
+    if (gemm_ok && M > kGemvMaxM)
         return launch_gemm(X, packed, scales, scale_t == MNB_F16, zp, Y, (int)M, (int)N, (int)K, bs, flags,
                            (cudaStream_t)stream);
-    // decode GEMV launches of up to 16 tokens; chunk offsets are multiples of 16
-    // rows, so every chunk keeps the 16-byte alignment of X and Y
+    // decode GEMV launches of up to 24 (fp16) or 16 (fp32) tokens; chunk
+    // offsets are multiples of 8 rows, so every chunk keeps the 16-byte
+    // alignment of X and Y
     const size_t elem = (act_t == MNB_F16) ? 2 : 4;
-    for (int64_t m0 = 0; m0 < M; m0 += 16) {
-        const int mc = (int)((M - m0 < 16) ? (M - m0) : 16);
+    const int64_t chunk = (act_t == MNB_F16) ? kGemvMaxM : 16;
+    for (int64_t m0 = 0; m0 < M; m0 += chunk) {
+        const int mc = (int)((M - m0 < chunk) ? (M - m0) : chunk);
         rc = launch_gemv(static_cast<const unsigned char *>(X) + (size_t)m0 * (size_t)K * elem, act_t == MNB_F16,
                          packed, scales, scale_t == MNB_F16, zp,
                          static_cast<unsigned char *>(Y) + (size_t)m0 * (size_t)N * elem, mc, (int)N, (int)K, bs,

@@ -585,7 +585,7 @@ int plan_gemv(int M, int N, int K, int esz, int MP, int sms, Params &p, int &gri
 int launch_gemv(const void *X, int act_f16, const uint8_t *packed, const void *scales,
                 int scale_f16, const uint8_t *zp, void *Y, int M, int N, int K, int bs,
                 unsigned flags, cudaStream_t s) {
-    if (act_f16 && M > g_gemv_f16_cc_max_m) {   // tensor-core paths, weights streamed by TMA
+    if (act_f16 && (M > g_gemv_f16_cc_max_m || M > 16)) {   // tensor-core paths, weights streamed by TMA
         if (g_gemv_stream) {
             const int rc = launch_gemv_stream(X, packed, scales, scale_f16, zp, Y, M, N, K, bs, flags, s);
             if (rc != 1)

@@ -1,4 +1,4 @@
-// gemv_tc.cu -- decode-shaped MatMulNBits with fp16 activations (1 <= M <= 16):
+// gemv_tc.cu -- decode-shaped MatMulNBits with fp16 activations (1 <= M <= 32):
 // Y[M][N] = X[M][K] . dequant(W)^T, the per-token decoder step of
 // "Qwen3-ASR-0.6B -- ONNX for the browser" ("Graph contracts": decoder_step)
 // and of "Mega-ASR -- INT4 ONNX (GPTQ-calibrated)" (decoder_step_int4).
@@ -326,9 +326,10 @@ __device__ void argmax_finish(const TcParams &p, float (&best_v)[NT][2], int (&b
 }
 
 template <int NT, class C>
-__global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_constant__ CUtensorMap wmap,
-                                                              const TcParams p) {
+__global__ void __launch_bounds__(kThreads, NT >= 4 ? 1 : 2) gemv_tc_kernel(const __grid_constant__ CUtensorMap wmap,
+                                                                           const TcParams p) {
     constexpr int MP = 8 * NT;
+    constexpr bool kArgmax = NT <= 2;   // greedy decoding serves M <= 16
     extern __shared__ unsigned char smem_raw[];
     const int tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
@@ -520,7 +521,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
                     if (m < p.M && n < p.N) {
                         const __half h = __float2half_rn(out[t][e]);
                         p.Y[(int64_t)m * p.N + n] = h;
-                        if (p.argmax)   // rows ascend within a lane: '>' keeps the first maximum
+                        if (kArgmax && p.argmax)   // rows ascend within a lane: '>' keeps the first maximum
                             if (__half2float(h) > best_v[t][e & 1]) {
                                 best_v[t][e & 1] = __half2float(h);
                                 best_i[t][e & 1] = n;
@@ -609,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
             for (int e = 0; e < 8; e++) acc[t][e >> 2][e & 3] = 0.f;
     }
 
-    if (p.argmax)
+    if (kArgmax && p.argmax)
         argmax_finish<NT>(p, best_v, best_i, reinterpret_cast<uint2 *>(red), warp, lane, g, c, tid);
 
     // every issued box was waited for above; after a timeout, let the copies
@@ -673,7 +674,7 @@ static int launch_tc_common(const void *X, const uint8_t *packed, const void *sc
     EncodeTiledFn encode = tensor_map_encoder();
     if (!encode)
         return fail(MNB_ERR_CUDA, "mnb_gemv: cuTensorMapEncodeTiled unavailable");
-    const int NT = (M <= 8) ? 1 : 2;
+    const int NT = (M <= 8) ? 1 : (M <= 16) ? 2 : 4;   // MMA column groups of 8 tokens
     const int MP = 8 * NT;
     const int sms = device_sm_count();
 
@@ -697,9 +698,10 @@ static int launch_tc_common(const void *X, const uint8_t *packed, const void *sc
     // costed in box-times on the busiest warp: rounds of tile groups x (boxes
     // per warp + a per-round reduction cost: none when warps own whole rows,
     // more when the partial sums meet across a cluster).  Fitted on the
-    // decoder shapes at M <= 8 (one MMA column group); at 9 <= M <= 16 a box
-    // costs twice as much (two column groups) and a cluster reduction grows
-    // with the cluster (measured: 3 box-times per CTA of the cluster).
+    // decoder shapes at M <= 8 (one MMA column group); with more column groups
+    // a box costs proportionally more and a cluster reduction grows with the
+    // cluster (measured at two groups: 3 box-times per CTA of the cluster).
+    // Four column groups take the registers of two CTAs: one CTA per SM.
     const int nbx_all = (K + kBoxK - 1) / kBoxK;
     auto smem_for = [&](int W, int S, int &nbx_w, int &kcta, int &xs_stride) {
         nbx_w = (nbx_all + W * S - 1) / (W * S);
@@ -719,7 +721,7 @@ static int launch_tc_common(const void *X, const uint8_t *packed, const void *sc
             const size_t sm_ = smem_for(w, sc, nbx_w, kcta, xs_stride);
             if (sm_ > 200 * 1024)
                 continue;
-            const int per_sm = (sm_ <= 110 * 1024) ? 2 : 1;
+            const int per_sm = (NT < 4 && sm_ <= 110 * 1024) ? 2 : 1;
             double cost;
             if (w == 1 && sc == 1) {
                 const int warps = sms * per_sm * kWarps;
@@ -730,7 +732,7 @@ static int launch_tc_common(const void *X, const uint8_t *packed, const void *sc
                 int maxcl = sms * per_sm / sc;
                 if (maxcl < 1) maxcl = 1;
                 const int rounds = (groups + maxcl - 1) / maxcl;
-                const double red = (sc == 1) ? 0.5 * groups_f : (NT == 1 ? 1.6 : 3.0 * sc);
+                const double red = (sc == 1) ? 0.5 * groups_f : (NT == 1 ? 1.6 : 1.5 * groups_f * sc);
                 cost = rounds * (1.15 * groups_f * nbx_w + red);
             }
             if (W == 0 || cost < best - 1e-9 || (cost < best + 1e-9 && sc < S) ||
@@ -755,7 +757,7 @@ static int launch_tc_common(const void *X, const uint8_t *packed, const void *sc
     if (smem > 220 * 1024)
         return fail(MNB_ERR_SHAPE, "mnb_gemv: K=%d too large for M=%d", K, M);
     p.independent = (p.W == 1 && p.S == 1);
-    const int per_sm = (smem <= 110 * 1024) ? 2 : 1;
+    const int per_sm = (NT < 4 && smem <= 110 * 1024) ? 2 : 1;
     int grid;
     if (p.independent) {
         const int groups = (p.ntiles + kWarps - 1) / kWarps;
@@ -792,8 +794,10 @@ static int launch_tc_common(const void *X, const uint8_t *packed, const void *sc
     if (has_zp) { MNB_TC_S(NT_, B_, true); } else { MNB_TC_S(NT_, B_, false); }
     if (NT == 1) {
         if (bs64) { MNB_TC_Z(1, true); } else { MNB_TC_Z(1, false); }
-    } else {
+    } else if (NT == 2) {
         if (bs64) { MNB_TC_Z(2, true); } else { MNB_TC_Z(2, false); }
+    } else {
+        if (bs64) { MNB_TC_Z(4, true); } else { MNB_TC_Z(4, false); }
     }
 #undef MNB_TC_Z
 #undef MNB_TC_S

@@ -121,7 +121,7 @@ def fuse_decoder(linears, swiglu=False):
 class Pass:
     """A chain of MatMulNBits calls with one X / Y buffer pair per linear.
 
-    kind = "gemv" (decode step, M <= 16), "gemm" (prefill) or "matmul" (any M:
+    kind = "gemv" (decode step, M <= 32), "gemm" (prefill) or "matmul" (any M:
     mnb_matmul picks the kernel).  With pdl=True each
     launch may overlap the tail of the previous one (weights stream early, X is
     read after the previous kernel completes).  An optional int8 embedding

@@ -74,7 +74,8 @@ def test_packed_sizes_rejects(lib):
 
 def test_gemv_argument_checks(lib):
     g = lib.mnb_gemv
-    assert g(A, F16, A, A, F16, A, A, 17, 64, 64, 32, 0, None) == UNSUPPORTED
+    assert g(A, F16, A, A, F16, A, A, 33, 64, 64, 32, 0, None) == UNSUPPORTED    # fp16: M <= 32
+    assert g(A, F32, A, A, F32, A, A, 17, 64, 64, 32, 0, None) == UNSUPPORTED    # fp32: M <= 16
     assert g(A, F16, A, A, F16, A, A, 1, 64, 96, 64, 0, None) == SHAPE          # K % bs
     assert g(A, F16, A, A, F16, A, A, 1, 64, 64, 16, 0, None) == SHAPE          # bs
     assert g(None, F16, A, A, F16, A, A, 1, 64, 64, 32, 0, None) == INVALID

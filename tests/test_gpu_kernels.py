@@ -111,6 +111,12 @@ GEMV_CASES = [
     (6, 2000, 2048, 64, True, "f16", np.float16),
     (1, 300, 4096, 64, False, "f16", np.float32),
     (4, 3333, 1024, 32, False, "f16", np.float16),
+    # four MMA column groups (17 <= M <= 32)
+    (17, 2048, 2048, 32, True, "f16", np.float16),
+    (24, 1000, 6144, 32, True, "f16", np.float16),
+    (32, 6144, 2048, 32, True, "f16", np.float16),
+    (32, 300, 1024, 64, False, "f16", np.float32),
+    (29, 151936 // 8, 1024, 32, True, "f16", np.float16),
 ]
 
 
