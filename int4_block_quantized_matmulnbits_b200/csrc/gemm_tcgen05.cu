@@ -158,6 +158,29 @@ __device__ __forceinline__ float4 ld_dsmem_f4(const float *local, uint32_t rank)
     return v;
 }
 
+// Adds the NPEER other cluster ranks' partial sums of NQ column quads (quads
+// q0 .. q0+NQ-1 of a 16-column chunk) to f: every remote load is issued before
+// the first add (a remote shared-memory read takes about a microsecond), and
+// the adds run in rank order, so the sum does not depend on timing.
+template <int NPEER, int NQ>
+__device__ __forceinline__ void add_peers(float f[16], const float *chunk, int rank, int q0) {
+    float4 o[NQ][NPEER];
+#pragma unroll
+    for (int j = 0; j < NQ; j++)
+#pragma unroll
+        for (int qi = 0; qi < NPEER; qi++)
+            o[j][qi] = ld_dsmem_f4(chunk + 4 * (q0 + j), (uint32_t)(qi + (qi >= rank ? 1 : 0)));
+#pragma unroll
+    for (int j = 0; j < NQ; j++)
+#pragma unroll
+        for (int qi = 0; qi < NPEER; qi++) {
+            f[4 * (q0 + j)] += o[j][qi].x;
+            f[4 * (q0 + j) + 1] += o[j][qi].y;
+            f[4 * (q0 + j) + 2] += o[j][qi].z;
+            f[4 * (q0 + j) + 3] += o[j][qi].w;
+        }
+}
+
 // Scale (fp16 bits) and zero point of one thread's 32-k half of a stage (one
 // block of 32, or half a block of 64).
 struct SZ {
@@ -440,21 +463,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float4 o = own[j];
                     f[4 * j] = o.x; f[4 * j + 1] = o.y; f[4 * j + 2] = o.z; f[4 * j + 3] = o.w;
                 }
-                // the peers' partials: all loads of a column quad in flight at once,
-                // then the adds (in rank order, so the sum does not depend on timing)
+                // the peers' partials, requested together and added in rank order
+                const float *chunk = red + row * red_pitch + c16 * 16;
+                if (p.S == 2) {
+                    add_peers<1, 4>(f, chunk, rank, 0);
+                } else if (p.S == 4) {
+                    add_peers<3, 2>(f, chunk, rank, 0);   // two halves of the chunk: fewer live registers
+                    add_peers<3, 2>(f, chunk, rank, 2);
+                } else {
 #pragma unroll
-                for (int j = 0; j < 4; j++) {
-                    float4 o4[kMaxCluster];
+                    for (int j = 0; j < 4; j++) {
+                        float4 o4[kMaxCluster];
 #pragma unroll
-                    for (int qq = 0; qq < kMaxCluster; qq++)
-                        if (qq < p.S && qq != rank)
-                            o4[qq] = ld_dsmem_f4(red + row * red_pitch + c16 * 16 + 4 * j, (uint32_t)qq);
+                        for (int qq = 0; qq < kMaxCluster; qq++)
+                            if (qq < p.S && qq != rank)
+                                o4[qq] = ld_dsmem_f4(red + row * red_pitch + c16 * 16 + 4 * j, (uint32_t)qq);
 #pragma unroll
-                    for (int qq = 0; qq < kMaxCluster; qq++)
-                        if (qq < p.S && qq != rank) {
-                            f[4 * j] += o4[qq].x; f[4 * j + 1] += o4[qq].y;
-                            f[4 * j + 2] += o4[qq].z; f[4 * j + 3] += o4[qq].w;
-                        }
+                        for (int qq = 0; qq < kMaxCluster; qq++)
+                            if (qq < p.S && qq != rank) {
+                                f[4 * j] += o4[qq].x; f[4 * j + 1] += o4[qq].y;
+                                f[4 * j + 2] += o4[qq].z; f[4 * j + 3] += o4[qq].w;
+                            }
+                    }
                 }
                 store_y(c16 * 16, f);
             }
