@@ -57,6 +57,7 @@ constexpr int kPR = 4;                         // stages of scales / zero points
 constexpr int kWS = 4;                         // fp16 weight tiles in the ring
 constexpr int kPS = 8;                         // packed weight tiles in flight
 constexpr int kMaxCluster = 8;
+constexpr uint32_t kChunkBytes = kBM * 16 * 4;   // one 16-column chunk of fp32 partial sums
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
 
 struct GemmParams {
@@ -147,38 +148,23 @@ __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ float4 ld_dsmem_f4(const float *local, uint32_t rank) {
+
+// Address of the same shared-memory location in cluster rank `rank`.
+__device__ __forceinline__ uint32_t map_cluster(uint32_t local, uint32_t rank) {
     uint32_t remote;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
-    float4 v;
-    asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(remote)
-                 : "memory");
-    return v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(rank));
+    return remote;
 }
 
-// Adds the NPEER other cluster ranks' partial sums of NQ column quads (quads
-// q0 .. q0+NQ-1 of a 16-column chunk) to f: every remote load is issued before
-// the first add (a remote shared-memory read takes about a microsecond), and
-// the adds run in rank order, so the sum does not depend on timing.
-template <int NPEER, int NQ>
-__device__ __forceinline__ void add_peers(float f[16], const float *chunk, int rank, int q0) {
-    float4 o[NQ][NPEER];
-#pragma unroll
-    for (int j = 0; j < NQ; j++)
-#pragma unroll
-        for (int qi = 0; qi < NPEER; qi++)
-            o[j][qi] = ld_dsmem_f4(chunk + 4 * (q0 + j), (uint32_t)(qi + (qi >= rank ? 1 : 0)));
-#pragma unroll
-    for (int j = 0; j < NQ; j++)
-#pragma unroll
-        for (int qi = 0; qi < NPEER; qi++) {
-            f[4 * (q0 + j)] += o[j][qi].x;
-            f[4 * (q0 + j) + 1] += o[j][qi].y;
-            f[4 * (q0 + j) + 2] += o[j][qi].z;
-            f[4 * (q0 + j) + 3] += o[j][qi].w;
-        }
+// Copies `bytes` from this CTA's shared memory into a cluster rank's, completing
+// on that rank's mbarrier.
+__device__ __forceinline__ void bulk_copy_to_rank(uint32_t dst_cluster, uint32_t src, uint32_t bytes,
+                                                  uint32_t bar_cluster) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            dst_cluster),
+        "r"(src), "r"(bytes), "r"(bar_cluster)
+        : "memory");
 }
 
 // Scale (fp16 bits) and zero point of one thread's 32-k half of a stage (one
@@ -272,7 +258,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto xfull = [&](int i) { return bars + 8u * (uint32_t)(2 * PS + 2 * WS + i % XS); };
     auto xempty = [&](int i) { return bars + 8u * (uint32_t)(2 * PS + 2 * WS + XS + i % XS); };
     const uint32_t acc_full = bars + 8u * (uint32_t)(2 * PS + 2 * WS + 2 * XS);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + (acc_full + 8 - base));
+    const uint32_t red_bar = acc_full + 8;   // K split: the other ranks' partial sums have landed
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + (acc_full + 16 - base));
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     if (tid == 0) {
@@ -289,6 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(xempty(i), 1);
         }
         mbar_init(acc_full, 1);
+        mbar_init(red_bar, 1);
         *abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -414,8 +402,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16);
         const int m0 = m_tile * BN;
         const int nchunk = BN / 16;
-        const int red_pitch = BN + 4;            // floats per row of the partial-sum buffer
-        float *red = reinterpret_cast<float *>(base_ptr);   // reuses the ring buffers
         const bool have = mbar_wait(acc_full, 0, abort) && nk > 0;
         tc_fence_after();
         pdl_wait();
@@ -440,55 +426,69 @@ __global__ void __launch_bounds__(kThreads, 1)
                 store_y(c16 * 16, f);
             }
         } else {
-            // park this rank's partial sums, then each rank reduces its own chunks
+            // K split over the cluster.  Each rank parks its partial sums
+            // chunk-major ([16-column chunk][row][16] fp32, 8 KB per chunk); chunk c
+            // belongs to rank c % S.  Every rank then sends each chunk it does not
+            // own to its owner with one bulk copy into the owner's receive area
+            // (shared-memory loads across the cluster, 16 bytes per request, were
+            // measured ~4x slower), completing on the owner's barrier; each owner
+            // adds the copies to its own sums in rank order and stores its chunks.
+            float *park = reinterpret_cast<float *>(base_ptr);   // reuses the ring buffers
+            const int owned_max = (nchunk + p.S - 1) / p.S;
+            float *recv = park + nchunk * kBM * 16;             // [S - 1 senders][owned_max][chunk]
             for (int c16 = grp; c16 < nchunk; c16 += 4) {
                 uint32_t v[16];
                 if (have) {
                     tc_ld16(taddr + (uint32_t)(c16 * 16), v);
                     tc_wait_ld();
                 }
-                float4 *dst = reinterpret_cast<float4 *>(red + row * red_pitch + c16 * 16);
+                float4 *dst = reinterpret_cast<float4 *>(park + (c16 * kBM + row) * 16);
 #pragma unroll
                 for (int j = 0; j < 4; j++)
                     dst[j] = have ? make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
                                                 __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]))
                                   : make_float4(0.f, 0.f, 0.f, 0.f);
             }
-            cluster_sync();
+            fence_proxy_async_smem();   // the bulk copies read the parked sums
+            if (warp == 3 && lane == 0) {
+                const int owned = (nchunk - rank + p.S - 1) / p.S;
+                mbar_expect_tx(red_bar, (uint32_t)((p.S - 1) * owned) * kChunkBytes);
+            }
+            cluster_sync();   // every rank has parked and armed its barrier
+            if (warp == 3 && lane == 0) {
+                for (int c16 = 0; c16 < nchunk; c16++) {
+                    const int owner = c16 % p.S;
+                    if (owner == rank)
+                        continue;
+                    const int slot = rank - (rank > owner ? 1 : 0);   // senders in rank order
+                    const uint32_t src = smem_u32(park + c16 * kBM * 16);
+                    const uint32_t dst = smem_u32(recv + (slot * owned_max + c16 / p.S) * kBM * 16);
+                    bulk_copy_to_rank(map_cluster(dst, (uint32_t)owner), src, kChunkBytes,
+                                      map_cluster(red_bar, (uint32_t)owner));
+                }
+            }
+            const bool got = mbar_wait(red_bar, 0, abort);
             for (int c16 = rank + p.S * grp; c16 < nchunk; c16 += 4 * p.S) {
                 float f[16];
-                const float4 *own = reinterpret_cast<const float4 *>(red + row * red_pitch + c16 * 16);
+                const float4 *own = reinterpret_cast<const float4 *>(park + (c16 * kBM + row) * 16);
 #pragma unroll
                 for (int j = 0; j < 4; j++) {
                     const float4 o = own[j];
                     f[4 * j] = o.x; f[4 * j + 1] = o.y; f[4 * j + 2] = o.z; f[4 * j + 3] = o.w;
                 }
-                // the peers' partials, requested together and added in rank order
-                const float *chunk = red + row * red_pitch + c16 * 16;
-                if (p.S == 2) {
-                    add_peers<1, 4>(f, chunk, rank, 0);
-                } else if (p.S == 4) {
-                    add_peers<3, 2>(f, chunk, rank, 0);   // two halves of the chunk: fewer live registers
-                    add_peers<3, 2>(f, chunk, rank, 2);
-                } else {
+                for (int sl = 0; sl < p.S - 1; sl++) {
+                    const float4 *in = reinterpret_cast<const float4 *>(recv + ((sl * owned_max + c16 / p.S) * kBM + row) * 16);
 #pragma unroll
                     for (int j = 0; j < 4; j++) {
-                        float4 o4[kMaxCluster];
-#pragma unroll
-                        for (int qq = 0; qq < kMaxCluster; qq++)
-                            if (qq < p.S && qq != rank)
-                                o4[qq] = ld_dsmem_f4(red + row * red_pitch + c16 * 16 + 4 * j, (uint32_t)qq);
-#pragma unroll
-                        for (int qq = 0; qq < kMaxCluster; qq++)
-                            if (qq < p.S && qq != rank) {
-                                f[4 * j] += o4[qq].x; f[4 * j + 1] += o4[qq].y;
-                                f[4 * j + 2] += o4[qq].z; f[4 * j + 3] += o4[qq].w;
-                            }
+                        const float4 o = in[j];
+                        f[4 * j] += o.x; f[4 * j + 1] += o.y; f[4 * j + 2] += o.z; f[4 * j + 3] += o.w;
                     }
                 }
+                if (!got)
+                    continue;
                 store_y(c16 * 16, f);
             }
-            cluster_sync();   // every rank has read what it needs: the buffers may go
+            cluster_sync();   // every copy into a rank has landed (it waited) before any rank exits
         }
     }
     if (p.S > 1 && warp < 3) {
@@ -564,11 +564,13 @@ int launch_gemm(const void *X, const uint8_t *packed, const void *scales, int sc
     if (xstages > 8) xstages = 8;
     if (xstages < 2) xstages = 2;
     const size_t ring_bytes = (size_t)fixed + (size_t)xstages * BN * 128;
-    // the cluster reduction reuses the rings for [128][BN + 4] fp32
-    if (S > 1 && ring_bytes < (size_t)kBM * (BN + 4) * 4)
+    // the cluster reduction reuses the rings: the parked sums [BN / 16][128][16]
+    // fp32 and the copies received from the other S - 1 ranks
+    const size_t chunks = (size_t)BN / 16, owned_max = (chunks + S - 1) / S;
+    if (S > 1 && ring_bytes < (chunks + (size_t)(S - 1) * owned_max) * kChunkBytes)
         return fail(MNB_ERR_SHAPE, "mnb_gemm: reduction buffer does not fit");
     p.xstages = xstages;
-    const size_t smem = 1024 + ring_bytes + 8 * (2 * kPS + 2 * kWS + 2 * xstages + 1) + 16;
+    const size_t smem = 1024 + ring_bytes + 8 * (2 * kPS + 2 * kWS + 2 * xstages + 2) + 16;
     if (smem > 232448)
         return fail(MNB_ERR_SHAPE, "mnb_gemm: shared memory plan too large");
 
