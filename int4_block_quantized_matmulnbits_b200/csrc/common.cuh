@@ -120,4 +120,39 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *map, uint3
 
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
+// ---- cluster, MMA and int4 unpack helpers shared by the kernels ------------
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// D += A . B on the legacy tensor path: m16n8k16, fp16 inputs, fp32 accumulator.
+__device__ __forceinline__ void mma16816(float d[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// One 32-bit word of nibbles e0..e7 of a row -> the A-operand half2 (e0,e4),
+// 16(e1,e5), (e2,e6), 16(e3,e7): (1024 + q) - (1024 + zp) = q - zp exactly,
+// times the fp16 scale = fp16_rn((q - zp) * s) (x16 for the high nibbles, also
+// exact).  Z = 1024 + zp and Zhi = 1024 + 16 zp as fp16 pairs.
+__device__ __forceinline__ void dq_word(uint32_t w, uint32_t s2, uint32_t Z, uint32_t Zhi, uint32_t &a0,
+                                        uint32_t &a1, uint32_t &a2, uint32_t &a3) {
+    const uint32_t w8 = w >> 8;
+    const half2 s = u32_as_h2(s2);
+    a0 = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(w, 0x000F000Fu, 0x64006400u)), u32_as_h2(Z)), s));
+    a1 = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(w, 0x00F000F0u, 0x64006400u)), u32_as_h2(Zhi)), s));
+    a2 = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(w8, 0x000F000Fu, 0x64006400u)), u32_as_h2(Z)), s));
+    a3 = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(w8, 0x00F000F0u, 0x64006400u)), u32_as_h2(Zhi)), s));
+}
+
 }  // namespace mnb

@@ -111,13 +111,6 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *map, uint3
         : "memory");
 }
 
-__device__ __forceinline__ void mma16816(float d[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
 
 // One 32-bit word of nibbles e0..e7 of a row -> the fp16 pairs (e0,e4) (e1,e5)
 // (e2,e6) (e3,e7) of fp16_rn((q - zp) * scale).  q - zp is exact first:

@@ -88,15 +88,7 @@ struct TcParams {
     unsigned *ws_count;   // CTAs done; the last one resets it to 0
 };
 
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
 
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
 
 __device__ __forceinline__ float ld_dsmem_f32(const float *local, uint32_t rank) {
     uint32_t remote;
@@ -106,13 +98,6 @@ __device__ __forceinline__ float ld_dsmem_f32(const float *local, uint32_t rank)
     return v;
 }
 
-__device__ __forceinline__ void mma16816(float d[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
 
 // Bounded wait on a warp-private mbarrier.  After the first timeout (*dead set)
 // it returns at once, so the warp runs to the end without waiting again.
@@ -218,19 +203,6 @@ __device__ __forceinline__ void param_next_box(const TcParams &p, ParamCursor &q
     q.k0 += kBoxK;
 }
 
-// One 32-bit word of nibbles (e0..e7) of a row -> the four A-operand half2
-// (e0,e4), 16*(e1,e5), (e2,e6), 16*(e3,e7): (1024 + q) - (1024 + zp) = q - zp
-// exactly, times the scale = fp16_rn((q - zp) * s) (x16 for the high nibbles,
-// exact).
-__device__ __forceinline__ void dq_word(uint32_t w, uint32_t s2, uint32_t Z, uint32_t Zhi, uint32_t &a0,
-                                        uint32_t &a1, uint32_t &a2, uint32_t &a3) {
-    const uint32_t w8 = w >> 8;
-    const half2 s = u32_as_h2(s2);
-    a0 = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(w, 0x000F000Fu, 0x64006400u)), u32_as_h2(Z)), s));
-    a1 = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(w, 0x00F000F0u, 0x64006400u)), u32_as_h2(Zhi)), s));
-    a2 = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(w8, 0x000F000Fu, 0x64006400u)), u32_as_h2(Z)), s));
-    a3 = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(w8, 0x00F000F0u, 0x64006400u)), u32_as_h2(Zhi)), s));
-}
 
 // silu(x) = x * sigmoid(x), in fp32.
 __device__ __forceinline__ float silu(float x) { return x / (1.0f + __expf(-x)); }
