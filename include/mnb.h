@@ -269,7 +269,9 @@ MNB_API int mnb_embed_gather(const int8_t *table, const float *row_scales, int64
  * Failure: a wait inside the kernel that exceeds 2 s sets bit 1 (a weight
  * copy) or bit 2 (a task's inputs) of the status word read by
  * mnb_device_status; the kernel then exits early, Y is undefined and the
- * workspace must be zero-filled again.
+ * workspace must be zero-filled again.  A call that finds the workspace's
+ * abort word still set (a failed call before it) runs no task, writes no Y
+ * and sets bit 3.
  * Errors: MNB_ERR_INVALID_ARG, MNB_ERR_SHAPE, MNB_ERR_ALIGN,
  *         MNB_ERR_UNSUPPORTED (M > 8, mixed layouts), MNB_ERR_CUDA. */
 typedef struct mnb_gemv_task {
@@ -291,7 +293,8 @@ MNB_API int mnb_gemv_chain(const void *plan, const void *plan_device, void *work
                            unsigned flags, void *stream);
 
 /* Reads (and, if clear != 0, zeroes) the library's device status word on the
- * current device: bit 0 = a GEMM mbarrier wait timed out.  Synchronizes the
+ * current device: bit 0 = a GEMM or GEMV mbarrier wait timed out; bits 1-3 =
+ * mnb_gemv_chain (see there).  Synchronizes the
  * device.  Errors: MNB_ERR_INVALID_ARG (NULL), MNB_ERR_CUDA. */
 MNB_API int mnb_device_status(unsigned *status_out, int clear);
 

@@ -34,7 +34,8 @@
 // failure in a device status word and in the workspace's abort word, which the
 // other CTAs poll; all CTAs then leave the task loop together, drain their
 // copies and exit.  The counters are then left as they were: the caller zeroes
-// the workspace before the next call.
+// the workspace before the next call, and a call that finds the abort word set
+// runs no task (status bit) rather than trust stale counters.
 #include <cuda.h>
 
 #include <algorithm>
@@ -311,8 +312,16 @@ __global__ void __launch_bounds__(kMaxThreads, 1) gemv_chain_kernel(const ChainP
     }
     pdl_wait();
     const half2 sixteenth = __floats2half2_rn(0.0625f, 0.0625f);
+    // an abort word left set by a call that failed: the counters may be stale,
+    // so run nothing (the caller zero-fills the workspace again)
+    if (tid == ctl && ld_acquire_gpu(p.cnt + p.ntasks) != 0u) {
+        flags[0] = 1;
+        atomicOr(&g_chain_status, 4u);
+    }
+    __syncthreads();
+    const int ntasks_run = flags[0] ? 0 : p.ntasks;
 
-    for (int j = 0; j < p.ntasks; j++) {
+    for (int j = 0; j < ntasks_run; j++) {
         const TaskInfo *t = ti + j;
         const int nbx = t->nbx, N = t->N;
         __half *Y = t->Y;
@@ -719,7 +728,7 @@ int read_chain_status(unsigned *out, int clear) {
     }
     if (e != cudaSuccess)
         return fail(MNB_ERR_CUDA, "mnb_device_status: %s", cudaGetErrorString(e));
-    *out |= v << 1;   // bits 1 (a weight copy) and 2 (a task's inputs)
+    *out |= v << 1;   // bits 1 (a weight copy), 2 (a task's inputs), 3 (a workspace left dirty)
     return MNB_OK;
 }
 

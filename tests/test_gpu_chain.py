@@ -149,3 +149,28 @@ def test_chain_q_equal_zp_gives_exact_zero(mnb, cuda_dev):
     tasks = [(x, to_dev(packed, cuda_dev), to_dev(scales, cuda_dev), to_dev(zb, cuda_dev), Y, N, K, 0)]
     _run(mnb, tasks, M, 32, cuda_dev)
     assert int(Y.count_nonzero()) == 0
+
+
+def test_chain_refuses_a_workspace_left_dirty(mnb, cuda_dev):
+    # a failed call leaves the abort word set; the next call must run nothing
+    # and say so, and run normally once the workspace is zero-filled again
+    rng = np.random.default_rng(4)
+    M, N, K = 1, 2048, 1024
+    host, dev_w = _weights(rng, N, K, 32, True, cuda_dev)
+    x = torch.randn((M, K), generator=torch.Generator().manual_seed(8)).half().to(cuda_dev)
+    Y = torch.full((M, N), 7.0, dtype=torch.float16, device=cuda_dev)
+    tasks = [(x, *dev_w, Y, N, K, 0)]
+    plan = mnb.mnb_gemv_chain_plan(tasks, M, 32)
+    plan_dev = plan.to(cuda_dev)
+    ws = torch.zeros(mnb.mnb_gemv_chain_workspace_bytes(1), dtype=torch.uint8, device=cuda_dev)
+    ws.view(torch.int32)[1] = 1   # the abort word follows the one task counter
+    mnb.mnb_device_status(clear=True)
+    mnb.mnb_gemv_chain(plan, plan_dev, ws)
+    torch.cuda.synchronize()
+    assert mnb.mnb_device_status(clear=True) & (1 << 3)
+    assert bool((Y == 7.0).all()), "no task may run on a dirty workspace"
+    ws.zero_()
+    mnb.mnb_gemv_chain(plan, plan_dev, ws)
+    torch.cuda.synchronize()
+    assert mnb.mnb_device_status() == 0
+    assert_close(np_of(Y.float()), oracle.matmul(np_of(x.float()), *host, K, 32), "f16")
