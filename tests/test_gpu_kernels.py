@@ -404,6 +404,25 @@ def test_gemm_matches_dequantized_weights_exactly_where_exact(mnb, cuda_dev):
     assert np.array_equal(np_of(Y).astype(np.float64), ref.astype(np.float16).astype(np.float64))
 
 
+@pytest.mark.parametrize("M,N,K", [(1024, 256, 512), (64, 1024, 2048), (256, 512, 2048)])
+def test_gemm_split_k_is_deterministic(mnb, cuda_dev, M, N, K):
+    # these shapes split K over 2- and 4-CTA clusters; the owner of each column
+    # chunk adds the other ranks' partial sums in rank order, so repeated calls
+    # give the same bits
+    rng = np.random.default_rng(M + N)
+    packed, scales, zp = random_packed(rng, N, K, 32, True, np.float16)
+    dp, ds, dz = to_dev(packed, cuda_dev), to_dev(scales, cuda_dev), to_dev(zp, cuda_dev)
+    X = torch.randn((M, K), generator=torch.Generator().manual_seed(N)).half().to(cuda_dev)
+    outs = []
+    for _ in range(3):
+        Y = torch.empty((M, N), dtype=torch.float16, device=cuda_dev)
+        mnb.mnb_gemm(X, dp, ds, dz, Y, M, N, K, 32)
+        outs.append(Y)
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
+    assert_close(np_of(outs[0].float()), oracle.matmul(np_of(X.float()), packed, scales, zp, K, 32), "f16")
+
+
 def test_gemm_q_equal_zp_gives_exact_zero(mnb, cuda_dev):
     N, K, bs, M = 128, 256, 64, 70
     z = np.random.default_rng(2).integers(0, 16, (N, K // bs))
