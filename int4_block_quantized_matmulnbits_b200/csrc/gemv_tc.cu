@@ -394,11 +394,15 @@ __global__ void __launch_bounds__(kThreads, NT >= 4 ? 1 : 2) gemv_tc_kernel(cons
     }
     __syncthreads();
 
-    float acc[NT][2][4];       // two accumulator chains (chunk 2c and 2c+1)
+    // independent MMA accumulator chains per token group: chunk 2c + h, and with
+    // one column group also the word parity (shorter dependency chains;
+    // measured 1.4 % faster on the 1.7B step at M = 1, slower at M = 16)
+    constexpr int kChains = (NT == 1) ? 4 : 2;
+    float acc[NT][kChains][4];
 #pragma unroll
     for (int t = 0; t < NT; t++)
 #pragma unroll
-        for (int e = 0; e < 8; e++) acc[t][e >> 2][e & 3] = 0.f;
+        for (int e = 0; e < 4 * kChains; e++) acc[t][e >> 2][e & 3] = 0.f;
 
     bool dead = false;
     int tile = first_tile, j = 0, r = 0;
@@ -446,8 +450,9 @@ __global__ void __launch_bounds__(kThreads, NT >= 4 ? 1 : 2) gemv_tc_kernel(cons
                     uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
                     dq_word(wa[w], sa, Za, Zha, a0, a1, a2, a3);
                     dq_word(wb[w], sb, Zb, Zhb, b0, b1, b2, b3);
-                    mma16816(acc[t][h], a0, b0, a1, b1, xv.x, xv.y);
-                    mma16816(acc[t][h], a2, b2, a3, b3, xv.z, xv.w);
+                    float *ac = acc[t][kChains == 4 ? 2 * h + (w & 1) : h];
+                    mma16816(ac, a0, b0, a1, b1, xv.x, xv.y);
+                    mma16816(ac, a2, b2, a3, b3, xv.z, xv.w);
                 }
             }
         }
@@ -472,7 +477,11 @@ __global__ void __launch_bounds__(kThreads, NT >= 4 ? 1 : 2) gemv_tc_kernel(cons
 #pragma unroll
         for (int t = 0; t < NT; t++)
 #pragma unroll
-            for (int e = 0; e < 4; e++) out[t][e] = acc[t][0][e] + acc[t][1][e];
+            for (int e = 0; e < 4; e++) {
+                out[t][e] = acc[t][0][e] + acc[t][1][e];
+                if (kChains == 4)
+                    out[t][e] += acc[t][kChains - 2][e] + acc[t][kChains - 1][e];
+            }
         const int tile_done = tile;
         tile = ntile;
         j = 0;
@@ -579,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, NT >= 4 ? 1 : 2) gemv_tc_kernel(cons
 #pragma unroll
         for (int t = 0; t < NT; t++)
 #pragma unroll
-            for (int e = 0; e < 8; e++) acc[t][e >> 2][e & 3] = 0.f;
+            for (int e = 0; e < 4 * kChains; e++) acc[t][e >> 2][e & 3] = 0.f;
     }
 
     if (kArgmax && p.argmax)
