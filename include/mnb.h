@@ -64,7 +64,7 @@ enum {
     MNB_ERR_INVALID_ARG = -1, /* NULL pointer, negative size, unknown dtype     */
     MNB_ERR_SHAPE = -2,       /* bs not 32/64, K % bs != 0, size too large      */
     MNB_ERR_ALIGN = -3,       /* a pointer is not aligned as documented         */
-    MNB_ERR_UNSUPPORTED = -4, /* a valid request this build does not serve      */
+    MNB_ERR_UNSUPPORTED = -4, /* a valid request the library does not serve     */
     MNB_ERR_CUDA = -5,        /* a CUDA runtime call or launch failed           */
     MNB_ERR_TIMEOUT = -6      /* a device-side bounded wait gave up (see below) */
 };
