@@ -406,16 +406,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         };
         if (p.S == 1) {
-            for (int c16 = grp; c16 < nchunk; c16 += 4) {
-                uint32_t v[16];
-                float f[16];
+            // two 16-column chunks per tensor-memory load round trip
+            for (int c16 = grp; c16 < nchunk; c16 += 8) {
+                const bool two = c16 + 4 < nchunk;
+                uint32_t v[2][16];
                 if (have) {
-                    tc_ld16(taddr + (uint32_t)(c16 * 16), v);
+                    tc_ld16(taddr + (uint32_t)(c16 * 16), v[0]);
+                    if (two)
+                        tc_ld16(taddr + (uint32_t)((c16 + 4) * 16), v[1]);
                     tc_wait_ld();
                 }
 #pragma unroll
-                for (int j = 0; j < 16; j++) f[j] = have ? __uint_as_float(v[j]) : 0.f;
-                store_y(c16 * 16, f);
+                for (int h = 0; h < 2; h++) {
+                    if (h == 1 && !two)
+                        break;
+                    float f[16];
+#pragma unroll
+                    for (int j = 0; j < 16; j++) f[j] = have ? __uint_as_float(v[h][j]) : 0.f;
+                    store_y((c16 + 4 * h) * 16, f);
+                }
             }
         } else {
             // K split over the cluster.  Each rank parks its partial sums
@@ -428,18 +437,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             float *park = reinterpret_cast<float *>(base_ptr);   // reuses the ring buffers
             const int owned_max = (nchunk + p.S - 1) / p.S;
             float *recv = park + nchunk * kBM * 16;             // [S - 1 senders][owned_max][chunk]
-            for (int c16 = grp; c16 < nchunk; c16 += 4) {
-                uint32_t v[16];
+            for (int c16 = grp; c16 < nchunk; c16 += 8) {
+                const bool two = c16 + 4 < nchunk;
+                uint32_t v[2][16];
                 if (have) {
-                    tc_ld16(taddr + (uint32_t)(c16 * 16), v);
+                    tc_ld16(taddr + (uint32_t)(c16 * 16), v[0]);
+                    if (two)
+                        tc_ld16(taddr + (uint32_t)((c16 + 4) * 16), v[1]);
                     tc_wait_ld();
                 }
-                float4 *dst = reinterpret_cast<float4 *>(park + (c16 * kBM + row) * 16);
 #pragma unroll
-                for (int j = 0; j < 4; j++)
-                    dst[j] = have ? make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                                __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]))
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int h = 0; h < 2; h++) {
+                    if (h == 1 && !two)
+                        break;
+                    float4 *dst = reinterpret_cast<float4 *>(park + ((c16 + 4 * h) * kBM + row) * 16);
+#pragma unroll
+                    for (int j = 0; j < 4; j++)
+                        dst[j] = have ? make_float4(__uint_as_float(v[h][4 * j]), __uint_as_float(v[h][4 * j + 1]),
+                                                    __uint_as_float(v[h][4 * j + 2]), __uint_as_float(v[h][4 * j + 3]))
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
             }
             fence_proxy_async_smem();   // the bulk copies read the parked sums
             if (warp == 3 && lane == 0) {
