@@ -40,7 +40,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (dram__bytes_read.sum + dram__bytes_write.sum): the decode GEMV averaged over
 # the 197 launches of a decode step, the GEMM on the layer-0 q projection at
 # M = 1024.  Set to None when a kernel changes.
-NCU_TRAFFIC = {"gemv_tc_kernel": 5105538, "gemm_kernel": 6685952}
+NCU_TRAFFIC = {"gemv_tc_kernel": 5105538, "gemm_kernel": 6686976}
 
 
 def job_gbs(world, bytes_per_rank, ms_max):
