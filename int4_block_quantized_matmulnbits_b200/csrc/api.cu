@@ -58,6 +58,21 @@ int device_sm_count() {
     return counts[dev];
 }
 
+cudaError_t ensure_dynamic_smem(const void *kernel, int bytes, int *cache) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (dev < 0 || dev >= kMaxDevices)
+        return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (bytes <= cache[dev])
+        return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess)
+        cache[dev] = bytes;   // two threads racing here both set the same attribute
+    return e;
+}
+
 // Limits: sizes fit comfortably in 32-bit element indices of one row and in
 // 64-bit byte offsets overall.
 static const int64_t kMaxDim = (int64_t)1 << 30;

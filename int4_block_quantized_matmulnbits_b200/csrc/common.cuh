@@ -29,6 +29,13 @@ EncodeTiledFn tensor_map_encoder();
 // Streaming multiprocessors of the current device (cached per device).
 int device_sm_count();
 
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current
+// device when it is below that; `cache` (one entry per device, zero-initialized
+// by the caller as a static array of kMaxDevices) remembers what each device
+// was given.  Returns a cudaError_t.
+constexpr int kMaxDevices = 128;
+cudaError_t ensure_dynamic_smem(const void *kernel, int bytes, int *cache);
+
 // ---------------------------------------------------------------- device PTX
 
 __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t magic) {

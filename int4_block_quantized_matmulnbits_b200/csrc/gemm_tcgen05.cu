@@ -607,12 +607,11 @@ int launch_gemm(const void *X, const uint8_t *packed, const void *scales, int sc
             return fail(MNB_ERR_CUDA, "mnb_gemm: cuTensorMapEncodeTiled (W) failed (%d)", (int)cr);
     }
 
-    static int configured = 0;
-    if ((int)smem > configured) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static int configured[kMaxDevices] = {};
+    {
+        cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(gemm_kernel), (int)smem, configured);
         if (e != cudaSuccess)
             return fail(MNB_ERR_CUDA, "mnb_gemm: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-        configured = (int)smem;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(n_tiles * S), (unsigned)mt, 1);

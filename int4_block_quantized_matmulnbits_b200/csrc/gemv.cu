@@ -491,12 +491,11 @@ __global__ void __launch_bounds__(kThreads, (MODE == MODE_MMA) ? 2 : 1) gemv_ker
 template <int MODE, bool ACT_F16, int MP>
 int launch_one(const Params &p, int grid, size_t smem, unsigned flags, cudaStream_t s) {
     auto fn = gemv_kernel<MODE, ACT_F16, MP>;
-    static int configured = 0;   // largest dynamic shared memory opted into so far
-    if ((int)smem > 48 * 1024 && (int)smem > configured) {
-        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static int configured[kMaxDevices] = {};   // largest dynamic shared memory opted into, per device
+    if ((int)smem > 48 * 1024) {
+        cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(fn), (int)smem, configured);
         if (e != cudaSuccess)
             return fail(MNB_ERR_CUDA, "mnb_gemv: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-        configured = (int)smem;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid, 1, 1);

@@ -552,12 +552,11 @@ constexpr size_t kSmemLimit = 227 * 1024;
 template <bool BS64, bool ZP>
 int launch_chain_t(const ChainHeader &h, const ChainParams &p, unsigned flags, cudaStream_t s) {
     auto fn = gemv_chain_kernel<BS64, ZP>;
-    static int configured = 0;
-    if (h.smem > configured) {
-        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, h.smem);
+    static int configured[kMaxDevices] = {};
+    {
+        cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(fn), h.smem, configured);
         if (e != cudaSuccess)
             return fail(MNB_ERR_CUDA, "mnb_gemv_chain: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-        configured = h.smem;
     }
     // every CTA waits for all others: the grid must be resident at once
     int per_sm = 0;

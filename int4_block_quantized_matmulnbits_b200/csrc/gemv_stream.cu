@@ -407,12 +407,11 @@ template <bool BS64, bool ZP, bool SF32>
 int launch_stream(const CUtensorMap maps[3], const StreamParams &p, int grid, size_t smem, unsigned flags,
                   cudaStream_t s) {
     auto fn = gemv_stream_kernel<BS64, ZP, SF32>;
-    static size_t configured = 0;
-    if (smem > configured) {
-        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static int configured[kMaxDevices] = {};
+    {
+        cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(fn), (int)smem, configured);
         if (e != cudaSuccess)
             return fail(MNB_ERR_CUDA, "mnb_gemv: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-        configured = smem;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid, 1, 1);

@@ -609,12 +609,11 @@ __global__ void __launch_bounds__(kThreads, NT >= 4 ? 1 : 2) gemv_tc_kernel(cons
 template <int NT, class C>
 int launch_tc(const CUtensorMap &map, const TcParams &p, int grid, size_t smem, unsigned flags, cudaStream_t s) {
     auto fn = gemv_tc_kernel<NT, C>;
-    static int configured = 0;
-    if ((int)smem > configured) {
-        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static int configured[kMaxDevices] = {};
+    {
+        cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(fn), (int)smem, configured);
         if (e != cudaSuccess)
             return fail(MNB_ERR_CUDA, "mnb_gemv: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-        configured = (int)smem;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid, 1, 1);
