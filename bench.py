@@ -36,11 +36,29 @@ WORKLOAD = ("qwen3-1.7b-shaped decode step, M=1: 28 layers x (q 2048->2048, k/v 
             "int4 block 32 asymmetric, fp16 activations and scales, weights N(0,0.02) with 1% outliers x8")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM bytes (read + write) per launch from ncu captures of the current kernels
-# (dram__bytes_read.sum + dram__bytes_write.sum): the decode GEMV averaged over
-# the 197 launches of a decode step, the GEMM on the layer-0 q projection at
-# M = 1024.  Set to None when a kernel changes.
-NCU_TRAFFIC = {"gemv_tc_kernel": 5105538, "gemm_kernel": 6686976}
+DECODE_KERNEL = "gemv_tc_kernel"   # the kernel of the decode step's launches
+NOMINAL = {"hbm_gbs": 8000.0, "tc_tflops": 2250.0}   # B200 spec sheet: HBM3e, dense fp16/bf16
+
+
+def ncu_traffic(kernel):
+    """DRAM bytes (read + write) per launch of `kernel` from the committed ncu
+    summaries under profiles/, which record them in a line
+    ``traffic: kernel=<name> source=<file> sha1=<hex> bytes_per_launch=<n>``.
+    None unless the kernel's source file still has that hash (the counters
+    describe the kernel as it was captured)."""
+    import glob
+    import hashlib
+    import re
+
+    pat = re.compile(r"traffic: kernel=(\S+) source=(\S+) sha1=([0-9a-f]+) bytes_per_launch=(\d+)")
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        for m in pat.finditer(open(path).read()):
+            if m.group(1) != kernel:
+                continue
+            src = os.path.join(ROOT, m.group(2))
+            if os.path.exists(src) and hashlib.sha1(open(src, "rb").read()).hexdigest() == m.group(3):
+                return {"bytes_per_launch": int(m.group(4)), "profile": os.path.relpath(path, ROOT)}
+    return None
 
 
 def job_gbs(world, bytes_per_rank, ms_max):
@@ -177,12 +195,10 @@ def build_model(cfg_name, dev, lm_head=True):
 
 
 def fill(p, seed):
-    import torch
-
     import workloads
 
     for i, x in enumerate(p.X):
-        x.copy_(workloads.activations(seed, x.shape[0], x.shape[1], torch.float16, tag=i, device=x.device))
+        x.copy_(workloads.activations(seed, x.shape[0], x.shape[1], x.dtype, tag=i, device=x.device))
 
 
 def timed_replays(p, steps, warmup, ranks, tag="timed"):
@@ -339,6 +355,190 @@ def profile_part(args, dev, ranks):
         p.run()
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
+
+
+def oracle_rate(fn, units, seconds=1.5):
+    """Units per second of the oracle call fn() repeated for about `seconds`
+    (at least once), and the repetitions."""
+    t = 0.0
+    reps = 0
+    while t < seconds or reps == 0:
+        t0 = time.perf_counter()
+        fn()
+        t += time.perf_counter() - t0
+        reps += 1
+    return units * reps / t, reps
+
+
+def bench_single_gemv(dev, ranks, hbm, with_oracle):
+    """The single fp32 GEMV (M=1, K=1024, N=2048, block 32 with zero points,
+    fp32 activations and scales).  Latency: 200 dependent launches on ONE copy
+    of the weights (L2-resident, as a lone call in a decoder would be); GB/s:
+    200 dependent launches over 200 distinct copies (269 MB, larger than L2)."""
+    import numpy as np
+    import torch
+
+    import workloads
+    from int4_block_quantized_matmulnbits_b200.step import Pass, QLinear
+
+    cfg = workloads.CONFIGS["single_gemv"]
+    lin = cfg["linears"][0]
+    W = workloads.weight(cfg["seed"], lin.layer, lin.proj, lin.N, lin.K, device=dev)
+    one = QLinear.quantize(W, cfg["bs"], cfg["has_zp"], torch.float32, name="single")
+    copies = [QLinear.quantize(W, cfg["bs"], cfg["has_zp"], torch.float32, name=f"single{i}") for i in range(200)]
+    out = {"weight_bytes": one.nbytes, "launches": 200}
+    for key, lins in (("l2_resident", [one] * 200), ("rotated_copies", copies)):
+        p = Pass(lins, 1, "gemv", torch.float32, pdl=True)
+        fill(p, cfg["seed"])
+        p.capture()
+        t = timed_replays(p, 20, 3, ranks) / 20
+        us = t * 1000.0 / len(lins)
+        out[key] = {"us_per_call": round(us, 3), "weight_gbs": round(one.nbytes / (us * 1e-6) / 1e9, 1),
+                    "frac_hbm": round(one.nbytes / (us * 1e-6) / 1e9 / hbm, 4)}
+        del p
+    del copies, one
+    if with_oracle:
+        import oracle
+
+        Wn = W.cpu().numpy()
+        pk, sc, zp = oracle.quantize_rtn(Wn, cfg["bs"], True, np.float32)
+        X = workloads.activations(cfg["seed"], 1, lin.K, torch.float32).numpy()
+        nbytes = sum(oracle.packed_sizes(lin.N, lin.K, cfg["bs"], np.float32, True))
+        gbs, reps = oracle_rate(lambda: oracle.matmul(X, pk, sc, zp, lin.K, cfg["bs"]), nbytes)
+        out["cpu_oracle"] = {"weight_gbs": round(gbs / 1e9, 4), "us_per_call": round(nbytes / gbs * 1e6, 1),
+                             "cores": oracle.num_threads(), "sample": f"the whole GEMV, {reps} calls"}
+    del W
+    return out
+
+
+def oracle_layer_gbs(cfg_name, layer=0, M=1, seconds=1.5):
+    """The oracle over one layer's 7 projections of a workload at M tokens:
+    weight GB/s (its own RTN of the same seeded weights, prepared untimed)."""
+    import numpy as np
+    import torch
+
+    import oracle
+    import workloads
+
+    cfg = workloads.CONFIGS[cfg_name]
+    sdt = np.float16 if cfg["scale"] == "f16" else np.float32
+    items = []
+    for l in workloads.config_linears(cfg_name):
+        if l.layer != layer:
+            continue
+        W = workloads.weight(cfg["seed"], l.layer, l.proj, l.N, l.K, cfg.get("outliers", False)).numpy()
+        q = oracle.quantize_rtn(W, cfg["bs"], cfg["has_zp"], sdt)
+        X = workloads.activations(cfg["seed"], M, l.K, torch.float16, tag=l.proj).float().numpy()
+        items.append((X, q, l.K))
+    nbytes = sum(sum(oracle.packed_sizes(q[0].shape[0], K, cfg["bs"], sdt, cfg["has_zp"])) for _, q, K in items)
+
+    def run():
+        for X, (pk, sc, zp), K in items:
+            oracle.matmul(X, pk, sc, zp, K, cfg["bs"])
+
+    gbs, reps = oracle_rate(run, nbytes, seconds)
+    return {"weight_gbs": round(gbs / 1e9, 4), "cores": oracle.num_threads(),
+            "sample": f"the 7 projections of layer {layer} at M={M}, {reps} passes"}
+
+
+def bench_step(cfg_name, dev, ranks, hbm, Ms, steps=50):
+    """Decode steps (all projections + lm_head, one mnb_gemv each, CUDA graph,
+    PDL) of a workload at each M: us per step and weight GB/s."""
+    import torch
+
+    from int4_block_quantized_matmulnbits_b200.step import Pass
+
+    cfg, lins = build_model(cfg_name, dev)
+    out = {"launches_per_step": len(lins), "weight_bytes_per_step": sum(l.nbytes for l in lins)}
+    for M in Ms:
+        p = Pass(lins, M, "gemv", torch.float16, pdl=True)
+        fill(p, cfg["seed"] + M)
+        p.capture()
+        t = timed_replays(p, steps, 5, ranks) / steps
+        gbs = p.weight_bytes / (t * 1e-3) / 1e9
+        out[f"M{M}"] = {"us_per_step": round(t * 1000, 2), "weight_gbs": round(gbs, 1),
+                        "frac_hbm": round(gbs / hbm, 4)}
+        del p
+    return cfg, lins, out
+
+
+def bench_layout_variant(cfg_name, dev, ranks, hbm, tc_burst, with_oracle):
+    """Layout variants at 0.6B shapes: decode steps at M in gemv_M (with the
+    lm_head), prefill passes through mnb_gemm at M in gemm_M (no lm_head)."""
+    import torch
+
+    import workloads
+    from int4_block_quantized_matmulnbits_b200.step import Pass
+
+    cfg = workloads.CONFIGS[cfg_name]
+    cfg, lins, out = bench_step(cfg_name, dev, ranks, hbm, cfg["gemv_M"])
+    body = [l for l in lins if l.N != workloads.VOCAB]
+    for M in cfg["gemm_M"]:
+        p = Pass(body, M, "gemm", torch.float16, pdl=True)
+        fill(p, cfg["seed"] + M)
+        p.capture()
+        t = timed_replays(p, 10, 3, ranks) / 10
+        tf = p.flops / (t * 1e-3) / 1e12
+        out[f"gemm_M{M}"] = {"ms_per_pass": round(t, 4), "tflops": round(tf, 1),
+                             "frac_tc_burst": round(tf / tc_burst, 4),
+                             "weight_gbs": round(p.weight_bytes / (t * 1e-3) / 1e9, 1)}
+        del p
+    del lins
+    torch.cuda.empty_cache()
+    if with_oracle:
+        out["cpu_oracle"] = oracle_layer_gbs(cfg_name)
+    return out
+
+
+def bench_embed(dev, ranks, hbm, with_oracle):
+    """mnb_embed_gather over the int8 table [151936, 1024] (155.6 MB, larger
+    than L2) with fp32 row scales: 4096 uniformly random ids per call into
+    fp16 rows; 40 calls per replay, each with its own id set."""
+    import torch
+
+    import int4_block_quantized_matmulnbits_b200 as mnb
+    import workloads
+
+    e = workloads.EMBED
+    table, scales, ids = workloads.embed_inputs(e["seed"], e["V"], e["D"], e["T"])
+    table, scales = table.to(dev), scales.to(dev)
+    g = torch.Generator(device="cpu").manual_seed(e["seed"] * 7 + 1)
+    id_sets = [torch.randint(0, e["V"], (e["T"],), generator=g, dtype=torch.int32).to(dev) for _ in range(40)]
+    outs = [torch.empty((e["T"], e["D"]), dtype=torch.float16, device=dev) for _ in range(40)]
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+
+    def run():
+        for i, o in zip(id_sets, outs):
+            mnb.mnb_embed_gather(table, scales, e["V"], e["D"], i, e["T"], o, None, s)
+
+    with torch.cuda.stream(s):
+        run()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        run()
+
+    class G:
+        def replay(self):
+            graph.replay()
+
+    t = timed_replays(G(), 20, 3, ranks) / 20
+    us = t * 1000.0 / len(id_sets)
+    nbytes = e["T"] * (e["D"] + 4 + 4) + e["T"] * e["D"] * 2   # rows, scale, id read; fp16 rows written
+    gbs = nbytes / (us * 1e-6) / 1e9
+    out = {"ids_per_call": e["T"], "bytes_per_call": nbytes, "us_per_call": round(us, 3), "gbs": round(gbs, 1),
+           "frac_hbm": round(gbs / hbm, 4), "calls_per_replay": len(id_sets)}
+    if with_oracle:
+        import numpy as np
+
+        import oracle
+
+        tn, sn, idn = table.cpu().numpy(), scales.cpu().numpy(), ids.numpy()
+        ogbs, reps = oracle_rate(lambda: oracle.embed_gather(tn, sn, idn, np.float16), nbytes)
+        out["cpu_oracle"] = {"gbs": round(ogbs / 1e9, 4), "cores": 1,
+                             "sample": f"one call of 4096 ids, {reps} calls (the oracle's gather is one thread)"}
+    return out
 
 
 def run_gpu(args, world, rank, local):
@@ -520,7 +720,8 @@ def run_gpu(args, world, rank, local):
         assert pf.flops == sum(2 * M * l.N * l.K for l in body)
         tflops = pf.flops / (t * 1e-3) / 1e12
         prefill_fused[str(M)] = {"launches_per_pass": len(fbody), "ms_per_pass": round(t, 4),
-                                 "tflops": round(tflops, 1), "frac_tc_sustained": round(tflops / tc_sust, 4)}
+                                 "tflops": round(tflops, 1), "frac_tc_burst": round(tflops / tc_burst, 4),
+                                 "frac_tc_sustained": round(tflops / tc_sust, 4)}
         del pf
         torch.cuda.empty_cache()
     del fbody
@@ -552,6 +753,19 @@ def run_gpu(args, world, rank, local):
                            "weight_gbs": round(ep.weight_bytes / (t * 1e-3) / 1e9, 1)}
         del ep
     del elins
+    del lins, body
+    torch.cuda.empty_cache()
+    with_oracle = rank == 0 and world == 1
+    single = bench_single_gemv(dev, ranks, hbm, with_oracle)
+    torch.cuda.empty_cache()
+    _, l06, step06 = bench_step("qwen3_0p6b_decode", dev, ranks, hbm, [1], steps=200)
+    del l06
+    torch.cuda.empty_cache()
+    if with_oracle:
+        step06["cpu_oracle"] = oracle_layer_gbs("qwen3_0p6b_decode")
+    variants = {v: bench_layout_variant(v, dev, ranks, hbm, tc_burst, with_oracle)
+                for v in ("qwen3_0p6b_bs64", "qwen3_0p6b_nozp")}
+    embed = bench_embed(dev, ranks, hbm, with_oracle)
     torch.cuda.empty_cache()
     assert mnb.mnb_device_status() == 0, "a GEMM wait timed out"
 
@@ -563,6 +777,8 @@ def run_gpu(args, world, rank, local):
                "sample": f"oracle.matmul over the 7 projections of layer 0 of the decode step at M=1, "
                          f"{reps} passes, {dt:.1f} s wall on {sample.cores} threads"}
 
+    dec_traffic = ncu_traffic(DECODE_KERNEL)
+    gemm_traffic = ncu_traffic("gemm_kernel")
     if rank == 0:
         out = {
             "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
@@ -573,11 +789,13 @@ def run_gpu(args, world, rank, local):
                        "weight_bytes_per_step": wbytes, "graph": True, "pdl": True,
                        "l2": "inputs larger than L2 (weights of one step > 126 MB)",
                        "parallelism": f"replicas x{world}"},
-            "roofline": {"bound": "hbm", "kernel": "gemv_tc_kernel", "achieved": round(achieved, 1), "peak": hbm,
+            "roofline": {"bound": "hbm", "kernel": DECODE_KERNEL, "achieved": round(achieved, 1), "peak": hbm,
                          "unit": "GB/s", "frac": round(achieved / hbm, 4),
-                         "traffic": NCU_TRAFFIC["gemv_tc_kernel"],
+                         "traffic": (dec_traffic or {}).get("bytes_per_launch"),
+                         "traffic_source": (dec_traffic or {}).get("profile"),
                          "peak_source": f"{peak_src} hbm_gbs", "bytes_per_launch": round(per_launch_bytes),
-                         "us_per_launch": round(per_launch_us, 3)},
+                         "us_per_launch": round(per_launch_us, 3),
+                         "frac_of_nominal_8000_gbs": round(achieved / NOMINAL["hbm_gbs"], 4)},
             "lm_head_alone": {"bytes": lm.nbytes, "us": round(lm_ms * 1000, 2), "gbs": round(lm_gbs, 1),
                               "frac_hbm": round(lm_gbs / hbm, 4),
                               "us_with_greedy_argmax": round(lmg_ms * 1000, 2)},
@@ -590,10 +808,18 @@ def run_gpu(args, world, rank, local):
             "cached_prefill": cached,
             "audio_encoder_prefill": encoder,
             "roofline_prefill": {"bound": "tensor", "kernel": "gemm_kernel", "M": 1024,
-                                 "achieved": prefill["1024"]["tflops"], "peak": tc_sust, "unit": "TFLOP/s",
-                                 "frac": prefill["1024"]["frac_tc_sustained"],
-                                 "traffic": NCU_TRAFFIC["gemm_kernel"], "traffic_of": "layer-0 q projection",
-                                 "peak_source": f"{peak_src} bf16_tflops_sustained (fp16 = bf16 nominal rate)"},
+                                 "achieved": prefill["1024"]["tflops"], "peak": tc_burst, "unit": "TFLOP/s",
+                                 "frac": prefill["1024"]["frac_tc_burst"],
+                                 "traffic": (gemm_traffic or {}).get("bytes_per_launch"),
+                                 "traffic_of": "layer-0 q projection",
+                                 "traffic_source": (gemm_traffic or {}).get("profile"),
+                                 "peak_source": f"{peak_src} bf16_tflops, the burst figure: the timed region is a "
+                                                f"~0.1 s run of 196 GEMMs (fp16 = bf16 nominal rate)",
+                                 "frac_of_nominal_2250_tflops": round(prefill["1024"]["tflops"] / NOMINAL["tc_tflops"], 4)},
+            "single_gemv_fp32": single,
+            "decode_step_qwen3_0p6b": step06,
+            "layout_variants": variants,
+            "embed_gather": embed,
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_val, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},

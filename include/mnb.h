@@ -66,7 +66,10 @@ enum {
     MNB_ERR_ALIGN = -3,       /* a pointer is not aligned as documented         */
     MNB_ERR_UNSUPPORTED = -4, /* a valid request the library does not serve     */
     MNB_ERR_CUDA = -5,        /* a CUDA runtime call or launch failed           */
-    MNB_ERR_TIMEOUT = -6      /* a device-side bounded wait gave up (see below) */
+    MNB_ERR_TIMEOUT = -6      /* a device-side bounded wait gave up: returned by
+                                 mnb_device_status, which reads the word the
+                                 kernels set (kernel launches return before the
+                                 wait happens) */
 };
 
 /* Flags for mnb_gemv / mnb_gemm. */
@@ -125,6 +128,9 @@ MNB_API int mnb_dequantize(const uint8_t *packed, const void *scales, mnb_dtype 
  * Y = X . dequant(W)^T.
  *   act_t  = dtype of X and Y (fp32 or fp16); scale_t = dtype of scales.
  *   Accumulation is fp32.  Bandwidth-bound: streams the packed weights once.
+ *   With fp16 activations an fp32 scale takes part as fp16_rn(scale) (the
+ *   fp16 arithmetic of the q4f16 graphs); with fp32 activations every step
+ *   is fp32.
  * Errors: MNB_ERR_INVALID_ARG, MNB_ERR_SHAPE, MNB_ERR_ALIGN,
  *         MNB_ERR_UNSUPPORTED (M above the limit), MNB_ERR_CUDA. */
 MNB_API int mnb_gemv(const void *X, mnb_dtype act_t, const uint8_t *packed, const void *scales,
@@ -176,8 +182,10 @@ MNB_API int mnb_gemv_argmax(const void *X, const uint8_t *packed, const void *sc
  * loads the library, held until the process exits.  With 148 SMs that covers
  * every M in [1, 16]; a request needing more returns MNB_ERR_SHAPE with a
  * message.  Nothing is allocated: the first call on each device looks up the
- * array's device address (make that first call before any stream capture),
- * and each call clears the array's counter on `stream` before its kernel.
+ * array's device address (make that first call before any stream capture)
+ * and keeps it for the life of the process, so a cudaDeviceReset of that
+ * device makes later calls unusable (the kept address is stale); each call
+ * clears the array's counter on `stream` before its kernel.
  * All calls on one GPU share the one array, which keeps the last call's
  * contents: calls that may run at the same time on the GPU (other streams,
  * other host threads) race on it and must be serialized by the caller.
@@ -189,15 +197,16 @@ MNB_API int mnb_gemv_argmax_noalloc(const void *X, const uint8_t *packed, const 
 
 /* Prefill-shaped MatMulNBits on the tensor cores, any M >= 1 (tuned for
  * M >= 64: the full-length prefill of "Mega-ASR -- INT4 ONNX", "What's in this
- * repo": decoder_prefill).  Y = X . dequant(W)^T with fp16 X and Y; each
- * weight is dequantized to fp16_rn((q - zp) * scale) and the products are
- * accumulated in fp32.
- *   act_t must be MNB_F16; N must be a multiple of 128 and K of 64.
+ * repo": decoder_prefill).  Y = X . dequant(W)^T with fp16 X, scales and Y (the
+ * q4f16 variant of "Qwen3-ASR-0.6B -- ONNX for the browser", "Pick a
+ * variant"); each weight is dequantized to fp16_rn((q - zp) * scale), the
+ * value mnb_dequantize writes, and the products are accumulated in fp32.
+ *   act_t and scale_t must be MNB_F16; N must be a multiple of 128 and K of 64.
  * A device-side wait that exceeds its iteration limit makes the kernel stop,
  * sets a bit in the library's device status word (see mnb_device_status) and
  * leaves Y incomplete; the call itself returned MNB_OK by then.
  * Errors: MNB_ERR_INVALID_ARG, MNB_ERR_SHAPE, MNB_ERR_ALIGN,
- *         MNB_ERR_UNSUPPORTED (fp32 activations), MNB_ERR_CUDA. */
+ *         MNB_ERR_UNSUPPORTED (fp32 activations or fp32 scales), MNB_ERR_CUDA. */
 MNB_API int mnb_gemm(const void *X, mnb_dtype act_t, const uint8_t *packed, const void *scales,
              mnb_dtype scale_t, const uint8_t *zp, void *Y, int64_t M, int64_t N, int64_t K,
              int bs, unsigned flags, void *stream);
@@ -210,9 +219,9 @@ MNB_API int mnb_gemm(const void *X, mnb_dtype act_t, const uint8_t *packed, cons
  * this one call:
  *   M <= 24 with fp16 X (M <= 16 with fp32 X): one mnb_gemv (measured faster
  *     than the tensor-core GEMM up to 24 tokens);
- *   M >= 25 with fp16 X, N % 128 == 0, K % 64 == 0: mnb_gemm;
- *   otherwise (fp32 X, or shapes the GEMM does not take): mnb_gemv launches
- *     of up to 24 (fp16) or 16 (fp32) tokens.
+ *   M >= 25 with fp16 X and scales, N % 128 == 0, K % 64 == 0: mnb_gemm;
+ *   otherwise (fp32 X or scales, or shapes the GEMM does not take):
+ *     mnb_gemv launches of up to 24 (fp16 X) or 16 (fp32 X) tokens.
  * Requires X, packed and Y 16-byte aligned.
  * Errors: MNB_ERR_INVALID_ARG, MNB_ERR_SHAPE, MNB_ERR_ALIGN, MNB_ERR_CUDA. */
 MNB_API int mnb_matmul(const void *X, mnb_dtype act_t, const uint8_t *packed, const void *scales, mnb_dtype scale_t,
@@ -293,9 +302,12 @@ MNB_API int mnb_gemv_chain(const void *plan, const void *plan_device, void *work
                            unsigned flags, void *stream);
 
 /* Reads (and, if clear != 0, zeroes) the library's device status word on the
- * current device: bit 0 = a GEMM or GEMV mbarrier wait timed out; bits 1-3 =
- * mnb_gemv_chain (see there).  Synchronizes the
- * device.  Errors: MNB_ERR_INVALID_ARG (NULL), MNB_ERR_CUDA. */
+ * current device into *status_out: bit 0 = a GEMM or GEMV mbarrier wait timed
+ * out; bits 1-3 = mnb_gemv_chain (see there).  Synchronizes the device.
+ * Returns MNB_ERR_TIMEOUT (with *status_out written) when any of bits 0-2 is
+ * set, i.e. a bounded wait inside a kernel gave up since the word was last
+ * cleared; MNB_OK otherwise.
+ * Errors: MNB_ERR_INVALID_ARG (NULL), MNB_ERR_CUDA, MNB_ERR_TIMEOUT. */
 MNB_API int mnb_device_status(unsigned *status_out, int clear);
 
 #ifdef __cplusplus

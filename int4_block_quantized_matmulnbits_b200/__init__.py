@@ -244,7 +244,10 @@ def mnb_embed_gather(table, row_scales, V, D, ids, T, out, status=None, stream=N
 
 def mnb_device_status(clear=False) -> int:
     """The library's device status word (bit 0: a GEMM or GEMV wait timed out;
-    bits 1-2: mnb_gemv_chain); synchronizes."""
+    bits 1-3: mnb_gemv_chain); synchronizes.  A timeout (MNB_ERR_TIMEOUT from
+    the C call) is reported through the returned word, not raised."""
     v = ctypes.c_uint()
-    _check("mnb_device_status", _lib.mnb_device_status(ctypes.byref(v), int(bool(clear))))
+    rc = _lib.mnb_device_status(ctypes.byref(v), int(bool(clear)))
+    if rc != -6:
+        _check("mnb_device_status", rc)
     return v.value

@@ -287,6 +287,8 @@ int mnb_gemm(const void *X, mnb_dtype act_t, const uint8_t *packed, const void *
         return rc;
     if (act_t != MNB_F16)
         return fail(MNB_ERR_UNSUPPORTED, "%s: the tensor-core path takes fp16 activations", fn);
+    if (scale_t != MNB_F16)
+        return fail(MNB_ERR_UNSUPPORTED, "%s: the tensor-core path takes fp16 scales (the q4f16 variant)", fn);
     if (N % 128 != 0 || K % 64 != 0)
         return fail(MNB_ERR_SHAPE, "%s: N=%lld must be a multiple of 128 and K=%lld of 64", fn,
                     (long long)N, (long long)K);
@@ -315,7 +317,7 @@ int mnb_matmul(const void *X, mnb_dtype act_t, const uint8_t *packed, const void
         return fail(MNB_ERR_INVALID_ARG, "%s: unknown flags 0x%x", fn, flags);
     if (M == 0 || N == 0)
         return MNB_OK;
-    const bool gemm_ok = act_t == MNB_F16 && N % 128 == 0 && K % 64 == 0;
+    const bool gemm_ok = act_t == MNB_F16 && scale_t == MNB_F16 && N % 128 == 0 && K % 64 == 0;
     if (gemm_ok && M > kGemvMaxM)
         return launch_gemm(X, packed, scales, scale_t == MNB_F16, zp, Y, (int)M, (int)N, (int)K, bs, flags,
                            (cudaStream_t)stream);
@@ -401,7 +403,13 @@ int mnb_device_status(unsigned *status_out, int clear) {
     clear_error();
     if (!status_out)
         return fail(MNB_ERR_INVALID_ARG, "mnb_device_status: NULL output");
-    return read_device_status(status_out, clear);
+    *status_out = 0;
+    const int rc = read_device_status(status_out, clear);
+    if (rc)
+        return rc;
+    if (*status_out & 7u)   // bits 0-2: a bounded wait inside a kernel gave up
+        return fail(MNB_ERR_TIMEOUT, "mnb_device_status: a device-side wait timed out (status 0x%x)", *status_out);
+    return MNB_OK;
 }
 
 }  // extern "C"

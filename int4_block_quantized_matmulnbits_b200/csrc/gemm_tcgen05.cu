@@ -40,6 +40,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "mnb_tune.h"
 
 namespace mnb {
 
@@ -65,7 +66,7 @@ struct GemmParams {
     const uint8_t *zp;
     __half *Y;
     int M, N, K;
-    int bs_shift, nb, zpb, scale_f16;
+    int bs_shift, nb, zpb;
     int BN;        // tokens per CTA (multiple of 16, <= 256)
     int xstages;   // depth of the X ring
     int tmem_cols; // power of two >= BN
@@ -172,11 +173,7 @@ __device__ __forceinline__ SZ load_sz(const GemmParams &p, int n, int k) {
     if (k >= p.K)
         return r;
     const int b = k >> (5 + p.bs_shift);
-    if (p.scale_f16)
-        r.s = __ldg(reinterpret_cast<const unsigned short *>(p.scales) + (int64_t)n * p.nb + b);
-    else
-        r.s = __half_as_ushort(
-            __float2half_rn(__ldg(reinterpret_cast<const float *>(p.scales) + (int64_t)n * p.nb + b)));
+    r.s = __ldg(reinterpret_cast<const unsigned short *>(p.scales) + (int64_t)n * p.nb + b);   // fp16 scales only
     if (p.zp) {
         const uint32_t zb = __ldg(p.zp + (int64_t)n * p.zpb + (b >> 1));
         r.z = (b & 1) ? (zb >> 4) : (zb & 15u);
@@ -562,7 +559,7 @@ int launch_gemm(const void *X, const uint8_t *packed, const void *scales, int sc
     p.bs_shift = (bs == 64) ? 1 : 0;
     p.nb = K / bs;
     p.zpb = (p.nb + 1) / 2;
-    p.scale_f16 = scale_f16;
+    (void)scale_f16;   // the entry point admits fp16 scales only
     p.BN = BN;
     p.tmem_cols = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
     p.S = S;
@@ -653,8 +650,6 @@ int read_device_status(unsigned *out, int clear) {
     cudaError_t e = cudaMemcpyFromSymbol(out, g_mnb_status, sizeof(unsigned));
     if (e == cudaSuccess) {
         int rc = read_gemv_status(out, clear);
-        if (!rc)
-            rc = read_stream_status(out, clear);
         if (!rc)
             rc = read_chain_status(out, clear);
         if (rc)

@@ -1,7 +1,8 @@
-// gemv.cu -- decode-shaped MatMulNBits, Y[M][N] = X[M][K] . dequant(W)^T with
-// 1 <= M <= 16 (the per-token decoder_step of "Qwen3-ASR-0.6B -- ONNX for the
-// browser", "Graph contracts", and of "Mega-ASR -- INT4 ONNX", "What's in this
-// repo": decoder_step_int4).
+// gemv.cu -- decode-shaped MatMulNBits with fp32 activations (the q4 variant of
+// "Qwen3-ASR-0.6B -- ONNX for the browser", "Pick a variant"):
+// Y[M][N] = X[M][K] . dequant(W)^T with 1 <= M <= 16 (the per-token
+// decoder_step of the same page, "Graph contracts").  fp16 activations go to
+// gemv_tc.cu.
 //
 // This is HBM-bound: every packed byte is read exactly once, so the kernel is
 // built around moving weight bytes.
@@ -23,17 +24,11 @@
 //     memory): no global scratch, no second kernel, no atomics.
 //   * X for the CTA's K range is staged permuted, so one 16-byte load yields
 //     the activation pairs that match the dequantized weight pairs.
-// Unpack + dequant happen in registers: (mask | 0x6400) turns a nibble q into
-// the fp16 1024+q exactly, and one half2 subtract (or fma for the high nibble,
-// 1024+16q) leaves the exact q - zp.  Two inner products:
-//   MMA (fp16 activations): the weight half2s are scaled to
-//     fp16_rn((q - zp) * scale) and fed to mma.sync m16n8k16 with fp32
-//     accumulation; the 16 rows are the MMA's M, the tokens its N (8 or 16).
-//     This keeps the multiply-adds off the CUDA cores, whose issue slots the
-//     unpack already fills.
-//   CC (fp32 activations, and an fp16 variant): CUDA-core FMAs, fp32 partial
-//     per chunk, times the scale, summed in fp32, reduced across the 4 lanes of
-//     a row with warp shuffles.
+// Unpack + dequant happen in registers: (0x4B000000 | q) is the fp32 2^23 + q
+// exactly, so subtracting 2^23 + zp leaves the exact q - zp.  The inner product
+// takes true fp32 FMAs (the fp32 tolerance leaves no room for fp16 products):
+// an fp32 partial per 32-k chunk, times the scale, summed in fp32, reduced
+// across the 4 lanes of a row with warp shuffles.
 #include "common.cuh"
 #include "internal.h"
 
@@ -48,7 +43,6 @@ constexpr int kPF = 4;            // super-chunks in flight per warp
 constexpr int kSuper = 128;       // k per super-chunk
 constexpr int kMaxCluster = 8;
 
-enum { MODE_MMA = 0, MODE_CC = 1 };
 
 struct Params {
     const void *X;
@@ -71,8 +65,7 @@ struct Params {
 
 struct Slot {
     uint4 p0, p1;      // 32 nibbles of row g and of row g+8
-    uint32_t s0, s1;   // scales, already in the inner product's type: fp16 bits
-                       // (tensor-core path) or fp32 bits (CUDA-core path)
+    float s0, s1;      // scales as fp32
     uint32_t z0, z1;   // zero point nibble (8 when absent)
 };
 
@@ -101,14 +94,12 @@ __device__ __forceinline__ void cursor_tile(const Params &p, Cursor &q, int tile
 }
 
 // Loads the cursor's super-chunk (nothing when !live or past K), then advances.
-// SCALE_F16: deliver the scales as fp16 bits (an fp32 scale is rounded once,
-// here); else as fp32 bits.
-template <bool SCALE_F16>
+// Scales are delivered as fp32 (an fp16 scale converts exactly).
 __device__ __forceinline__ Slot load_advance(const Params &p, Cursor &q, bool live, int zsh,
                                              int tile_step_base, int g, int kfirst) {
     Slot s;
     s.p0 = s.p1 = make_uint4(0, 0, 0, 0);
-    s.s0 = s.s1 = 0;
+    s.s0 = s.s1 = 0.f;
     s.z0 = s.z1 = 8;
     if (live && q.k < p.K) {
 #pragma unroll
@@ -118,14 +109,9 @@ __device__ __forceinline__ Slot load_advance(const Params &p, Cursor &q, bool li
             const int64_t rows8 = r ? 8 : 0;
             const uint4 v = ldg_stream_v4(q.p0 + rows8 * (p.K / 2));
             const uint8_t *sp = q.s0 + rows8 * p.nb * (p.scale_f16 ? 2 : 4);
-            uint32_t sb;
-            if (p.scale_f16) {
-                const unsigned short h = __ldg(reinterpret_cast<const unsigned short *>(sp));
-                sb = SCALE_F16 ? (uint32_t)h : __float_as_uint(__half2float(__ushort_as_half(h)));
-            } else {
-                const float f = __ldg(reinterpret_cast<const float *>(sp));
-                sb = SCALE_F16 ? (uint32_t)__half_as_ushort(__float2half_rn(f)) : __float_as_uint(f);
-            }
+            const float sb = p.scale_f16
+                                 ? __half2float(__ushort_as_half(__ldg(reinterpret_cast<const unsigned short *>(sp))))
+                                 : __ldg(reinterpret_cast<const float *>(sp));
             uint32_t z = 8;
             if (p.zp)
                 z = ((uint32_t)__ldg(q.z0 + rows8 * p.zpb) >> zsh) & 15u;
@@ -148,39 +134,6 @@ __device__ __forceinline__ Slot load_advance(const Params &p, Cursor &q, bool li
     return s;
 }
 
-// 8 nibbles -> 4 half2 of exact (q - zp): (e0,e4), (e1,e5), (e2,e6), (e3,e7).
-__device__ __forceinline__ void dq_word(uint32_t w, uint32_t Z, uint32_t Zhi, uint32_t out[4]) {
-    const half2 sixteenth = __floats2half2_rn(0.0625f, 0.0625f);
-    const uint32_t lo0 = lop3_and_or(w, 0x000F000Fu, 0x64006400u);
-    const uint32_t hi0 = lop3_and_or(w, 0x00F000F0u, 0x64006400u);
-    const uint32_t w8 = w >> 8;
-    const uint32_t lo1 = lop3_and_or(w8, 0x000F000Fu, 0x64006400u);
-    const uint32_t hi1 = lop3_and_or(w8, 0x00F000F0u, 0x64006400u);
-    out[0] = h2_as_u32(__hsub2(u32_as_h2(lo0), u32_as_h2(Z)));
-    out[1] = h2_as_u32(__hfma2(u32_as_h2(hi0), sixteenth, u32_as_h2(Zhi)));
-    out[2] = h2_as_u32(__hsub2(u32_as_h2(lo1), u32_as_h2(Z)));
-    out[3] = h2_as_u32(__hfma2(u32_as_h2(hi1), sixteenth, u32_as_h2(Zhi)));
-}
-
-// 16 half2 of exact (q - zp) for one 16-byte chunk; element order per word as dq_word.
-__device__ __forceinline__ void dq_chunk(const uint4 &p, uint32_t z, uint32_t out[16]) {
-    const uint32_t Z = 0x64006400u | (z * 0x00010001u);          // 1024 + zp
-    const uint32_t Zhi = 0xD400D400u + (z * 0x00100010u);        // -(64 + zp)
-    dq_word(p.x, Z, Zhi, out + 0);
-    dq_word(p.y, Z, Zhi, out + 4);
-    dq_word(p.z, Z, Zhi, out + 8);
-    dq_word(p.w, Z, Zhi, out + 12);
-}
-
-__device__ __forceinline__ half2 scale_h2(uint32_t h16) { return u32_as_h2(h16 | (h16 << 16)); }
-
-__device__ __forceinline__ void mma16816(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
 __device__ __forceinline__ uint4 lds128(const unsigned char *p) { return *reinterpret_cast<const uint4 *>(p); }
 
 
@@ -193,11 +146,10 @@ __device__ __forceinline__ float ld_dsmem_f32(const float *local, uint32_t rank)
     return v;
 }
 
-// MP: tokens held per thread (MMA: 8 or 16, CC: 1, 2, 4, 8 or 16).
-template <int MODE, bool ACT_F16, int MP>
-__global__ void __launch_bounds__(kThreads, (MODE == MODE_MMA) ? 2 : 1) gemv_kernel(const Params p) {
+// MP: tokens held per thread (1, 2, 4, 8 or 16).
+template <int MP>
+__global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const Params p) {
     extern __shared__ __align__(16) unsigned char smem[];
-    constexpr int NT = (MODE == MODE_MMA) ? MP / 8 : 1;
     const int tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, c = lane & 3;
@@ -226,31 +178,13 @@ __global__ void __launch_bounds__(kThreads, (MODE == MODE_MMA) ? 2 : 1) gemv_ker
     Slot ring[kPF];
 #pragma unroll
     for (int i = 0; i < kPF; i++)
-        ring[i] = load_advance<MODE == MODE_MMA>(p, cur_ld, i < total, zsh, tile_base, g, kfirst);
+        ring[i] = load_advance(p, cur_ld, i < total, zsh, tile_base, g, kfirst);
     pdl_launch_dependents();
     pdl_wait();
 
     // ---- stage X[0:M, kcta0 : kcta0 + kcta), zero past K
     const int nsc_cta = W * p.nsc_w;
-    if (ACT_F16) {
-        const __half *X = reinterpret_cast<const __half *>(p.X);
-        const int per_tok = nsc_cta * 16;                      // 16-byte units of 8 halves
-        for (int u = tid; u < p.M * per_tok; u += kThreads) {
-            const int m = u / per_tok;
-            const int r = u - m * per_tok;
-            const int sc = r >> 4, cc = (r >> 2) & 3, w = r & 3;
-            const int k = kcta0 + sc * kSuper + cc * 32 + w * 8;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (k < p.K)
-                v = ldg_v4(X + (int64_t)m * p.K + k);
-            uint4 o;   // (x0,x4) (x1,x5) (x2,x6) (x3,x7)
-            o.x = __byte_perm(v.x, v.z, 0x5410);
-            o.y = __byte_perm(v.x, v.z, 0x7632);
-            o.z = __byte_perm(v.y, v.w, 0x5410);
-            o.w = __byte_perm(v.y, v.w, 0x7632);
-            *reinterpret_cast<uint4 *>(xs + m * p.xs_stride + sc * 256 + w * 64 + cc * 16) = o;
-        }
-    } else {
+    {
         const float *X = reinterpret_cast<const float *>(p.X);
         const int per_tok = nsc_cta * 32;                      // 16-byte units of 4 floats
         for (int u = tid; u < p.M * per_tok; u += kThreads) {
@@ -266,18 +200,12 @@ __global__ void __launch_bounds__(kThreads, (MODE == MODE_MMA) ? 2 : 1) gemv_ker
     }
     __syncthreads();
 
-    float accm[NT][4];                        // MMA accumulators
-    float accc[2][MP];                        // CC accumulators: rows g, g+8 x tokens
-#pragma unroll
-    for (int t = 0; t < NT; t++)
-#pragma unroll
-        for (int i = 0; i < 4; i++) accm[t][i] = 0.f;
+    float acc[2][MP];   // rows g, g+8 x tokens
 #pragma unroll
     for (int r = 0; r < 2; r++)
 #pragma unroll
-        for (int m = 0; m < MP; m++) accc[r][m] = 0.f;
+        for (int m = 0; m < MP; m++) acc[r][m] = 0.f;
 
-    const unsigned char *xs_base = xs;
     int cr = 0, csc = 0;   // position being consumed
     for (int base = 0; base < total; base += kPF) {
 #pragma unroll
@@ -285,109 +213,40 @@ __global__ void __launch_bounds__(kThreads, (MODE == MODE_MMA) ? 2 : 1) gemv_ker
             if (base + i >= total)
                 break;
             const Slot cur = ring[i];
-            ring[i] = load_advance<MODE == MODE_MMA>(p, cur_ld, base + i + kPF < total, zsh, tile_base, g,
-                                                       kfirst);
+            ring[i] = load_advance(p, cur_ld, base + i + kPF < total, zsh, tile_base, g, kfirst);
             const int sc = wk * p.nsc_w + csc;   // super-chunk inside the CTA's X range
 
-            if (MODE == MODE_MMA) {
-                uint32_t wa[16], wb[16];
-                dq_chunk(cur.p0, cur.z0, wa);
-                dq_chunk(cur.p1, cur.z1, wb);
-                const half2 s0 = scale_h2(cur.s0);
-                const half2 s1 = scale_h2(cur.s1);
+            // exact (q - zp) as fp32 via 2^23 + q
+            const float zb0 = 8388608.f + (float)cur.z0, zb1 = 8388608.f + (float)cur.z1;
+            const uint32_t w0[4] = {cur.p0.x, cur.p0.y, cur.p0.z, cur.p0.w};
+            const uint32_t w1[4] = {cur.p1.x, cur.p1.y, cur.p1.z, cur.p1.w};
+            float fa[32], fb[32];
 #pragma unroll
-                for (int j = 0; j < 16; j++) {
-                    wa[j] = h2_as_u32(__hmul2(u32_as_h2(wa[j]), s0));
-                    wb[j] = h2_as_u32(__hmul2(u32_as_h2(wb[j]), s1));
-                }
+            for (int e = 0; e < 32; e++) {
+                const uint32_t na = (w0[e >> 3] >> (4 * (e & 7))) & 15u;
+                const uint32_t nb = (w1[e >> 3] >> (4 * (e & 7))) & 15u;
+                fa[e] = __uint_as_float(0x4B000000u | na) - zb0;
+                fb[e] = __uint_as_float(0x4B000000u | nb) - zb1;
+            }
 #pragma unroll
-                for (int t = 0; t < NT; t++) {
-                    uint32_t xb[16];
-                    const int tok = g + 8 * t;
-                    if (tok < p.M) {
-                        const unsigned char *xa = xs_base + tok * p.xs_stride + sc * 256 + c * 16;
+            for (int m = 0; m < MP; m++) {
+                if (m >= p.M)
+                    break;
+                const unsigned char *xa = xs + m * p.xs_stride + sc * 512 + c * 16;
+                float pa = 0.f, pb = 0.f;
 #pragma unroll
-                        for (int w = 0; w < 4; w++) {
-                            const uint4 v = lds128(xa + w * 64);
-                            xb[4 * w + 0] = v.x; xb[4 * w + 1] = v.y;
-                            xb[4 * w + 2] = v.z; xb[4 * w + 3] = v.w;
-                        }
-                    } else {
+                for (int j = 0; j < 8; j++) {
+                    const uint4 v = lds128(xa + j * 64);
+                    const float xv[4] = {__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z),
+                                         __uint_as_float(v.w)};
 #pragma unroll
-                        for (int j = 0; j < 16; j++) xb[j] = 0u;
-                    }
-#pragma unroll
-                    for (int q = 0; q < 8; q++) {
-                        const uint32_t a[4] = {wa[2 * q], wb[2 * q], wa[2 * q + 1], wb[2 * q + 1]};
-                        mma16816(accm[t], a, xb[2 * q], xb[2 * q + 1]);
+                    for (int e = 0; e < 4; e++) {
+                        pa = fmaf(xv[e], fa[4 * j + e], pa);
+                        pb = fmaf(xv[e], fb[4 * j + e], pb);
                     }
                 }
-            } else if (ACT_F16) {
-                uint32_t wa[16], wb[16];
-                dq_chunk(cur.p0, cur.z0, wa);
-                dq_chunk(cur.p1, cur.z1, wb);
-                const float s0 = __uint_as_float(cur.s0);
-                const float s1 = __uint_as_float(cur.s1);
-#pragma unroll
-                for (int m = 0; m < MP; m++) {
-                    if (m >= p.M)
-                        break;
-                    const unsigned char *xa = xs_base + m * p.xs_stride + sc * 256 + c * 16;
-                    uint32_t xb[16];
-#pragma unroll
-                    for (int w = 0; w < 4; w++) {
-                        const uint4 v = lds128(xa + w * 64);
-                        xb[4 * w + 0] = v.x; xb[4 * w + 1] = v.y;
-                        xb[4 * w + 2] = v.z; xb[4 * w + 3] = v.w;
-                    }
-                    half2 a0 = __float2half2_rn(0.f), a1 = a0, b0 = a0, b1 = a0;
-#pragma unroll
-                    for (int j = 0; j < 16; j += 2) {
-                        a0 = __hfma2(u32_as_h2(wa[j]), u32_as_h2(xb[j]), a0);
-                        a1 = __hfma2(u32_as_h2(wa[j + 1]), u32_as_h2(xb[j + 1]), a1);
-                        b0 = __hfma2(u32_as_h2(wb[j]), u32_as_h2(xb[j]), b0);
-                        b1 = __hfma2(u32_as_h2(wb[j + 1]), u32_as_h2(xb[j + 1]), b1);
-                    }
-                    const float2 fa0 = __half22float2(a0), fa1 = __half22float2(a1);
-                    const float2 fb0 = __half22float2(b0), fb1 = __half22float2(b1);
-                    accc[0][m] = fmaf(s0, (fa0.x + fa0.y) + (fa1.x + fa1.y), accc[0][m]);
-                    accc[1][m] = fmaf(s1, (fb0.x + fb0.y) + (fb1.x + fb1.y), accc[1][m]);
-                }
-            } else {
-                // fp32 activations: exact (q - zp) as fp32 via 2^23 + q
-                const float s0 = __uint_as_float(cur.s0);
-                const float s1 = __uint_as_float(cur.s1);
-                const float zb0 = 8388608.f + (float)cur.z0, zb1 = 8388608.f + (float)cur.z1;
-                const uint32_t w0[4] = {cur.p0.x, cur.p0.y, cur.p0.z, cur.p0.w};
-                const uint32_t w1[4] = {cur.p1.x, cur.p1.y, cur.p1.z, cur.p1.w};
-                float fa[32], fb[32];
-#pragma unroll
-                for (int e = 0; e < 32; e++) {
-                    const uint32_t na = (w0[e >> 3] >> (4 * (e & 7))) & 15u;
-                    const uint32_t nb = (w1[e >> 3] >> (4 * (e & 7))) & 15u;
-                    fa[e] = __uint_as_float(0x4B000000u | na) - zb0;
-                    fb[e] = __uint_as_float(0x4B000000u | nb) - zb1;
-                }
-#pragma unroll
-                for (int m = 0; m < MP; m++) {
-                    if (m >= p.M)
-                        break;
-                    const unsigned char *xa = xs_base + m * p.xs_stride + sc * 512 + c * 16;
-                    float pa = 0.f, pb = 0.f;
-#pragma unroll
-                    for (int j = 0; j < 8; j++) {
-                        const uint4 v = lds128(xa + j * 64);
-                        const float xv[4] = {__uint_as_float(v.x), __uint_as_float(v.y),
-                                             __uint_as_float(v.z), __uint_as_float(v.w)};
-#pragma unroll
-                        for (int e = 0; e < 4; e++) {
-                            pa = fmaf(xv[e], fa[4 * j + e], pa);
-                            pb = fmaf(xv[e], fb[4 * j + e], pb);
-                        }
-                    }
-                    accc[0][m] = fmaf(s0, pa, accc[0][m]);
-                    accc[1][m] = fmaf(s1, pb, accc[1][m]);
-                }
+                acc[0][m] = fmaf(cur.s0, pa, acc[0][m]);
+                acc[1][m] = fmaf(cur.s1, pb, acc[1][m]);
             }
 
             if (++csc < p.nsc_w)
@@ -395,59 +254,35 @@ __global__ void __launch_bounds__(kThreads, (MODE == MODE_MMA) ? 2 : 1) gemv_ker
             // ---- end of this round's tile for every warp of the CTA (uniform)
             csc = 0;
             const int r = cr++;
-            if (MODE == MODE_CC) {
 #pragma unroll
-                for (int rr = 0; rr < 2; rr++)
+            for (int rr = 0; rr < 2; rr++)
 #pragma unroll
-                    for (int m = 0; m < MP; m++) {
-                        accc[rr][m] += __shfl_xor_sync(0xffffffffu, accc[rr][m], 1);
-                        accc[rr][m] += __shfl_xor_sync(0xffffffffu, accc[rr][m], 2);
-                    }
-            }
+                for (int m = 0; m < MP; m++) {
+                    acc[rr][m] += __shfl_xor_sync(0xffffffffu, acc[rr][m], 1);
+                    acc[rr][m] += __shfl_xor_sync(0xffffffffu, acc[rr][m], 2);
+                }
+            float *Y = reinterpret_cast<float *>(p.Y);
             if (W == 1 && p.S == 1) {
                 // the warp holds the whole dot product: write Y straight from registers
                 const int n0 = tile_at(r, slot) * kRows + g;
-                if (MODE == MODE_MMA) {
-#pragma unroll
-                    for (int t = 0; t < NT; t++)
-#pragma unroll
-                        for (int e = 0; e < 4; e++) {
-                            const int m = 8 * t + 2 * c + (e & 1);
-                            const int n = n0 + 8 * (e >> 1);
-                            if (m < p.M && n < p.N)
-                                reinterpret_cast<__half *>(p.Y)[(int64_t)m * p.N + n] = __float2half_rn(accm[t][e]);
-                        }
-                } else if (c == 0) {
+                if (c == 0) {
 #pragma unroll
                     for (int rr = 0; rr < 2; rr++)
 #pragma unroll
                         for (int m = 0; m < MP; m++) {
                             const int n = n0 + 8 * rr;
-                            if (m < p.M && n < p.N) {
-                                if (ACT_F16)
-                                    reinterpret_cast<__half *>(p.Y)[(int64_t)m * p.N + n] = __float2half_rn(accc[rr][m]);
-                                else
-                                    reinterpret_cast<float *>(p.Y)[(int64_t)m * p.N + n] = accc[rr][m];
-                            }
+                            if (m < p.M && n < p.N)
+                                Y[(int64_t)m * p.N + n] = acc[rr][m];
                         }
                 }
             } else {
                 // partials: warps of a tile in shared memory, then CTAs of the cluster
-                if (MODE == MODE_MMA) {
-#pragma unroll
-                    for (int t = 0; t < NT; t++) {
-                        const int m0 = 8 * t + 2 * c;
-                        red[(warp * kRows + g) * MP + m0] = accm[t][0];
-                        red[(warp * kRows + g) * MP + m0 + 1] = accm[t][1];
-                        red[(warp * kRows + g + 8) * MP + m0] = accm[t][2];
-                        red[(warp * kRows + g + 8) * MP + m0 + 1] = accm[t][3];
-                    }
-                } else if (c == 0) {
+                if (c == 0) {
 #pragma unroll
                     for (int rr = 0; rr < 2; rr++)
 #pragma unroll
                         for (int m = 0; m < MP; m++)
-                            red[(warp * kRows + g + 8 * rr) * MP + m] = accc[rr][m];
+                            red[(warp * kRows + g + 8 * rr) * MP + m] = acc[rr][m];
                 }
                 __syncthreads();
                 for (int idx = tid; idx < TPC * kRows * MP; idx += kThreads) {
@@ -468,29 +303,22 @@ __global__ void __launch_bounds__(kThreads, (MODE == MODE_MMA) ? 2 : 1) gemv_ker
                         float v = part[idx];
                         for (int q = 1; q < p.S; q++)
                             v += ld_dsmem_f32(part + idx, (uint32_t)q);
-                        if (ACT_F16)
-                            reinterpret_cast<__half *>(p.Y)[(int64_t)m * p.N + n] = __float2half_rn(v);
-                        else
-                            reinterpret_cast<float *>(p.Y)[(int64_t)m * p.N + n] = v;
+                        Y[(int64_t)m * p.N + n] = v;
                     }
                 }
                 if (p.S > 1) cluster_sync(); else __syncthreads();
             }
 #pragma unroll
-            for (int t = 0; t < NT; t++)
-#pragma unroll
-                for (int e = 0; e < 4; e++) accm[t][e] = 0.f;
-#pragma unroll
             for (int rr = 0; rr < 2; rr++)
 #pragma unroll
-                for (int m = 0; m < MP; m++) accc[rr][m] = 0.f;
+                for (int m = 0; m < MP; m++) acc[rr][m] = 0.f;
         }
     }
 }
 
-template <int MODE, bool ACT_F16, int MP>
+template <int MP>
 int launch_one(const Params &p, int grid, size_t smem, unsigned flags, cudaStream_t s) {
-    auto fn = gemv_kernel<MODE, ACT_F16, MP>;
+    auto fn = gemv_kernel<MP>;
     static int configured[kMaxDevices] = {};   // largest dynamic shared memory opted into, per device
     if ((int)smem > 48 * 1024) {
         cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(fn), (int)smem, configured);
@@ -524,20 +352,13 @@ int launch_one(const Params &p, int grid, size_t smem, unsigned flags, cudaStrea
     return MNB_OK;
 }
 
-
 }  // namespace
-
-// Which inner product serves fp16 activations at M = 1 and 2: MMA by default.
-static int g_gemv_f16_cc_max_m = 0;
-// 1: fp16 activations go to the warp-specialized streaming kernel for the shapes
-// it serves.  Off by default: on the decoder shapes it is not yet faster than
-// the general TMA kernel.
-static int g_gemv_stream = 0;
 
 // Work decomposition: K slices = W warps x S CTAs per tile, chosen so that
 // about two CTAs of 8 warps per SM have work; rounds of tiles per CTA, with the
 // CTA count balanced so every CTA walks the same number of rounds.
-int plan_gemv(int M, int N, int K, int esz, int MP, int sms, Params &p, int &grid, size_t &smem) {
+static int plan_gemv(int M, int N, int K, int MP, int sms, Params &p, int &grid, size_t &smem) {
+    const int esz = 4;   // fp32 activations
     const int tiles = (N + kRows - 1) / kRows;
     const int nsc_all = (K + kSuper - 1) / kSuper;
     const int target_warps = sms * 2 * kWarps;
@@ -576,20 +397,9 @@ int plan_gemv(int M, int N, int K, int esz, int MP, int sms, Params &p, int &gri
 int launch_gemv(const void *X, int act_f16, const uint8_t *packed, const void *scales,
                 int scale_f16, const uint8_t *zp, void *Y, int M, int N, int K, int bs,
                 unsigned flags, cudaStream_t s) {
-    if (act_f16 && (M > g_gemv_f16_cc_max_m || M > 16)) {   // tensor-core paths, weights streamed by TMA
-        if (g_gemv_stream) {
-            const int rc = launch_gemv_stream(X, packed, scales, scale_f16, zp, Y, M, N, K, bs, flags, s);
-            if (rc != 1)
-                return rc;
-        }
+    if (act_f16)   // tensor-core path, weights streamed by TMA
         return launch_gemv_tc(X, packed, scales, scale_f16, zp, Y, M, N, K, bs, flags, s);
-    }
-    const int mode = MODE_CC;
-    int MP;
-    if (mode == MODE_MMA)
-        MP = (M <= 8) ? 8 : 16;
-    else
-        MP = (M <= 1) ? 1 : (M <= 2) ? 2 : (M <= 4) ? 4 : (M <= 8) ? 8 : 16;
+    const int MP = (M <= 1) ? 1 : (M <= 2) ? 2 : (M <= 4) ? 4 : (M <= 8) ? 8 : 16;
 
     Params p;
     p.X = X; p.packed = packed; p.scales = scales; p.zp = zp; p.Y = Y;
@@ -600,43 +410,16 @@ int launch_gemv(const void *X, int act_f16, const uint8_t *packed, const void *s
     p.scale_f16 = scale_f16;
     int grid = 0;
     size_t smem = 0;
-    int rc = plan_gemv(M, N, K, act_f16 ? 2 : 4, MP, device_sm_count(), p, grid, smem);
+    int rc = plan_gemv(M, N, K, MP, device_sm_count(), p, grid, smem);
     if (rc)
         return rc;
-
-    if (mode == MODE_MMA) {
-        if (MP == 8) return launch_one<MODE_MMA, true, 8>(p, grid, smem, flags, s);
-        return launch_one<MODE_MMA, true, 16>(p, grid, smem, flags, s);
-    }
-    if (act_f16) {
-        if (MP == 1) return launch_one<MODE_CC, true, 1>(p, grid, smem, flags, s);
-        return launch_one<MODE_CC, true, 2>(p, grid, smem, flags, s);
-    }
     switch (MP) {
-        case 1: return launch_one<MODE_CC, false, 1>(p, grid, smem, flags, s);
-        case 2: return launch_one<MODE_CC, false, 2>(p, grid, smem, flags, s);
-        case 4: return launch_one<MODE_CC, false, 4>(p, grid, smem, flags, s);
-        case 8: return launch_one<MODE_CC, false, 8>(p, grid, smem, flags, s);
-        default: return launch_one<MODE_CC, false, 16>(p, grid, smem, flags, s);
+        case 1: return launch_one<1>(p, grid, smem, flags, s);
+        case 2: return launch_one<2>(p, grid, smem, flags, s);
+        case 4: return launch_one<4>(p, grid, smem, flags, s);
+        case 8: return launch_one<8>(p, grid, smem, flags, s);
+        default: return launch_one<16>(p, grid, smem, flags, s);
     }
 }
 
 }  // namespace mnb
-
-// Tuning hook: fp16 GEMVs with M <= max_m use the CUDA-core inner product
-// (0 = always the tensor-core one; at most 2).  Not part of the stable ABI.
-extern "C" MNB_API int mnb_tune_gemv_f16_cc_max_m(int max_m) {
-    if (max_m < 0 || max_m > 2)
-        return MNB_ERR_INVALID_ARG;
-    mnb::g_gemv_f16_cc_max_m = max_m;
-    return MNB_OK;
-}
-
-// Tuning hook: 0 (default) sends every fp16 GEMV to the general TMA kernel, 1
-// lets the streaming kernel take the shapes it serves.  Not part of the stable ABI.
-extern "C" MNB_API int mnb_tune_gemv_stream(int enable) {
-    if (enable != 0 && enable != 1)
-        return MNB_ERR_INVALID_ARG;
-    mnb::g_gemv_stream = enable;
-    return MNB_OK;
-}

@@ -42,6 +42,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "mnb_tune.h"
 
 namespace mnb {
 
@@ -102,6 +103,11 @@ struct ChainParams {
     const ChainTask *tasks;
     unsigned *cnt;       // [ntasks] completion counters, then the abort word
     int ntasks, M, depth, xs_stride, nw;   // nw: compute warps per CTA
+    // fault injection for tests of the timeout path (mnb_test_chain_withhold):
+    // no CTA counts task `withhold` complete (-1: none), and a wait for a
+    // task's inputs gives up after task_wait_ns
+    int withhold;
+    unsigned long long task_wait_ns;
 };
 
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src) {
@@ -338,7 +344,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) gemv_chain_kernel(const ChainP
                         if (ld_acquire_gpu(cp) >= grid)
                             break;
                         if ((i & 63) == 0 &&
-                            (ld_acquire_gpu(p.cnt + p.ntasks) != 0u || globaltimer() - tw > kWaitLimitNs)) {
+                            (ld_acquire_gpu(p.cnt + p.ntasks) != 0u || globaltimer() - tw > p.task_wait_ns)) {
                             flags[0] = 1;
                             atomicOr(&g_chain_status, 2u);
                             atomicExch(p.cnt + p.ntasks, 1u);
@@ -520,7 +526,8 @@ __global__ void __launch_bounds__(kMaxThreads, 1) gemv_chain_kernel(const ChainP
             // by the barrier above) are visible before its count is.  This warp
             // issues no copies, so the release waits for nothing else.
             if (j < p.ntasks - 1) {
-                red_release_gpu(p.cnt + j, 1u);
+                if (j != p.withhold)
+                    red_release_gpu(p.cnt + j, 1u);
             } else if (atom_add_acq_rel_gpu(p.cnt + j, 1u) == grid - 1) {
                 for (int i = 0; i < p.ntasks; i++)   // every CTA is past its last wait
                     p.cnt[i] = 0u;
@@ -587,6 +594,10 @@ int launch_chain_t(const ChainHeader &h, const ChainParams &p, unsigned flags, c
 }
 
 }  // namespace
+
+// Fault injection for tests (mnb_test_chain_withhold): read at each launch.
+static int g_withhold = -1;
+static unsigned long long g_task_wait_ns = kWaitLimitNs;
 
 size_t gemv_chain_plan_bytes(int ntasks) {
     if (ntasks < 1 || ntasks > 65536)
@@ -708,6 +719,8 @@ int launch_gemv_chain(const void *plan, const void *plan_device, void *workspace
     p.depth = h.depth;
     p.xs_stride = h.xs_stride;
     p.nw = h.nw;
+    p.withhold = (g_withhold < h.ntasks - 1) ? g_withhold : -1;   // the last task's count resets the counters
+    p.task_wait_ns = g_task_wait_ns;
     if (h.nw < 7 || h.nw > kMaxWarps || h.depth < 2 || h.depth > kMaxDepth)
         return fail(MNB_ERR_INVALID_ARG, "%s: corrupt plan header", fn);
     if (h.bs == 64) {
@@ -732,3 +745,15 @@ int read_chain_status(unsigned *out, int clear) {
 }
 
 }  // namespace mnb
+
+// Test hook: every later mnb_gemv_chain launch on any thread withholds the
+// completion count of task `task` (-1: none; the last task's count is never
+// withheld) and gives up a wait for a task's inputs after wait_limit_us
+// microseconds (0: the default 2 s).  Declared in mnb_tune.h.
+extern "C" MNB_API int mnb_test_chain_withhold(int task, int wait_limit_us) {
+    if (task < -1 || wait_limit_us < 0 || wait_limit_us > 2000000)
+        return MNB_ERR_INVALID_ARG;
+    mnb::g_withhold = task;
+    mnb::g_task_wait_ns = wait_limit_us ? (unsigned long long)wait_limit_us * 1000ull : mnb::kWaitLimitNs;
+    return MNB_OK;
+}

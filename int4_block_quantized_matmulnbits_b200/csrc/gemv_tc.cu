@@ -38,6 +38,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "mnb_tune.h"
 
 namespace mnb {
 

@@ -22,11 +22,6 @@ int launch_gemv(const void *X, int act_f16, const uint8_t *packed, const void *s
 int launch_gemv_tc(const void *X, const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,
                    void *Y, int M, int N, int K, int bs, unsigned flags, cudaStream_t s);
 
-// Warp-specialized decode kernel for the shapes it serves (M <= 8, K % 256 == 0,
-// aligned scales); returns 1 without launching anything for other shapes.
-int launch_gemv_stream(const void *X, const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,
-                       void *Y, int M, int N, int K, int bs, unsigned flags, cudaStream_t s);
-
 // Decode GEMV with the SwiGLU epilogue over gate/up rows interleaved in 8-row groups.
 int launch_gemv_swiglu(const void *X, const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,
                        void *Y, int M, int N, int K, int bs, unsigned flags, cudaStream_t s);
@@ -60,7 +55,6 @@ int launch_gemv_chain(const void *plan, const void *plan_device, void *workspace
 
 int read_device_status(unsigned *out, int clear);
 int read_gemv_status(unsigned *out, int clear);     // ORs the decode kernel's word into *out
-int read_stream_status(unsigned *out, int clear);   // same for the streaming decode kernel
 int read_chain_status(unsigned *out, int clear);    // the chain kernel's bits, shifted to bits 1-2
 
 }  // namespace mnb

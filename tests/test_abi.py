@@ -12,6 +12,7 @@ import oracle
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "mnb.h")
+TUNE_HEADER = os.path.join(ROOT, "include", "mnb_tune.h")
 
 OK, INVALID, SHAPE, ALIGN, UNSUPPORTED = 0, -1, -2, -3, -4
 F32, F16 = 0, 1
@@ -30,8 +31,8 @@ def lib(mnb):
     return mnb._lib
 
 
-def declared_functions():
-    text = open(HEADER).read()
+def declared_functions(path=HEADER):
+    text = open(path).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(mnb_[a-z0-9_]+)\s*\(", text)))
 
@@ -47,6 +48,24 @@ def test_library_exports_every_declared_symbol(mnb):
     raw = ctypes.CDLL(mnb.lib_path)
     for name in declared_functions():
         assert hasattr(raw, name), name
+
+
+def exported_functions(path):
+    """Names of the mnb_* functions the shared library exports (nm -D)."""
+    import subprocess
+
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True, check=True).stdout
+    return sorted({ln.split()[-1] for ln in out.splitlines() if ln.split() and ln.split()[-1].startswith("mnb_")})
+
+
+def test_every_exported_symbol_is_declared(mnb):
+    # the stable entry points in mnb.h, the tuning hooks in mnb_tune.h; nothing else
+    declared = set(declared_functions()) | set(declared_functions(TUNE_HEADER))
+    exported = exported_functions(mnb.lib_path)
+    assert exported, "nm found no mnb_* symbols"
+    assert sorted(set(exported) - declared) == []
+    for name in declared_functions(TUNE_HEADER):
+        assert name in exported, name
 
 
 def test_version_and_empty_error(mnb):
@@ -91,6 +110,7 @@ def test_gemv_argument_checks(lib):
 def test_gemm_argument_checks(lib):
     g = lib.mnb_gemm
     assert g(A, F32, A, A, F16, A, A, 64, 128, 64, 32, 0, None) == UNSUPPORTED   # fp32 activations
+    assert g(A, F16, A, A, F32, A, A, 64, 128, 64, 32, 0, None) == UNSUPPORTED   # fp32 scales (q4 + fp16 X)
     assert g(A, F16, A, A, F16, A, A, 64, 100, 64, 32, 0, None) == SHAPE          # N % 128
     assert g(A, F16, A, A, F16, A, A, 64, 128, 96, 32, 0, None) == SHAPE          # K % 64
     assert g(A, F16, A + 4, A, F16, A, A, 64, 128, 64, 32, 0, None) == ALIGN

@@ -174,3 +174,64 @@ def test_chain_refuses_a_workspace_left_dirty(mnb, cuda_dev):
     torch.cuda.synchronize()
     assert mnb.mnb_device_status() == 0
     assert_close(np_of(Y.float()), oracle.matmul(np_of(x.float()), *host, K, 32), "f16")
+
+
+def test_chain_task_wait_times_out_and_reports_it(mnb, cuda_dev):
+    # fault made on the host: the test hook withholds task 0's completion count,
+    # so task 1's bounded wait for its inputs runs out (after 5 ms here).  The
+    # kernel must return, set status bit 2 and the abort word, leave the later
+    # tasks' outputs untouched; the next call must refuse the dirty workspace
+    # (bit 3); after zero-filling it, a normal call gives correct results.
+    rng = np.random.default_rng(11)
+    M, bs = 2, 32
+    shapes = [(2048, 1024), (1024, 2048), (1024, 1024)]   # task j reads task j-1's Y
+    x0 = torch.randn((M, 1024), generator=torch.Generator().manual_seed(12)).half().to(cuda_dev)
+    host, tasks, Ys = [], [], []
+    X = x0
+    for j, (N, K) in enumerate(shapes):
+        h, d = _weights(rng, N, K, bs, True, cuda_dev)
+        Y = torch.full((M, N), 7.0, dtype=torch.float16, device=cuda_dev)
+        tasks.append((X, *d, Y, N, K, 1 if j else 0))
+        host.append(h)
+        Ys.append(Y)
+        X = Y
+    plan = mnb.mnb_gemv_chain_plan(tasks, M, bs)
+    plan_dev = plan.to(cuda_dev)
+    ws = torch.zeros(mnb.mnb_gemv_chain_workspace_bytes(len(tasks)), dtype=torch.uint8, device=cuda_dev)
+    mnb.mnb_device_status(clear=True)
+    assert mnb._lib.mnb_test_chain_withhold(0, 5000) == 0
+    try:
+        mnb.mnb_gemv_chain(plan, plan_dev, ws)
+        torch.cuda.synchronize()
+    finally:
+        assert mnb._lib.mnb_test_chain_withhold(-1, 0) == 0
+    st = ctypes_status(mnb)
+    assert st["rc"] == -6 and st["word"] & (1 << 2), st
+    assert int(ws.view(torch.int32)[len(tasks)].item()) != 0, "the abort word must be raised"
+    assert bool((Ys[1] == 7.0).all()) and bool((Ys[2] == 7.0).all()), "tasks after the timeout must not run"
+    # the same workspace again: refused, nothing runs
+    mnb.mnb_gemv_chain(plan, plan_dev, ws)
+    torch.cuda.synchronize()
+    st = ctypes_status(mnb)
+    assert st["rc"] == 0 and st["word"] == (1 << 3), st
+    assert bool((Ys[2] == 7.0).all())
+    # zero-filled again: a normal call
+    ws.zero_()
+    mnb.mnb_gemv_chain(plan, plan_dev, ws)
+    torch.cuda.synchronize()
+    assert mnb.mnb_device_status() == 0
+    assert int(ws.count_nonzero()) == 0
+    X = np_of(x0.float())
+    for (N, K), h, Y in zip(shapes, host, Ys):
+        ref = oracle.matmul(X, *h, K, bs)
+        assert_close(np_of(Y.float()), ref, "f16")
+        X = np_of(Y.float())
+
+
+def ctypes_status(mnb):
+    """The C call's return code and the status word it read (then cleared)."""
+    import ctypes
+
+    v = ctypes.c_uint()
+    rc = mnb._lib.mnb_device_status(ctypes.byref(v), 1)
+    return {"rc": rc, "word": v.value}

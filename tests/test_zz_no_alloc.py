@@ -5,7 +5,8 @@ owns every device allocation, a decode thread that must not call the
 allocator between tokens).  For them the library keeps the scratch of
 mnb_gemv_argmax in a device array of its own.  Checked here against
 mnb_gemv_argmax with a caller workspace, on the same inputs, two calls in a
-row (the second call finds the first call's leftovers in the shared array).
+row (the second call finds the first call's leftovers in the shared array):
+the outputs must be identical, and right against the oracle.
 
 This file is named so that pytest collects it last.
 """
@@ -13,6 +14,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from tests.parity_util import assert_close, np_of, random_packed, to_dev
 
 pytestmark = pytest.mark.gpu
@@ -44,12 +46,20 @@ def test_noalloc_matches_workspace_entry_point(mnb, cuda_dev, M, N, K, bs, has_z
             else:
                 mnb.mnb_gemv_argmax(X, dp, ds, dz, Y, M, N, K, bs, ids, mx, ws)
             torch.cuda.synchronize()
-            outs.append((np_of(Y.float()), np_of(ids), np_of(mx)))
+            outs.append((Y, ids, mx))
         (y0, i0, m0), (y1, i1, m1) = outs
-        assert_close(y1, y0, "f16")
-        assert np.array_equal(i1, np.argmax(y1, axis=1))
-        assert np.array_equal(m1, y1[np.arange(M), i1])
-        assert np.all(y0[np.arange(M), i1] >= y0.max(axis=1) - 2e-2)
+        # the same kernel on the same inputs: identical logits, tokens and maxima
+        assert torch.equal(y1, y0)
+        assert torch.equal(i1, i0)
+        assert torch.equal(m1, m0)
+        # and both right: the logits within tolerance of the oracle, the token
+        # the first maximum of the logits, and a greedy choice for the oracle's
+        yn, idn = np_of(y1.float()), np_of(i1)
+        ref = oracle.matmul(np_of(X.float()), packed, scales, zp, K, bs)
+        assert_close(yn, ref, "f16")
+        assert np.array_equal(idn, np.argmax(yn, axis=1))
+        assert np.array_equal(np_of(m1), yn[np.arange(M), idn])
+        assert np.all(ref[np.arange(M), idn] >= ref.max(axis=1) - 2e-2)
 
 
 def test_noalloc_rejects_requests_outside_its_limits(mnb, cuda_dev):
