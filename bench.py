@@ -36,7 +36,7 @@ WORKLOAD = ("qwen3-1.7b-shaped decode step, M=1: 28 layers x (q 2048->2048, k/v 
             "int4 block 32 asymmetric, fp16 activations and scales, weights N(0,0.02) with 1% outliers x8")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-DECODE_KERNEL = "gemv_tc_kernel"   # the kernel of the decode step's launches
+DECODE_KERNEL = "gemv_resident_kernel"   # the kernel of the decode step's launches (M = 1)
 NOMINAL = {"hbm_gbs": 8000.0, "tc_tflops": 2250.0}   # B200 spec sheet: HBM3e, dense fp16/bf16
 
 
@@ -753,6 +753,7 @@ def run_gpu(args, world, rank, local):
                            "weight_gbs": round(ep.weight_bytes / (t * 1e-3) / 1e9, 1)}
         del ep
     del elins
+    n_launches = len(lins)
     del lins, body
     torch.cuda.empty_cache()
     with_oracle = rank == 0 and world == 1
@@ -785,7 +786,7 @@ def run_gpu(args, world, rank, local):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
             "data": "synthetic",
-            "config": {"workload": WORKLOAD, "M": 1, "launches_per_step": len(lins),
+            "config": {"workload": WORKLOAD, "M": 1, "launches_per_step": n_launches,
                        "weight_bytes_per_step": wbytes, "graph": True, "pdl": True,
                        "l2": "inputs larger than L2 (weights of one step > 126 MB)",
                        "parallelism": f"replicas x{world}"},
@@ -823,7 +824,7 @@ def run_gpu(args, world, rank, local):
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_val, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
-            "gpu_launches": args.steps * len(lins),
+            "gpu_launches": args.steps * n_launches,
             "clocks": clk.summary(),
         }
         print(json.dumps(out), flush=True)

@@ -28,6 +28,11 @@ MNB_API int mnb_tune_gemm_tiles(int min_bn, int max_bn, int max_split);
  * choice back to the planner. */
 MNB_API int mnb_tune_gemv_split(int w, int s);
 
+/* fp16 decode GEMV at M = 1: 1 (default) runs the kernel whose CTAs hold
+ * their whole share of the weights in shared memory, where the shape allows
+ * it; 0 runs the general decode kernel. */
+MNB_API int mnb_tune_gemv_resident(int enable);
+
 /* Fault injection for tests of mnb_gemv_chain's timeout path (no GPU fault,
  * no hang): every later launch leaves task `task` uncounted, so the next task
  * that waits for it gives up after wait_limit_us microseconds (0 = the

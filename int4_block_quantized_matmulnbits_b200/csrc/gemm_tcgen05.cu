@@ -651,6 +651,8 @@ int read_device_status(unsigned *out, int clear) {
     if (e == cudaSuccess) {
         int rc = read_gemv_status(out, clear);
         if (!rc)
+            rc = read_res_status(out, clear);
+        if (!rc)
             rc = read_chain_status(out, clear);
         if (rc)
             return rc;

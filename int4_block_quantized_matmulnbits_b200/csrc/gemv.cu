@@ -31,6 +31,7 @@
 // across the 4 lanes of a row with warp shuffles.
 #include "common.cuh"
 #include "internal.h"
+#include "mnb_tune.h"
 
 namespace mnb {
 
@@ -394,11 +395,20 @@ static int plan_gemv(int M, int N, int K, int MP, int sms, Params &p, int &grid,
     return MNB_OK;
 }
 
+// One-token fp16 calls go to the resident kernel (1) or the general one (0).
+static int g_resident = 1;
+
 int launch_gemv(const void *X, int act_f16, const uint8_t *packed, const void *scales,
                 int scale_f16, const uint8_t *zp, void *Y, int M, int N, int K, int bs,
                 unsigned flags, cudaStream_t s) {
-    if (act_f16)   // tensor-core path, weights streamed by TMA
+    if (act_f16) {   // tensor-core paths, weights moved by TMA
+        if (M == 1 && scale_f16 && g_resident) {
+            const int rc = launch_gemv_resident(X, packed, scales, zp, Y, N, K, bs, flags, s);
+            if (rc != 1)
+                return rc;
+        }
         return launch_gemv_tc(X, packed, scales, scale_f16, zp, Y, M, N, K, bs, flags, s);
+    }
     const int MP = (M <= 1) ? 1 : (M <= 2) ? 2 : (M <= 4) ? 4 : (M <= 8) ? 8 : 16;
 
     Params p;
@@ -423,3 +433,13 @@ int launch_gemv(const void *X, int act_f16, const uint8_t *packed, const void *s
 }
 
 }  // namespace mnb
+
+// Tuning hook: 1 (default) sends one-token fp16 GEMVs to the resident decode
+// kernel where it applies, 0 to the general decode kernel.  Declared in
+// mnb_tune.h.
+extern "C" MNB_API int mnb_tune_gemv_resident(int enable) {
+    if (enable != 0 && enable != 1)
+        return MNB_ERR_INVALID_ARG;
+    mnb::g_resident = enable;
+    return MNB_OK;
+}

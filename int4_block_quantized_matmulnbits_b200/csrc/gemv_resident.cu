@@ -1,0 +1,479 @@
+// gemv_resident.cu -- decode-shaped MatMulNBits for ONE token with fp16
+// activations: y[N] = x[K] . dequant(W)^T, the per-token decoder step of
+// "Qwen3-ASR-0.6B -- ONNX for the browser" ("Graph contracts": decoder_step,
+// input_embeds [1, 1, 1024]) and of "Mega-ASR -- INT4 ONNX (GPTQ-calibrated)"
+// (decoder_step_int4).
+//
+// A decode step is a chain of ~200 such GEMVs, each waiting for the one before
+// it.  Most move 1-7 MB of weights -- well under 2 us of HBM time -- so what
+// costs is the critical path from "previous kernel done" to "this kernel's y
+// stored".  This kernel is built to keep that path short:
+//   * Half an SM per CTA (8 warps, <= 128 registers, ~110 KB of shared
+//     memory), one CTA per SM.  While kernel i runs, the CTAs of kernel i+1
+//     (launched early by programmatic dependent launch) sit on the other half
+//     of every SM and pull ALL of their weights into shared memory: each warp
+//     owns a ring of `depth` slots, one slot = one 16-row x 256-k box of
+//     packed bytes (TMA, 128-byte swizzle) plus its scales and zero points
+//     (cp.async), completing on one mbarrier.  For the decoder's projections
+//     every unit fits in the rings, so after griddepcontrol.wait only x is
+//     read from memory; the lm_head streams through the same rings.
+//   * Work split: CTA b owns a contiguous run of 16-row tiles; its (tile, box)
+//     units are cut into one contiguous run per warp.  Tiles a warp covers
+//     whole are stored from registers; the partial sums of tiles cut between
+//     warps meet in shared memory and are added in warp order (deterministic).
+//     Nothing crosses CTAs: no cluster, no atomics, no global scratch.
+//   * Zero point and scale are applied per block AFTER the tensor core, not
+//     per weight.  The MMA (mma.sync m16n8k16, fp32 accumulation) takes the
+//     raw codes: (nibble | 0x6400) is the fp16 1024+q exactly for a low
+//     nibble, 1024+16q for a high nibble (met by x/16, staged exact), so 8
+//     weights cost one shift and four LOP3.  With one token, 7 of the MMA's 8
+//     columns would be wasted; instead column j collects block j of the box:
+//     the x fragment of the thread whose column is j holds x only for the k of
+//     block j, zeros elsewhere.  After a box the accumulator holds, for every
+//     (row, block), D = sum_k (1024 + q~) x~, started from -P with
+//     P = 1024 sum_k x~; the block's dot product is then
+//     sum_k (q - zp) x = D - zp Q, Q = sum_k x (both sums per block of x,
+//     computed once per call), and y += scale * (D - zp Q).  Four correction
+//     FMAs per thread per box replace two half2 operations per weight pair.
+// Every mbarrier wait is bounded in time; past the limit the kernel records
+// the failure in the device status word, lets its copies in flight land and
+// exits.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace mnb {
+
+__device__ unsigned g_res_status = 0;
+
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kRows = 16;
+constexpr int kBoxK = 256;                  // k per box: 8 blocks of 32 (4 of 64)
+constexpr int kBoxBytes = kRows * 128;
+constexpr int kParBytes = 320;              // 16 rows x 16 B of scales, then 16 rows x 4 B of zero points
+constexpr int kChunk = 80;                  // staged bytes per 32-k chunk of x: 64, then 16 of padding
+constexpr int kMaxDepth = 8;
+constexpr int kSmemBudget = 110 * 1024;     // two CTAs (of consecutive kernels) per SM
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+struct ResParams {
+    const __half *X;          // [K]
+    const uint8_t *scales;    // fp16 [N][nb]
+    const uint8_t *zp;        // [N][zpb] or null (zero point 8)
+    __half *Y;                // [N]
+    int N, K, nb, zpb;
+    int ntiles, nbx, nchunks; // ceil(N / 16), K / 256, K / 32
+    int tq, tr;               // tiles per CTA: tq, one more for CTAs below tr
+    int depth;                // ring slots per warp
+};
+
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_8(uint32_t dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+// One arrival on `bar` once all of this thread's earlier cp.async copies have
+// landed (the barrier's expected count includes it).
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+// Bounded wait on a warp-private mbarrier; after the first timeout it returns
+// at once, so the warp runs to the end without waiting again.
+__device__ __forceinline__ void slot_wait(uint32_t bar, uint32_t parity, bool &dead) {
+    if (dead || mbar_try_wait(bar, parity))
+        return;
+    const unsigned long long t0 = globaltimer();
+    for (uint32_t i = 1;; i++) {
+        if (mbar_try_wait(bar, parity))
+            return;
+        if ((i & 255) == 0 && globaltimer() - t0 > kWaitLimitNs) {
+            dead = true;
+            atomicOr(&g_res_status, 1u);
+            return;
+        }
+    }
+}
+
+// Requests unit (tile, box) into a ring slot: the packed box by TMA (lane 0),
+// the box's scales (lanes 0-15) and zero points (lanes 16-31) by cp.async.
+// Rows past N get no parameters (their sums are never stored).  Every lane
+// arrives on the slot's barrier once its copies have landed.
+template <bool BS64, bool ZP>
+__device__ __forceinline__ void issue(const CUtensorMap *wmap, const ResParams &p, int tile, int box, uint32_t box_dst,
+                                      uint32_t par_dst, uint32_t full, int lane) {
+    const int n0 = tile * kRows;
+    if (lane == 0) {
+        mbar_expect_tx(full, kBoxBytes);
+        tma_load_2d(box_dst, wmap, full, box * 128, n0);
+    }
+    if (lane < 16) {
+        if (n0 + lane < p.N) {
+            const uint8_t *src = p.scales + ((int64_t)(n0 + lane) * p.nb + box * (BS64 ? 4 : 8)) * 2;
+            if (BS64) cp_async_8(par_dst + lane * 16, src); else cp_async_16(par_dst + lane * 16, src);
+        }
+    } else if (ZP) {
+        const int row = lane - 16;
+        if (n0 + row < p.N) {
+            const uint8_t *src = p.zp + (int64_t)(n0 + row) * p.zpb + (BS64 ? (box >> 1) * 4 : box * 4);
+            cp_async_4(par_dst + 256 + row * 4, src);
+        }
+    }
+    cp_async_arrive(full);
+}
+
+// Scales of the box's columns 2c and 2c+1 (32-k chunks) of a row, from its
+// slot's parameter area, as fp32.
+template <bool BS64>
+__device__ __forceinline__ float2 scale_pair(const unsigned char *par, int row, int c) {
+    if (!BS64) {   // blocks 2c, 2c+1
+        const uint32_t v = *reinterpret_cast<const uint32_t *>(par + row * 16 + c * 4);
+        return __half22float2(u32_as_h2(v));
+    }
+    // block 64: columns 2c, 2c+1 are the two halves of block c of the box
+    const float s = __half2float(__ushort_as_half(*reinterpret_cast<const unsigned short *>(par + row * 16 + c * 2)));
+    return make_float2(s, s);
+}
+
+// Zero points of columns 2c, 2c+1 of a row, as fp32.
+template <bool BS64, bool ZP>
+__device__ __forceinline__ float2 zp_pair(const unsigned char *par, int row, int c, int box) {
+    if (!ZP)
+        return make_float2(8.f, 8.f);
+    if (!BS64) {
+        const uint32_t zb = par[256 + row * 4 + c];   // blocks 2c (low nibble) and 2c+1 (high)
+        return make_float2((float)(zb & 15u), (float)(zb >> 4));
+    }
+    const uint32_t zb = par[256 + row * 4 + (box & 1) * 2 + (c >> 1)];
+    const float z = (float)((c & 1) ? (zb >> 4) : (zb & 15u));
+    return make_float2(z, z);
+}
+
+template <bool BS64, bool ZP>
+__global__ void __launch_bounds__(kThreads, 2)
+    gemv_resident_kernel(const __grid_constant__ CUtensorMap wmap, const ResParams p) {
+    extern __shared__ unsigned char smem_raw[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, c = lane & 3;
+    const int D = p.depth;
+
+    // shared memory (1024-aligned): boxes | params | x | zero chunk | (P, Q) |
+    // partial sums | their tiles | barriers
+    const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    unsigned char *bp = smem_raw + (base - smem_u32(smem_raw));
+    unsigned char *pars = bp + kWarps * D * kBoxBytes;
+    unsigned char *xs = pars + kWarps * D * kParBytes;
+    unsigned char *zchunk = xs + p.nchunks * kChunk;
+    float2 *pq = reinterpret_cast<float2 *>(zchunk + kChunk);
+    float *part = reinterpret_cast<float *>(pq + p.nchunks);      // [warp][2 slots][16 rows]
+    int *part_tile = reinterpret_cast<int *>(part + kWarps * 2 * kRows);
+    const uint32_t bars = smem_u32(part_tile + kWarps * 2);
+    const uint32_t my_box = base + (uint32_t)(warp * D * kBoxBytes);
+    const unsigned char *my_box_ptr = bp + warp * D * kBoxBytes;
+    const uint32_t my_par = smem_u32(pars) + (uint32_t)(warp * D * kParBytes);
+    const unsigned char *my_par_ptr = pars + warp * D * kParBytes;
+    const uint32_t my_bars = bars + (uint32_t)(warp * D * 8);
+
+    // this CTA's tiles and this warp's run of (tile, box) units
+    const int cta = blockIdx.x;
+    const int Tc = p.tq + (cta < p.tr ? 1 : 0);
+    const int t0 = cta * p.tq + (cta < p.tr ? cta : p.tr);
+    const int U = Tc * p.nbx;
+    const int u0 = warp * U / kWarps, u1 = (warp + 1) * U / kWarps;
+
+    if (lane == 0) {
+        for (int d = 0; d < D; d++)
+            mbar_init(my_bars + 8 * d, 33);   // lane 0's expect_tx + one cp.async arrival per lane
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (tid < kWarps * 2)
+        part_tile[tid] = -1;
+    __syncwarp();
+
+    // ---- weights first: they do not depend on the previous kernel
+    int iu = u0, islot = 0;   // next unit to request, its slot
+    auto request = [&]() {
+        const int tl = iu / p.nbx;
+        issue<BS64, ZP>(&wmap, p, t0 + tl, iu - tl * p.nbx, my_box + islot * kBoxBytes, my_par + islot * kParBytes,
+                        my_bars + 8 * islot, lane);
+        ++iu;
+        if (++islot == D) islot = 0;
+    };
+    while (iu < u1 && iu - u0 < D)
+        request();
+    pdl_launch_dependents();
+    pdl_wait();
+
+    // ---- stage x: chunk j (k = 32j .. 32j+31) as four 16-byte words, word w =
+    // (x0,x4) (x1,x5)/16 (x2,x6) (x3,x7)/16 of k = 32j + 8w ..; and per chunk
+    // P = 1024 sum x~ and Q = sum x over the staged values x~ (x/16 counted
+    // back as 16 x~), so the correction matches the MMA's operands exactly
+    {
+        const half2 sixteenth = __floats2half2_rn(0.0625f, 0.0625f);
+        for (int j = tid; j < p.nchunks; j += kThreads) {
+            uint4 vv[4];
+#pragma unroll
+            for (int w = 0; w < 4; w++)
+                vv[w] = ldg_v4(p.X + j * 32 + 8 * w);
+            float lo = 0.f, hi = 0.f;   // sum of the low-position x, of the high-position x~
+#pragma unroll
+            for (int w = 0; w < 4; w++) {
+                const uint4 v = vv[w];
+                uint4 o;
+                o.x = __byte_perm(v.x, v.z, 0x5410);
+                o.y = h2_as_u32(__hmul2(u32_as_h2(__byte_perm(v.x, v.z, 0x7632)), sixteenth));
+                o.z = __byte_perm(v.y, v.w, 0x5410);
+                o.w = h2_as_u32(__hmul2(u32_as_h2(__byte_perm(v.y, v.w, 0x7632)), sixteenth));
+                *reinterpret_cast<uint4 *>(xs + j * kChunk + w * 16) = o;
+                const float2 a = __half22float2(u32_as_h2(o.x)), b = __half22float2(u32_as_h2(o.y));
+                const float2 e = __half22float2(u32_as_h2(o.z)), f = __half22float2(u32_as_h2(o.w));
+                lo += (a.x + a.y) + (e.x + e.y);
+                hi += (b.x + b.y) + (f.x + f.y);
+            }
+            pq[j] = make_float2(1024.f * (lo + hi), lo + 16.f * hi);
+        }
+        if (tid < kChunk / 16)
+            reinterpret_cast<uint4 *>(zchunk)[tid] = make_uint4(0, 0, 0, 0);
+    }
+    __syncthreads();
+
+    // ---- this warp's units
+    bool dead = false;
+    int cslot = 0, cph = 0;
+    float ya = 0.f, yb = 0.f;   // rows g and g+8 of the current tile segment
+    bool seg_from0 = false;
+    int nseg = 0;               // segments of this warp emitted so far
+    const int hm = g - 2 * c;   // the half (0 or 1) in which this thread's column takes x, if any
+    for (int u = u0; u < u1; u++) {
+        const int tl = u / p.nbx, box = u - tl * p.nbx;
+        if (u == u0 || box == 0) {
+            ya = yb = 0.f;
+            seg_from0 = (box == 0);
+        }
+        slot_wait(my_bars + 8 * cslot, (uint32_t)cph, dead);
+        dead = __any_sync(0xffffffffu, dead);   // one verdict per warp: it issues refills together
+        const unsigned char *bx = my_box_ptr + cslot * kBoxBytes;
+        const unsigned char *par = my_par_ptr + cslot * kParBytes;
+        const float4 pqv = *reinterpret_cast<const float4 *>(pq + box * 8 + 2 * c);   // P, Q of columns 2c, 2c+1
+        // two independent MMA chains (one per half of the box), the first
+        // started from -P
+        float acc2[2][4] = {{-pqv.x, -pqv.z, -pqv.x, -pqv.z}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int h = 0; h < 2; h++) {
+            float *acc = acc2[h];
+            const int chunk = 2 * c + h;
+            const uint4 va = *reinterpret_cast<const uint4 *>(bx + g * 128 + ((chunk ^ g) << 4));
+            const uint4 vb = *reinterpret_cast<const uint4 *>(bx + (g + 8) * 128 + ((chunk ^ g) << 4));
+            // x of chunk `chunk` goes to column `chunk` only: the thread whose
+            // column that is (g == chunk) reads it, every other thread zeros
+            const unsigned char *xa = (hm == h) ? xs + (box * 8 + chunk) * kChunk : zchunk;
+            const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
+            const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+            for (int w = 0; w < 4; w++) {
+                const uint4 xv = *reinterpret_cast<const uint4 *>(xa + w * 16);
+                const uint32_t a8 = wa[w] >> 8, b8 = wb[w] >> 8;
+                const uint32_t a0 = lop3_and_or(wa[w], 0x000F000Fu, 0x64006400u);   // (e0, e4): 1024 + q
+                const uint32_t a1 = lop3_and_or(wa[w], 0x00F000F0u, 0x64006400u);   // (e1, e5): 1024 + 16 q
+                const uint32_t a2 = lop3_and_or(a8, 0x000F000Fu, 0x64006400u);      // (e2, e6)
+                const uint32_t a3 = lop3_and_or(a8, 0x00F000F0u, 0x64006400u);      // (e3, e7)
+                const uint32_t b0 = lop3_and_or(wb[w], 0x000F000Fu, 0x64006400u);
+                const uint32_t b1 = lop3_and_or(wb[w], 0x00F000F0u, 0x64006400u);
+                const uint32_t b2 = lop3_and_or(b8, 0x000F000Fu, 0x64006400u);
+                const uint32_t b3 = lop3_and_or(b8, 0x00F000F0u, 0x64006400u);
+                mma16816(acc, a0, b0, a1, b1, xv.x, xv.y);
+                mma16816(acc, a2, b2, a3, b3, xv.z, xv.w);
+            }
+        }
+        // correction: columns 2c, 2c+1 of rows g and g+8
+        {
+            float acc[4];
+#pragma unroll
+            for (int e = 0; e < 4; e++) acc[e] = acc2[0][e] + acc2[1][e];
+            const float2 sa = scale_pair<BS64>(par, g, c), sb = scale_pair<BS64>(par, g + 8, c);
+            const float2 za = zp_pair<BS64, ZP>(par, g, c, box), zb = zp_pair<BS64, ZP>(par, g + 8, c, box);
+            if (!dead) {
+                ya = fmaf(sa.x, fmaf(-za.x, pqv.y, acc[0]), ya);
+                ya = fmaf(sa.y, fmaf(-za.y, pqv.w, acc[1]), ya);
+                yb = fmaf(sb.x, fmaf(-zb.x, pqv.y, acc[2]), yb);
+                yb = fmaf(sb.y, fmaf(-zb.y, pqv.w, acc[3]), yb);
+            }
+        }
+        __syncwarp();
+        if (++cslot == D) { cslot = 0; cph ^= 1; }
+        if (!dead && iu < u1) {
+            fence_proxy_async_smem();   // this warp's reads of the slot precede the TMA that refills it
+            request();
+        }
+        // ---- end of a tile segment
+        if (box == p.nbx - 1 || u + 1 == u1) {
+            ya += __shfl_xor_sync(0xffffffffu, ya, 1);
+            ya += __shfl_xor_sync(0xffffffffu, ya, 2);
+            yb += __shfl_xor_sync(0xffffffffu, yb, 1);
+            yb += __shfl_xor_sync(0xffffffffu, yb, 2);
+            const int tile = t0 + tl;
+            if (seg_from0 && box == p.nbx - 1) {
+                if (c == 0 && !dead) {
+                    const int n = tile * kRows + g;
+                    if (n < p.N) p.Y[n] = __float2half_rn(ya);
+                    if (n + 8 < p.N) p.Y[n + 8] = __float2half_rn(yb);
+                }
+            } else {
+                // a partial: the first segment of the run in slot 0, the last in slot 1
+                const int s = (nseg == 0) ? 0 : 1;
+                if (c == 0) {
+                    part[(warp * 2 + s) * kRows + g] = ya;
+                    part[(warp * 2 + s) * kRows + g + 8] = yb;
+                }
+                if (lane == 0)
+                    part_tile[warp * 2 + s] = tile;
+            }
+            ++nseg;
+        }
+    }
+    __syncthreads();
+
+    // ---- tiles cut between warps: the first warp slot holding a tile adds
+    // every slot holding it, in warp order, and stores the rows
+    {
+        const int sl = tid >> 4, row = tid & 15;   // 16 slots x 16 rows = 256 threads
+        const int tile = part_tile[sl];
+        bool leader = tile >= 0;
+        for (int q = 0; q < sl && leader; q++)
+            leader = part_tile[q] != tile;
+        if (leader) {
+            float v = 0.f;
+            for (int q = sl; q < kWarps * 2; q++)
+                if (part_tile[q] == tile)
+                    v += part[q * kRows + row];
+            const int n = tile * kRows + row;
+            if (n < p.N && !dead)
+                p.Y[n] = __float2half_rn(v);
+        }
+    }
+
+    // after a timeout: let the copies still in flight (at most one ring's
+    // worth) land before the CTA's shared memory is released
+    if (dead && lane == 0) {
+        const int issued = iu - u0;
+        for (int q = (issued > D ? issued - D : 0); q < issued; q++) {
+            const uint32_t bar = my_bars + 8 * (q % D);
+            const unsigned long long tw = globaltimer();
+            while (!mbar_try_wait(bar, (uint32_t)((q / D) & 1)) && globaltimer() - tw < kWaitLimitNs) {
+            }
+        }
+    }
+}
+
+size_t res_smem_bytes(int depth, int nchunks) {
+    return 1024 + (size_t)kWarps * depth * (kBoxBytes + kParBytes + 8) + (size_t)nchunks * (kChunk + 8) + kChunk +
+           (size_t)kWarps * 2 * (kRows * 4 + 4);
+}
+
+template <bool BS64, bool ZP>
+int launch_res_t(const CUtensorMap &map, const ResParams &p, int grid, size_t smem, unsigned flags, cudaStream_t s) {
+    auto fn = gemv_resident_kernel<BS64, ZP>;
+    static int configured[kMaxDevices] = {};
+    {
+        cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(fn), (int)smem, configured);
+        if (e != cudaSuccess)
+            return fail(MNB_ERR_CUDA, "mnb_gemv: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    int na = 0;
+    if (flags & MNB_FLAG_PDL) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        na++;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, fn, map, p);
+    if (e != cudaSuccess)
+        return fail(MNB_ERR_CUDA, "mnb_gemv: launch: %s", cudaGetErrorString(e));
+    return MNB_OK;
+}
+
+}  // namespace
+
+int launch_gemv_resident(const void *X, const uint8_t *packed, const void *scales, const uint8_t *zp, void *Y, int N,
+                         int K, int bs, unsigned flags, cudaStream_t s) {
+    const bool bs64 = (bs == 64), has_zp = (zp != nullptr);
+    if (K % kBoxK != 0 || (bs64 && has_zp && K % 512 != 0) || !aligned(scales, bs64 ? 8 : 16) ||
+        (has_zp && !aligned(zp, 4)))
+        return 1;   // not a shape this kernel serves
+    ResParams p;
+    p.X = static_cast<const __half *>(X);
+    p.scales = static_cast<const uint8_t *>(scales);
+    p.zp = zp;
+    p.Y = static_cast<__half *>(Y);
+    p.N = N;
+    p.K = K;
+    p.nb = K / bs;
+    p.zpb = (p.nb + 1) / 2;
+    p.ntiles = (N + kRows - 1) / kRows;
+    p.nbx = K / kBoxK;
+    p.nchunks = K / 32;
+    const int sms = device_sm_count();
+    const int grid = p.ntiles < sms ? p.ntiles : sms;
+    p.tq = p.ntiles / grid;
+    p.tr = p.ntiles % grid;
+    // the deepest ring (up to the most units a warp owns) that keeps two CTAs per SM
+    const int Umax = (p.tq + (p.tr ? 1 : 0)) * p.nbx;
+    const int per_warp = (Umax + kWarps - 1) / kWarps;
+    int depth = per_warp < kMaxDepth ? (per_warp < 2 ? 2 : per_warp) : kMaxDepth;
+    while (depth > 2 && res_smem_bytes(depth, p.nchunks) > (size_t)kSmemBudget)
+        --depth;
+    if (res_smem_bytes(depth, p.nchunks) > (size_t)kSmemBudget)
+        return 1;
+    p.depth = depth;
+    const size_t smem = res_smem_bytes(depth, p.nchunks);
+
+    EncodeTiledFn encode = tensor_map_encoder();
+    if (!encode)
+        return fail(MNB_ERR_CUDA, "mnb_gemv: cuTensorMapEncodeTiled unavailable");
+    CUtensorMap map;
+    const cuuint64_t gdim[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N};
+    const cuuint64_t gstride[1] = {(cuuint64_t)(K / 2)};
+    const cuuint32_t box[2] = {128, (cuuint32_t)kRows};
+    const cuuint32_t estride[2] = {1, 1};
+    CUresult cr = encode(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), gdim, gstride, box,
+                         estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS)
+        return fail(MNB_ERR_CUDA, "mnb_gemv: cuTensorMapEncodeTiled failed (%d)", (int)cr);
+    if (bs64) {
+        if (has_zp) return launch_res_t<true, true>(map, p, grid, smem, flags, s);
+        return launch_res_t<true, false>(map, p, grid, smem, flags, s);
+    }
+    if (has_zp) return launch_res_t<false, true>(map, p, grid, smem, flags, s);
+    return launch_res_t<false, false>(map, p, grid, smem, flags, s);
+}
+
+int read_res_status(unsigned *out, int clear) {
+    unsigned v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_res_status, sizeof(unsigned));
+    if (e == cudaSuccess && clear) {
+        const unsigned zero = 0;
+        e = cudaMemcpyToSymbol(g_res_status, &zero, sizeof(unsigned));
+    }
+    if (e != cudaSuccess)
+        return fail(MNB_ERR_CUDA, "mnb_device_status: %s", cudaGetErrorString(e));
+    *out |= v;   // bit 0, as the other decode kernels
+    return MNB_OK;
+}
+
+}  // namespace mnb

@@ -22,6 +22,12 @@ int launch_gemv(const void *X, int act_f16, const uint8_t *packed, const void *s
 int launch_gemv_tc(const void *X, const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,
                    void *Y, int M, int N, int K, int bs, unsigned flags, cudaStream_t s);
 
+// One-token decode GEMV (fp16 activations and scales) whose CTAs hold their
+// whole share of the weights in shared memory; returns 1 without launching
+// anything for shapes it does not serve.
+int launch_gemv_resident(const void *X, const uint8_t *packed, const void *scales, const uint8_t *zp, void *Y, int N,
+                         int K, int bs, unsigned flags, cudaStream_t s);
+
 // Decode GEMV with the SwiGLU epilogue over gate/up rows interleaved in 8-row groups.
 int launch_gemv_swiglu(const void *X, const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,
                        void *Y, int M, int N, int K, int bs, unsigned flags, cudaStream_t s);
@@ -55,6 +61,7 @@ int launch_gemv_chain(const void *plan, const void *plan_device, void *workspace
 
 int read_device_status(unsigned *out, int clear);
 int read_gemv_status(unsigned *out, int clear);     // ORs the decode kernel's word into *out
+int read_res_status(unsigned *out, int clear);      // same for the one-token resident decode kernel
 int read_chain_status(unsigned *out, int clear);    // the chain kernel's bits, shifted to bits 1-2
 
 }  // namespace mnb

@@ -138,6 +138,57 @@ def test_gemv_parity(mnb, cuda_dev, M, N, K, bs, has_zp, act, sdt):
     assert_close(np_of(Y.float()), ref, act)
 
 
+RESIDENT_CASES = [
+    # N, K, bs, has_zp: the one-token kernel whose CTAs hold their weights in
+    # shared memory (one tile per CTA, tiles cut between warps, several tiles
+    # per CTA, the streamed lm_head shape, ragged N, block 64, no zero points)
+    (2048, 2048, 32, True), (1024, 2048, 32, True), (6144, 2048, 32, True), (2048, 6144, 32, True),
+    (151936, 2048, 32, True), (1000, 1024, 32, True), (3000, 1024, 64, True), (777, 512, 64, False),
+    (50, 256, 32, True), (17, 2048, 32, False), (1, 256, 32, True), (4736, 3072, 64, True),
+]
+
+
+@pytest.mark.parametrize("N,K,bs,has_zp", RESIDENT_CASES)
+def test_gemv_resident_one_token(mnb, cuda_dev, N, K, bs, has_zp):
+    # M = 1 through the resident kernel (the default) and through the general
+    # decode kernel: both against the oracle
+    rng = np.random.default_rng(N + 7 * K)
+    packed, scales, zp = random_packed(rng, N, K, bs, has_zp, np.float16)
+    X = torch.randn((1, K), generator=torch.Generator().manual_seed(N)).half()
+    ref = oracle.matmul(X.float().numpy(), packed, scales, zp, K, bs)
+    for resident in (1, 0):
+        assert mnb._lib.mnb_tune_gemv_resident(resident) == 0
+        try:
+            Y = _run_gemv(mnb, cuda_dev, X.to(cuda_dev), packed, scales, zp, 1, N, K, bs)
+        finally:
+            mnb._lib.mnb_tune_gemv_resident(1)
+        assert_close(np_of(Y.float()), ref, "f16")
+    assert mnb.mnb_device_status() == 0
+
+
+def test_gemv_resident_large_inputs_and_pdl(mnb, cuda_dev):
+    # activations far from unit scale (the raw-code sums grow with |x|), and a
+    # chain of dependent PDL launches: each GEMV reads the previous one's output
+    rng = np.random.default_rng(3)
+    K = 2048
+    # x ~ 50 N(0, 1) meets scales 50x smaller, so every output stays near unit
+    # scale while the first GEMV's raw-code sums are 50x larger than usual
+    ws = [random_packed(rng, K, K, 32, True, np.float16, 0.2 / np.sqrt(K) / (50 if i == 0 else 1),
+                        0.6 / np.sqrt(K) / (50 if i == 0 else 1)) for i in range(4)]
+    x = (torch.randn((1, K), generator=torch.Generator().manual_seed(9)) * 50).half()
+    dev = [tuple(to_dev(a, cuda_dev) for a in w) for w in ws]
+    bufs = [x.to(cuda_dev)] + [torch.full((1, K), float("nan"), dtype=torch.float16, device=cuda_dev) for _ in ws]
+    for i, (p_, s_, z_) in enumerate(dev):
+        mnb.mnb_gemv(bufs[i], p_, s_, z_, bufs[i + 1], 1, K, K, 32, mnb.MNB_FLAG_PDL)
+    torch.cuda.synchronize()
+    cur = x.float().numpy()
+    for i, w in enumerate(ws):
+        ref = oracle.matmul(cur, *w, K, 32)
+        got = np_of(bufs[i + 1].float())
+        assert_close(got, ref, "f16")
+        cur = got   # the next GEMV read the fp16 values this one stored
+
+
 @pytest.mark.parametrize("N,K", [(64, 256), (80, 1024)])
 def test_gemv_q_equal_zp_gives_exact_zero(mnb, cuda_dev, N, K):
     bs, M = 32, 3
