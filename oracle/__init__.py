@@ -22,6 +22,12 @@ Parity status of each function (what pins it, in ``tests/test_oracle.py``):
   embed_gather   pinned: exact power-of-two scales, bad-id rows, table sizes.
   swiglu         pinned: closed forms (silu(0) = 0, silu(1) = 1/(1 + 1/e),
                  silu(x) - silu(-x) = x, the large-|x| limits).
+  gptq_hessian   pinned: exact rational sums on small integer inputs.
+  gptq_prepare   pinned: diagonal Hessians in closed form; U^T U H = I.
+  gptq_quantize  pinned: a diagonal Hessian reduces it to RTN exactly; an
+                 independent formulation (explicit inverse-Hessian downdates,
+                 float64) gives the same codes; lower proxy loss than RTN on
+                 correlated inputs; dead input features give zero weights.
 """
 from __future__ import annotations
 
@@ -49,8 +55,9 @@ def _load():
         lib.orc_dequantize.argtypes = [vp, vp, i32, vp, i64, i64, i64, i32, vp]
         lib.orc_matmul.argtypes = [vp, i64, i64, vp, vp, i32, vp, i64, i64, vp, i64, vp]
         lib.orc_embed_gather.argtypes = [vp, vp, i64, i64, vp, i64, i32, vp]
+        lib.orc_gptq_quantize.argtypes = [vp, vp, vp, i64, i64, i64, i32, i32, vp, vp, vp]
         for f in ("orc_packed_sizes", "orc_quantize_rtn", "orc_dequantize", "orc_matmul",
-                  "orc_embed_gather", "orc_num_threads"):
+                  "orc_embed_gather", "orc_num_threads", "orc_gptq_quantize"):
             getattr(lib, f).restype = i32
         _lib = lib
     return _lib
@@ -159,3 +166,53 @@ def embed_gather(table, row_scales, ids, out_dtype=np.float16):
     st = _load().orc_embed_gather(_ptr(table), _ptr(row_scales), V, D, _ptr(ids), T,
                                   int(np.dtype(out_dtype) == np.float16), _ptr(out))
     return out, st
+
+
+# ---- GPTQ ("Mega-ASR -- INT4 ONNX (GPTQ-calibrated)", "Conversion details" and
+# "GPTQ calibration"; the published GPTQ algorithm, see mnb_oracle.c) --------
+
+def gptq_hessian(X):
+    """H = X^T X over calibration rows X [T, K] (float64, exact products of the
+    given values): the raw sum.  The usual 2/T factor changes no result of the
+    method (U scales by a constant that the error feedback cancels) and is
+    left out."""
+    X = np.asarray(X, np.float64)
+    return X.T @ X
+
+
+def gptq_prepare(H, percdamp=0.01):
+    """(U, dead): dead input features (zero diagonal) get diagonal 1 and are
+    flagged; the diagonal is damped by percdamp times its mean; U is the upper
+    Cholesky factor of the inverse, H^-1 = U^T U.  float64."""
+    H = np.array(H, np.float64, copy=True)
+    K = H.shape[0]
+    d = np.diag(H).copy()
+    dead = d == 0
+    d[dead] = 1.0
+    H[np.arange(K), np.arange(K)] = d
+    damp = percdamp * np.mean(d)
+    H[np.arange(K), np.arange(K)] += damp
+    Hinv = np.linalg.inv(H)
+    U = np.linalg.cholesky(Hinv).T        # lower L with Hinv = L L^T; U = L^T
+    return U, dead.astype(np.uint8)
+
+
+def gptq_quantize(W, U, bs, has_zp=True, scale_dtype=np.float32, dead=None):
+    """GPTQ of fp32 W [N, K] with the fp32 factor U [K, K] (row-major upper):
+    (packed, scales, zp) in the layout of quantize_rtn."""
+    W = _c(W, np.float32)
+    U = _c(U, np.float32)
+    N, K = W.shape
+    if U.shape != (K, K) or K % bs or bs % 2:
+        raise ValueError("bad shape")
+    nb = K // bs
+    packed = np.zeros((N, K // 2), np.uint8)
+    scales = np.zeros((N, nb), scale_dtype)
+    zp = np.zeros((N, (nb + 1) // 2), np.uint8) if has_zp else None
+    dead = None if dead is None else _c(np.asarray(dead, np.uint8), np.uint8)
+    rc = _load().orc_gptq_quantize(_ptr(W), _ptr(U), _ptr(dead), N, K, bs, int(has_zp),
+                                   int(np.dtype(scale_dtype) == np.float16), _ptr(packed), _ptr(scales), _ptr(zp))
+    if rc != 0:
+        raise ValueError("bad shape")
+    return packed, scales, zp
+

@@ -43,9 +43,31 @@
  *      q = clamp(rint(v / scale) + 8, 0, 15); scale == 0 -> q = 8.
  *      PARITY UNPINNED by the pages (they only show is_symmetric=False).
  *   R9 embedding value = fp16_rn( fp32( fp32(int8) * fp32(row_scale) ) ).
+ *
+ * GPTQ ("Mega-ASR -- INT4 ONNX (GPTQ-calibrated)", "Conversion details":
+ * algo=GPTQ, block_size=32, is_symmetric=False; "GPTQ calibration": Hessian
+ * accumulated from calibration activations, Cholesky factorisation of its
+ * inverse, the inner loop run in fp32 on the GPU).  The pages name the method
+ * and do not print it; this is the published algorithm (Frantar et al.,
+ * "GPTQ: Accurate Post-Training Quantization for Generative Pre-trained
+ * Transformers", 2022), column by column without its lazy batching:
+ *     for each row, for i = 0 .. K-1:
+ *         at the first column of a block, the block's scale and zero point
+ *             from the row's CURRENT values of that block (RTN rule above);
+ *         q_i = the RTN code of w_i;  err = (w_i - (q_i - zp) * scale) / U[i][i];
+ *         w_k -= err * U[i][k]  for every k > i,
+ *     with U the upper Cholesky factor of H^-1 (H^-1 = U^T U).
+ *   R10 the block parameters use the weights as updated by every earlier column
+ *       (the lazy-batch implementations read them as of their last batch
+ *       boundary, a scheduling artefact not adopted here).
+ *   R11 codes, scales and zero points follow R1-R8 exactly (the same quantizer
+ *       as RTN), computed from the fp32 scale; fp16 scales are stored rounded
+ *       after the loop (R7).  The loop runs in fp32, the precision of the pages'
+ *       GPU port, one IEEE operation at a time in the order written.
  */
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 #ifdef _OPENMP
 #include <omp.h>
@@ -166,6 +188,93 @@ int orc_quantize_rtn(const float *W, int64_t N, int64_t K, int64_t bs, int has_z
         }
     }
     return ORC_OK;
+}
+
+/* ---- GPTQ quantization (readings R10, R11) -------------------------------- */
+
+/* W: fp32 [N][K] (read only).  U: fp32 [K][K], row-major upper Cholesky factor
+ * of the (damped) inverse Hessian; only U[i][k] with k >= i is read.  dead:
+ * K flags or NULL; a dead input feature's weights are zeroed before the loop.
+ * Outputs as orc_quantize_rtn. */
+int orc_gptq_quantize(const float *W, const float *U, const uint8_t *dead, int64_t N, int64_t K, int64_t bs,
+                      int has_zp, int scale_f16, uint8_t *packed, void *scales, uint8_t *zp)
+{
+    if (N < 0 || K <= 0 || bs <= 0 || K % bs != 0 || bs % 2 != 0)
+        return ORC_BAD;
+    int64_t nb = K / bs;
+    int64_t zp_row = (nb + 1) / 2;
+    memset(packed, 0, (size_t)(N * (K / 2)));
+    if (has_zp)
+        memset(zp, 0, (size_t)(N * zp_row));
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int64_t n = 0; n < N; n++) {
+        float *w = (float *)malloc((size_t)K * sizeof(float));
+        if (!w) {
+            bad = 1;
+            continue;
+        }
+        for (int64_t k = 0; k < K; k++)
+            w[k] = (dead && dead[k]) ? 0.0f : W[n * K + k];
+        uint8_t *prow = packed + n * (K / 2);
+        float s = 0.0f;
+        int z = 0;
+        for (int64_t i = 0; i < K; i++) {
+            if (i % bs == 0) {
+                /* the block's parameters from its current values */
+                int64_t b = i / bs;
+                const float *v = w + i;
+                if (has_zp) {
+                    float lo = 0.0f, hi = 0.0f;   /* R3 */
+                    for (int64_t j = 0; j < bs; j++) {
+                        if (v[j] < lo)
+                            lo = v[j];
+                        if (v[j] > hi)
+                            hi = v[j];
+                    }
+                    s = (hi - lo) / 15.0f;
+                    z = 0;
+                    if (s != 0.0f)
+                        z = clamp_0_15((int)rintf(-lo / s));
+                    nibble_set(zp + n * zp_row, b, z);
+                } else {
+                    float amax = 0.0f;   /* R8 */
+                    for (int64_t j = 0; j < bs; j++) {
+                        float a = fabsf(v[j]);
+                        if (a > amax)
+                            amax = a;
+                    }
+                    s = amax / 7.0f;
+                    z = 8;
+                }
+                if (scale_f16)
+                    ((_Float16 *)scales)[n * nb + b] = (_Float16)s;
+                else
+                    ((float *)scales)[n * nb + b] = s;
+            }
+            int q;
+            if (has_zp) {
+                q = 0;
+                if (s != 0.0f) {
+                    float t = w[i] / s;   /* R5 */
+                    t = t + (float)z;
+                    q = clamp_0_15((int)rintf(t));
+                }
+            } else {
+                q = 8;
+                if (s != 0.0f)
+                    q = clamp_0_15((int)rintf(w[i] / s) + 8);
+            }
+            nibble_set(prow, i, q);
+            /* error feedback through row i of U */
+            float dq = (float)(q - z) * s;
+            float err = (w[i] - dq) / U[i * K + i];
+            for (int64_t k = i + 1; k < K; k++)
+                w[k] = w[k] - err * U[i * K + k];
+        }
+        free(w);
+    }
+    return bad ? ORC_BAD : ORC_OK;
 }
 
 /* ---- dequantization --------------------------------------------------------- */

@@ -395,3 +395,144 @@ def test_swiglu_closed_forms():
     assert abs(s[5] - 40.0) < 1e-15 and abs(s[6]) < 1e-15
     # the up factor multiplies
     assert np.allclose(oracle.swiglu(x, 3.0 * ones), 3.0 * s, rtol=1e-15, atol=0)
+
+
+# ---- GPTQ ("Mega-ASR -- INT4 ONNX (GPTQ-calibrated)", "Conversion details":
+# algo=GPTQ; "GPTQ calibration") -------------------------------------------------
+
+def _codes(packed, K):
+    """Unpacked 4-bit codes [N, K] (low nibble first)."""
+    p = np.asarray(packed, np.uint8)
+    out = np.empty((p.shape[0], K), np.int64)
+    out[:, 0::2] = p & 15
+    out[:, 1::2] = p >> 4
+    return out
+
+
+def test_gptq_hessian_is_the_exact_gram_matrix():
+    rng = np.random.default_rng(0)
+    X = rng.integers(-7, 8, (9, 6)).astype(np.float64)
+    H = oracle.gptq_hessian(X)
+    ref = [[sum(int(X[t, i]) * int(X[t, j]) for t in range(9)) for j in range(6)] for i in range(6)]
+    assert np.array_equal(H, np.array(ref, np.float64))
+
+
+def test_gptq_prepare_diagonal_closed_form():
+    d = np.array([4.0, 0.0, 9.0, 2.25])            # feature 1 never active: dead
+    U, dead = oracle.gptq_prepare(np.diag(d), percdamp=0.01)
+    dd = np.array([4.0, 1.0, 9.0, 2.25])
+    damp = 0.01 * dd.mean()
+    assert np.array_equal(dead, [0, 1, 0, 0])
+    assert np.allclose(U, np.diag(1.0 / np.sqrt(dd + damp)), rtol=1e-15, atol=0)
+
+
+def test_gptq_prepare_factor_inverts_the_damped_hessian():
+    rng = np.random.default_rng(1)
+    X = rng.standard_normal((200, 48)) @ rng.standard_normal((48, 48))
+    H = oracle.gptq_hessian(X)
+    U, dead = oracle.gptq_prepare(H, percdamp=0.05)
+    assert not dead.any()
+    Hd = H + 0.05 * np.mean(np.diag(H)) * np.eye(48)
+    assert np.allclose(np.triu(U), U) and np.all(np.diag(U) > 0)     # upper, positive diagonal
+    assert np.allclose(U.T @ U @ Hd, np.eye(48), atol=1e-9)          # U^T U = Hd^-1
+
+
+@pytest.mark.parametrize("bs,has_zp,sdt", [(32, True, np.float16), (64, True, np.float32),
+                                           (32, False, np.float16), (64, False, np.float32)])
+def test_gptq_with_a_diagonal_hessian_is_rtn(bs, has_zp, sdt):
+    # uncorrelated inputs: U is diagonal, no error flows to later columns, and
+    # every block is quantized from its original values -- exactly RTN
+    rng = np.random.default_rng(bs + has_zp)
+    K, N = 4 * bs, 7
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    U, dead = oracle.gptq_prepare(np.diag(rng.uniform(0.5, 3.0, K)))
+    g = oracle.gptq_quantize(W, U.astype(np.float32), bs, has_zp, sdt, dead)
+    r = oracle.quantize_rtn(W, bs, has_zp, sdt)
+    assert np.array_equal(g[0], r[0])
+    assert np.array_equal(g[1].view(np.uint8), r[1].view(np.uint8))
+    if has_zp:
+        assert np.array_equal(g[2], r[2])
+
+
+def _gptq_by_downdates(W, H, bs, has_zp, percdamp=0.01):
+    """GPTQ written independently of the oracle: float64, with the explicit
+    inverse Hessian of the not-yet-quantized columns, downdated after each
+    column (w_F -= (w_i - q_i) H_F^-1[i, F] / H_F^-1[i, i]); the quantizer's
+    decisions in float32 as the method's.  Returns the codes [N, K]."""
+    K = H.shape[0]
+    Hd = np.array(H, np.float64)
+    d = np.diag(Hd).copy()
+    d[d == 0] = 1.0
+    Hd[np.arange(K), np.arange(K)] = d + percdamp * d.mean()
+    Hinv = np.linalg.inv(Hd)
+    coef = np.zeros((K, K))
+    for i in range(K):
+        coef[i, i + 1:] = Hinv[i, i + 1:] / Hinv[i, i]
+        Hinv = Hinv - np.outer(Hinv[:, i], Hinv[i, :]) / Hinv[i, i]
+    f32 = np.float32
+    codes = np.zeros(W.shape, np.int64)
+    for n in range(W.shape[0]):
+        w = W[n].astype(np.float64)
+        for i in range(K):
+            if i % bs == 0:
+                v = w[i:i + bs].astype(f32)
+                if has_zp:
+                    lo, hi = min(f32(0), v.min()), max(f32(0), v.max())
+                    s = f32(f32(hi - lo) / f32(15))
+                    z = int(np.clip(np.rint(f32(-lo) / s), 0, 15)) if s != 0 else 0
+                else:
+                    s = f32(np.abs(v).max() / f32(7))
+                    z = 8
+            wi = f32(w[i])
+            if s == 0:
+                q = 0 if has_zp else 8
+            elif has_zp:
+                q = int(np.clip(np.rint(f32(f32(wi / s) + f32(z))), 0, 15))
+            else:
+                q = int(np.clip(np.rint(f32(wi / s)) + 8, 0, 15))
+            codes[n, i] = q
+            w[i + 1:] -= (w[i] - (q - z) * float(s)) * coef[i, i + 1:]
+    return codes
+
+
+@pytest.mark.parametrize("seed,bs,has_zp", [(0, 32, True), (1, 64, True), (2, 32, False), (3, 32, True)])
+def test_gptq_matches_an_independent_formulation(seed, bs, has_zp):
+    rng = np.random.default_rng(seed)
+    K, N = 3 * bs, 6
+    X = rng.standard_normal((400, K)) @ rng.standard_normal((K, K)) * 0.3 + rng.standard_normal((400, K))
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    H = oracle.gptq_hessian(X)
+    U, dead = oracle.gptq_prepare(H)
+    packed, _, _ = oracle.gptq_quantize(W, U.astype(np.float32), bs, has_zp, np.float32, dead)
+    assert np.array_equal(_codes(packed, K), _gptq_by_downdates(W, H, bs, has_zp))
+
+
+def test_gptq_lowers_the_proxy_loss_below_rtn():
+    # correlated calibration inputs: GPTQ's error feedback must beat plain
+    # rounding on ||(W - W^) X^T||^2, the loss it minimizes
+    rng = np.random.default_rng(7)
+    K, N, bs = 128, 32, 32
+    X = rng.standard_normal((1024, K)) @ rng.standard_normal((K, K))
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    U, dead = oracle.gptq_prepare(oracle.gptq_hessian(X))
+    g = oracle.gptq_quantize(W, U.astype(np.float32), bs, True, np.float32, dead)
+    r = oracle.quantize_rtn(W, bs, True, np.float32)
+
+    def loss(q):
+        Wq = oracle.dequantize(q[0], q[1], q[2], K, bs)
+        return float(np.sum(((W.astype(np.float64) - Wq) @ X.T) ** 2))
+
+    assert loss(g) < 0.8 * loss(r)
+
+
+def test_gptq_dead_features_get_zero_weights():
+    rng = np.random.default_rng(8)
+    K, N, bs = 64, 5, 32
+    X = rng.standard_normal((300, K))
+    X[:, [3, 40]] = 0.0                      # two input features never active
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    U, dead = oracle.gptq_prepare(oracle.gptq_hessian(X))
+    assert dead[3] == 1 and dead[40] == 1 and dead.sum() == 2
+    p, s, z = oracle.gptq_quantize(W, U.astype(np.float32), bs, True, np.float32, dead)
+    Wq = oracle.dequantize(p, s, z, K, bs)
+    assert np.all(Wq[:, [3, 40]] == 0.0)
