@@ -301,6 +301,56 @@ MNB_API int mnb_gemv_chain_plan(const mnb_gemv_task *tasks, int ntasks, int64_t 
 MNB_API int mnb_gemv_chain(const void *plan, const void *plan_device, void *workspace, size_t ws_bytes,
                            unsigned flags, void *stream);
 
+/* ---- GPTQ quantization into the packed layout -----------------------------
+ * "Mega-ASR -- INT4 ONNX (GPTQ-calibrated)", "Conversion details" (algo=GPTQ,
+ * block_size=32, is_symmetric=False, bits=4) and "GPTQ calibration" (the
+ * Hessian accumulated from calibration activations, a Cholesky factorisation
+ * of its inverse, the inner loop in fp32 on the GPU, a diagonal-jitter retry
+ * when the fp32 factorisation fails).  The algorithm is the published GPTQ;
+ * the three calls below are its three stages.  Their outputs feed every
+ * MatMulNBits entry point above unchanged. */
+
+/* H (+)= X^T X: H fp32 [K][K] (row-major, full), X [T][K] fp32 or fp16
+ * calibration inputs (the activations the weight meets).  accumulate = 0
+ * overwrites H, 1 adds to it (several calibration batches).  The usual 2/T
+ * factor is left out: no result of the method depends on it.  fp32
+ * accumulation.  1 <= K <= 8192.
+ * Errors: MNB_ERR_INVALID_ARG, MNB_ERR_SHAPE, MNB_ERR_ALIGN, MNB_ERR_CUDA. */
+MNB_API int mnb_gptq_hessian(const void *X, mnb_dtype x_t, int64_t T, int64_t K, float *H, int accumulate,
+                             void *stream);
+
+/* Bytes of the workspace of mnb_gptq_prepare (0 when K is outside [1, 8192]). */
+MNB_API size_t mnb_gptq_workspace_bytes(int64_t K);
+
+/* From H (read only): dead[k] = 1 where H_kk == 0 (a feature the calibration
+ * never activated: its diagonal becomes 1 and mnb_gptq_quantize zeroes its
+ * weights), the diagonal damped by percdamp x its mean (0.01 is usual), and
+ * U fp32 [K][K] = the upper Cholesky factor of the damped H^-1 (H^-1 = U^T U,
+ * zeros below the diagonal).  If the fp32 factorisation meets a non-positive
+ * pivot it starts again with 10x the damping (0.001 after percdamp = 0), up
+ * to three times; *damp_used
+ * (host pointer, may be NULL) receives the damping that succeeded.  HOST-
+ * BLOCKING: synchronizes `stream` once per attempt.  workspace: device memory
+ * of mnb_gptq_workspace_bytes(K) bytes, 16-byte aligned, any contents.
+ * Errors: MNB_ERR_INVALID_ARG (also: no attempt succeeded), MNB_ERR_SHAPE,
+ *         MNB_ERR_ALIGN, MNB_ERR_CUDA. */
+MNB_API int mnb_gptq_prepare(const float *H, int64_t K, float percdamp, float *U, uint8_t *dead, void *workspace,
+                             size_t ws_bytes, float *damp_used, void *stream);
+
+/* GPTQ of fp32 W [N][K] (read only) with U from mnb_gptq_prepare and its dead
+ * flags (dead may be NULL: none).  Per row, column by column: a block's scale
+ * and zero point come from the row's current values of the block (the RTN
+ * rule of mnb_quantize_rtn, same has_zp variants), the code is the RTN code,
+ * and the rounding error err = (w_i - (q_i - zp) * scale) / U_ii is fed back:
+ * w_k -= err * U_ik for k > i.  Every step is one fp32 operation in that
+ * order, so the codes do not depend on the launch shape.  Writes packed,
+ * scales (fp16_rn of the fp32 scale when scale_t is MNB_F16) and zp in the
+ * layout above.  K <= 8192, K % bs == 0.
+ * Errors: MNB_ERR_INVALID_ARG, MNB_ERR_SHAPE, MNB_ERR_ALIGN, MNB_ERR_CUDA. */
+MNB_API int mnb_gptq_quantize(const float *W, const float *U, const uint8_t *dead, int64_t N, int64_t K, int bs,
+                              int has_zp, uint8_t *packed, void *scales, mnb_dtype scale_t, uint8_t *zp,
+                              void *stream);
+
 /* Reads (and, if clear != 0, zeroes) the library's device status word on the
  * current device into *status_out: bit 0 = a GEMM or GEMV mbarrier wait timed
  * out; bits 1-3 = mnb_gemv_chain (see there).  Synchronizes the device.

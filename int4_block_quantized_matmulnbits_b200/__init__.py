@@ -24,7 +24,8 @@ __all__ = [
     "mnb_gemv", "mnb_gemm", "mnb_embed_gather", "mnb_device_status",
     "mnb_gemv_argmax", "mnb_gemv_argmax_workspace_bytes", "mnb_gemv_argmax_noalloc", "mnb_gemv_swiglu",
     "mnb_gemv_task", "mnb_gemv_chain_plan_bytes", "mnb_gemv_chain_workspace_bytes", "mnb_gemv_chain_plan",
-    "mnb_gemv_chain", "mnb_matmul",
+    "mnb_gemv_chain", "mnb_matmul", "mnb_gptq_hessian", "mnb_gptq_workspace_bytes", "mnb_gptq_prepare",
+    "mnb_gptq_quantize",
 ]
 
 MNB_F32, MNB_F16 = 0, 1
@@ -77,6 +78,10 @@ def _load():
         "mnb_gemv_chain_workspace_bytes": ([i32], sz),
         "mnb_gemv_chain_plan": ([P(mnb_gemv_task), i32, i64, i32, vp, sz], i32),
         "mnb_gemv_chain": ([vp, vp, vp, sz, u32, vp], i32),
+        "mnb_gptq_hessian": ([vp, i32, i64, i64, vp, i32, vp], i32),
+        "mnb_gptq_workspace_bytes": ([i64], sz),
+        "mnb_gptq_prepare": ([vp, i64, ctypes.c_float, vp, vp, vp, sz, P(ctypes.c_float), vp], i32),
+        "mnb_gptq_quantize": ([vp, vp, vp, i64, i64, i32, i32, vp, vp, i32, vp, vp], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -251,3 +256,34 @@ def mnb_device_status(clear=False) -> int:
     if rc != -6:
         _check("mnb_device_status", rc)
     return v.value
+
+
+def mnb_gptq_hessian(X, H, accumulate=False, stream=None):
+    """H [K, K] fp32 (+)= X^T X for calibration inputs X [T, K] (fp32 or fp16)."""
+    T, K = X.shape
+    _check("mnb_gptq_hessian", _lib.mnb_gptq_hessian(_ptr(X), _dt(X), T, K, _ptr(H), int(bool(accumulate)),
+                                                     _stream(stream)))
+
+
+def mnb_gptq_workspace_bytes(K) -> int:
+    return _lib.mnb_gptq_workspace_bytes(K)
+
+
+def mnb_gptq_prepare(H, U, dead, workspace, percdamp=0.01, stream=None) -> float:
+    """U [K, K] fp32 = upper Cholesky factor of the damped H^-1; dead [K] uint8.
+    Synchronizes the stream; returns the damping that succeeded."""
+    K = H.shape[0]
+    d = ctypes.c_float()
+    _check("mnb_gptq_prepare", _lib.mnb_gptq_prepare(
+        _ptr(H), K, percdamp, _ptr(U), _ptr(dead), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        ctypes.byref(d), _stream(stream)))
+    return d.value
+
+
+def mnb_gptq_quantize(W, U, dead, bs, has_zp, packed, scales, zp, stream=None):
+    """GPTQ of fp32 W [N, K] into packed / scales / zp (the layout of mnb_quantize_rtn)."""
+    N, K = W.shape
+    _check("mnb_gptq_quantize", _lib.mnb_gptq_quantize(
+        _ptr(W), _ptr(U), _ptr(dead), N, K, bs, int(bool(has_zp)), _ptr(packed), _ptr(scales), _dt(scales),
+        _ptr(zp), _stream(stream)))
+

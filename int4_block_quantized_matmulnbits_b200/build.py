@@ -22,7 +22,7 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-Xptxas", "-warn-spills", "-I", os.path.join(ROOT, "include")]
-SOURCES = ["api.cu", "quantize.cu", "gemv.cu", "gemv_tc.cu", "gemv_resident.cu", "gemv_chain.cu", "gemm_tcgen05.cu", "embed.cu"]
+SOURCES = ["api.cu", "quantize.cu", "gemv.cu", "gemv_tc.cu", "gemv_resident.cu", "gemv_chain.cu", "gemm_tcgen05.cu", "embed.cu", "gptq.cu"]
 HEADERS = ["common.cuh", "internal.h"]
 
 

@@ -399,6 +399,69 @@ int mnb_gemv_chain(const void *plan, const void *plan_device, void *workspace, s
     return launch_gemv_chain(plan, plan_device, workspace, ws_bytes, flags, (cudaStream_t)stream);
 }
 
+static const int64_t kGptqMaxK = 8192;
+
+int mnb_gptq_hessian(const void *X, mnb_dtype x_t, int64_t T, int64_t K, float *H, int accumulate, void *stream) {
+    clear_error();
+    const char *fn = "mnb_gptq_hessian";
+    int rc;
+    if ((rc = check_dtype(fn, "input", x_t)))
+        return rc;
+    if (T < 0 || K < 1 || K > kGptqMaxK)
+        return fail(MNB_ERR_SHAPE, "%s: T=%lld, K=%lld (K must be in [1, %lld])", fn, (long long)T, (long long)K,
+                    (long long)kGptqMaxK);
+    if (T > kMaxDim)
+        return fail(MNB_ERR_SHAPE, "%s: T above 2^30", fn);
+    if (!H || (T > 0 && !X))
+        return fail(MNB_ERR_INVALID_ARG, "%s: NULL X or H", fn);
+    if (!aligned(H, 4) || !aligned(X, x_t == MNB_F32 ? 4 : 2))
+        return fail(MNB_ERR_ALIGN, "%s: X and H need their element alignment", fn);
+    return launch_gptq_hessian(X, x_t == MNB_F16, T, K, H, accumulate ? 1 : 0, (cudaStream_t)stream);
+}
+
+size_t mnb_gptq_workspace_bytes(int64_t K) {
+    if (K < 1 || K > kGptqMaxK)
+        return 0;
+    return gptq_workspace_bytes(K);
+}
+
+int mnb_gptq_prepare(const float *H, int64_t K, float percdamp, float *U, uint8_t *dead, void *workspace,
+                     size_t ws_bytes, float *damp_used, void *stream) {
+    clear_error();
+    const char *fn = "mnb_gptq_prepare";
+    if (K < 1 || K > kGptqMaxK)
+        return fail(MNB_ERR_SHAPE, "%s: K=%lld outside [1, %lld]", fn, (long long)K, (long long)kGptqMaxK);
+    if (!H || !U || !dead || !workspace)
+        return fail(MNB_ERR_INVALID_ARG, "%s: NULL H, U, dead or workspace", fn);
+    if (!(percdamp >= 0.f) || !(percdamp <= 1.f))
+        return fail(MNB_ERR_INVALID_ARG, "%s: percdamp %g outside [0, 1]", fn, (double)percdamp);
+    if (!aligned(H, 4) || !aligned(U, 4) || !aligned(workspace, 16))
+        return fail(MNB_ERR_ALIGN, "%s: H and U need 4-byte, the workspace 16-byte alignment", fn);
+    if (ws_bytes < gptq_workspace_bytes(K))
+        return fail(MNB_ERR_INVALID_ARG, "%s: workspace of %zu bytes, %zu needed", fn, ws_bytes,
+                    gptq_workspace_bytes(K));
+    return launch_gptq_prepare(H, K, percdamp, U, dead, workspace, damp_used, (cudaStream_t)stream);
+}
+
+int mnb_gptq_quantize(const float *W, const float *U, const uint8_t *dead, int64_t N, int64_t K, int bs, int has_zp,
+                      uint8_t *packed, void *scales, mnb_dtype scale_t, uint8_t *zp, void *stream) {
+    clear_error();
+    const char *fn = "mnb_gptq_quantize";
+    int rc;
+    if ((rc = check_dtype(fn, "scale", scale_t)) || (rc = check_weight_shape(fn, N, K, bs)))
+        return rc;
+    if (K > kGptqMaxK)
+        return fail(MNB_ERR_SHAPE, "%s: K=%lld above %lld", fn, (long long)K, (long long)kGptqMaxK);
+    if (N == 0)
+        return MNB_OK;
+    if (!W || !U || !packed || !scales || (has_zp && !zp))
+        return fail(MNB_ERR_INVALID_ARG, "%s: NULL pointer", fn);
+    if (!aligned(W, 4) || !aligned(U, 4) || !aligned(scales, scale_t == MNB_F32 ? 4 : 2))
+        return fail(MNB_ERR_ALIGN, "%s: W, U and scales need their element alignment", fn);
+    return launch_gptq_quantize(W, U, dead, N, K, bs, has_zp ? 1 : 0, packed, scales, scale_t == MNB_F16,
+                                has_zp ? zp : nullptr, (cudaStream_t)stream);
+}
+
 int mnb_device_status(unsigned *status_out, int clear) {
     clear_error();
     if (!status_out)

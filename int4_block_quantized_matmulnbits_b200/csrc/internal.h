@@ -59,6 +59,14 @@ int gemv_chain_plan(const mnb_gemv_task *tasks, int ntasks, int M, int bs, void 
 int launch_gemv_chain(const void *plan, const void *plan_device, void *workspace, size_t ws_bytes, unsigned flags,
                       cudaStream_t s);
 
+// GPTQ into the packed layout.
+size_t gptq_workspace_bytes(int64_t K);
+int launch_gptq_hessian(const void *X, int x_f16, int64_t T, int64_t K, float *H, int accumulate, cudaStream_t s);
+int launch_gptq_prepare(const float *H, int64_t K, float percdamp, float *U, uint8_t *dead, void *workspace,
+                        float *damp_used, cudaStream_t s);
+int launch_gptq_quantize(const float *W, const float *U, const uint8_t *dead, int64_t N, int64_t K, int bs,
+                         int has_zp, uint8_t *packed, void *scales, int scale_f16, uint8_t *zp, cudaStream_t s);
+
 int read_device_status(unsigned *out, int clear);
 int read_gemv_status(unsigned *out, int clear);     // ORs the decode kernel's word into *out
 int read_res_status(unsigned *out, int clear);      // same for the one-token resident decode kernel

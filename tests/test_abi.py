@@ -219,3 +219,31 @@ def test_matmul_argument_checks(lib):
     assert f(A, F16, A, A, F16, A, A, 17, 128, 64, 32, 0x80, None) == INVALID   # unknown flag
     assert f(A, 7, A, A, F16, A, A, 17, 128, 64, 32, 0, None) == INVALID        # dtype
     assert f(A, F16, A, A, F16, A, A, 0, 128, 64, 32, 0, None) == OK            # M = 0: nothing to do
+
+
+def test_gptq_argument_checks(lib):
+    vp = ctypes.c_void_p
+    h = lib.mnb_gptq_hessian
+    h.argtypes = [vp, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, vp, ctypes.c_int, vp]
+    assert h(A, F32, 10, 0, A, 0, None) == SHAPE                 # K = 0
+    assert h(A, F32, 10, 8193, A, 0, None) == SHAPE              # K above the limit
+    assert h(None, F32, 10, 64, A, 0, None) == INVALID
+    assert h(A, F32, 10, 64, A + 2, 0, None) == ALIGN
+    assert h(A, 7, 10, 64, A, 0, None) == INVALID                # dtype
+    wsb = lib.mnb_gptq_workspace_bytes
+    wsb.argtypes, wsb.restype = [ctypes.c_int64], ctypes.c_size_t
+    assert wsb(0) == 0 and wsb(8193) == 0 and wsb(64) >= 2 * 64 * 64 * 4
+    p = lib.mnb_gptq_prepare
+    p.argtypes = [vp, ctypes.c_int64, ctypes.c_float, vp, vp, vp, ctypes.c_size_t, vp, vp]
+    need = wsb(64)
+    assert p(A, 64, 0.01, A, A, A, need - 1, None, None) == INVALID   # workspace too small
+    assert p(A, 64, -1.0, A, A, A, need, None, None) == INVALID       # percdamp
+    assert p(A, 64, 0.01, A, None, A, need, None, None) == INVALID
+    assert p(A, 64, 0.01, A, A, A + 4, need, None, None) == ALIGN
+    q = lib.mnb_gptq_quantize
+    q.argtypes = [vp, vp, vp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_int, vp, vp, ctypes.c_int,
+                  vp, vp]
+    assert q(A, A, None, 4, 96, 64, 1, A, A, F16, A, None) == SHAPE    # K % bs
+    assert q(A, A, None, 4, 96, 48, 1, A, A, F16, A, None) == SHAPE    # bs
+    assert q(A, A, None, 4, 64, 32, 1, A, A, F16, None, None) == INVALID   # zp missing
+    assert q(A, A, None, 0, 64, 32, 1, A, A, F16, A, None) == OK       # nothing to do
