@@ -541,6 +541,69 @@ def bench_embed(dev, ranks, hbm, with_oracle):
     return out
 
 
+def bench_gptq(dev, ranks, with_oracle):
+    """GPTQ of the 1.7B decoder's layer-0 q projection (N = K = 2048) from 2048
+    calibration tokens (synthetic, correlated fp16 activations): device time
+    of each stage (CUDA events; the factorisation synchronizes its stream once)."""
+    import numpy as np
+    import torch
+
+    import int4_block_quantized_matmulnbits_b200 as mnb
+    import workloads
+
+    cfg = workloads.CONFIGS["qwen3_1p7b_decode"]
+    N = K = 2048
+    T, bs = 2048, cfg["bs"]
+    g = torch.Generator(device="cpu").manual_seed(cfg["seed"] * 1_000_003 + 4242)
+    mix = torch.eye(K) + torch.randn((K, K), generator=g) / K ** 0.5
+    X = (torch.randn((T, K), generator=g) @ mix).half().to(dev)
+    W = workloads.weight(cfg["seed"], 0, 0, N, K, True, device=dev)
+    H = torch.empty((K, K), dtype=torch.float32, device=dev)
+    U = torch.empty((K, K), dtype=torch.float32, device=dev)
+    dead = torch.empty((K,), dtype=torch.uint8, device=dev)
+    ws = torch.empty((mnb.mnb_gptq_workspace_bytes(K),), dtype=torch.uint8, device=dev)
+    packed = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((N, K // bs), dtype=torch.float16, device=dev)
+    zp = torch.empty((N, K // bs // 2), dtype=torch.uint8, device=dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    times = []
+    for rep in range(4):   # the first is warm-up
+        torch.cuda.synchronize()
+        ev[0].record()
+        mnb.mnb_gptq_hessian(X, H)
+        ev[1].record()
+        mnb.mnb_gptq_prepare(H, U, dead, ws, 0.01)
+        ev[2].record()
+        mnb.mnb_gptq_quantize(W, U, dead, bs, True, packed, scales, zp)
+        ev[3].record()
+        torch.cuda.synchronize()
+        if rep:
+            times.append([ev[i].elapsed_time(ev[i + 1]) for i in range(3)])
+    t = np.median(np.array(times), axis=0)
+    out = {"projection": "q of layer 0, N = K = 2048, block 32, zero points, fp16 scales", "calib_tokens": T,
+           "hessian_ms": round(float(t[0]), 3), "prepare_ms": round(float(t[1]), 3),
+           "quantize_ms": round(float(t[2]), 3), "total_ms": round(float(t.sum()), 3),
+           "weights_per_s": round(N * K / (float(t.sum()) * 1e-3), 1)}
+    if with_oracle:
+        import oracle
+
+        Xn = X.float().cpu().numpy()
+        Wn = W.cpu().numpy()
+        t0 = time.perf_counter()
+        Hn = oracle.gptq_hessian(Xn)
+        Un, deadn = oracle.gptq_prepare(Hn)
+        t1 = time.perf_counter()
+        rows = 128
+        oracle.gptq_quantize(Wn[:rows], Un.astype(np.float32), bs, True, np.float16, deadn)
+        t2 = time.perf_counter()
+        total = (t1 - t0) + (t2 - t1) * N / rows
+        out["cpu_oracle"] = {"total_s": round(total, 3), "weights_per_s": round(N * K / total, 1),
+                             "cores": oracle.num_threads(),
+                             "sample": f"Hessian and factor in full (numpy float64), the column loop on {rows} of "
+                                       f"{N} rows, scaled to all rows"}
+    return out
+
+
 def run_gpu(args, world, rank, local):
     import torch
 
@@ -768,6 +831,8 @@ def run_gpu(args, world, rank, local):
                 for v in ("qwen3_0p6b_bs64", "qwen3_0p6b_nozp")}
     embed = bench_embed(dev, ranks, hbm, with_oracle)
     torch.cuda.empty_cache()
+    gptq = bench_gptq(dev, ranks, with_oracle)
+    torch.cuda.empty_cache()
     assert mnb.mnb_device_status() == 0, "a GEMM wait timed out"
 
     cpu = None
@@ -821,6 +886,7 @@ def run_gpu(args, world, rank, local):
             "decode_step_qwen3_0p6b": step06,
             "layout_variants": variants,
             "embed_gather": embed,
+            "gptq": gptq,
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_val, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},

@@ -398,6 +398,8 @@ static int plan_gemv(int M, int N, int K, int MP, int sms, Params &p, int &grid,
 // One-token fp16 calls go to the resident kernel (1) or the general one (0).
 static int g_resident = 1;
 
+int gemv_resident_enabled() { return g_resident; }
+
 int launch_gemv(const void *X, int act_f16, const uint8_t *packed, const void *scales,
                 int scale_f16, const uint8_t *zp, void *Y, int M, int N, int K, int bs,
                 unsigned flags, cudaStream_t s) {

@@ -35,6 +35,9 @@
 //     sum_k (q - zp) x = D - zp Q, Q = sum_k x (both sums per block of x,
 //     computed once per call), and y += scale * (D - zp Q).  Four correction
 //     FMAs per thread per box replace two half2 operations per weight pair.
+//     The 16 MMAs of a box run as four independent accumulator chains: on
+//     the decoder's small projections each warp holds one to three boxes, so
+//     the latency of a chain, not the issue rate, sets the kernel's time.
 // Every mbarrier wait is bounded in time; past the limit the kernel records
 // the failure in the device status word, lets its copies in flight land and
 // exits.
@@ -69,7 +72,24 @@ struct ResParams {
     int ntiles, nbx, nchunks; // ceil(N / 16), K / 256, K / 32
     int tq, tr;               // tiles per CTA: tq, one more for CTAs below tr
     int depth;                // ring slots per warp
+    // greedy decoding: ids[0] = the first n of max y[n] (over the fp16 values
+    // stored), max_out[0] its value; per-CTA partials in a caller workspace,
+    // reduced by the last CTA to finish (counter in the workspace's header)
+    int argmax;
+    int32_t *ids;
+    float *max_out;
+    uint2 *ws_part;           // [gridDim.x] (value bits, index)
+    unsigned *ws_count;
 };
+
+// (value, index) pairs ordered by value, then by the SMALLER index: the greedy
+// token is the first maximum.
+__device__ __forceinline__ void keep_best(float v, int i, float &bv, int &bi) {
+    if (v > bv || (v == bv && i < bi)) {
+        bv = v;
+        bi = i;
+    }
+}
 
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -175,7 +195,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     float2 *pq = reinterpret_cast<float2 *>(zchunk + kChunk);
     float *part = reinterpret_cast<float *>(pq + p.nchunks);      // [warp][2 slots][16 rows]
     int *part_tile = reinterpret_cast<int *>(part + kWarps * 2 * kRows);
-    const uint32_t bars = smem_u32(part_tile + kWarps * 2);
+    uint2 *wbest = reinterpret_cast<uint2 *>(part_tile + kWarps * 2);   // greedy decoding: per warp
+    const uint32_t bars = smem_u32(wbest + kWarps);
     const uint32_t my_box = base + (uint32_t)(warp * D * kBoxBytes);
     const unsigned char *my_box_ptr = bp + warp * D * kBoxBytes;
     const uint32_t my_par = smem_u32(pars) + (uint32_t)(warp * D * kParBytes);
@@ -215,30 +236,31 @@ __global__ void __launch_bounds__(kThreads, 2)
     // ---- stage x: chunk j (k = 32j .. 32j+31) as four 16-byte words, word w =
     // (x0,x4) (x1,x5)/16 (x2,x6) (x3,x7)/16 of k = 32j + 8w ..; and per chunk
     // P = 1024 sum x~ and Q = sum x over the staged values x~ (x/16 counted
-    // back as 16 x~), so the correction matches the MMA's operands exactly
+    // back as 16 x~), so the correction matches the MMA's operands exactly.
+    // One 16-byte word per thread per pass (K / 8 is a multiple of 32, so every
+    // lane of a warp takes part in each pass); the four words of a chunk sit in
+    // four consecutive lanes, which add their sums by shuffles.
     {
         const half2 sixteenth = __floats2half2_rn(0.0625f, 0.0625f);
-        for (int j = tid; j < p.nchunks; j += kThreads) {
-            uint4 vv[4];
-#pragma unroll
-            for (int w = 0; w < 4; w++)
-                vv[w] = ldg_v4(p.X + j * 32 + 8 * w);
-            float lo = 0.f, hi = 0.f;   // sum of the low-position x, of the high-position x~
-#pragma unroll
-            for (int w = 0; w < 4; w++) {
-                const uint4 v = vv[w];
-                uint4 o;
-                o.x = __byte_perm(v.x, v.z, 0x5410);
-                o.y = h2_as_u32(__hmul2(u32_as_h2(__byte_perm(v.x, v.z, 0x7632)), sixteenth));
-                o.z = __byte_perm(v.y, v.w, 0x5410);
-                o.w = h2_as_u32(__hmul2(u32_as_h2(__byte_perm(v.y, v.w, 0x7632)), sixteenth));
-                *reinterpret_cast<uint4 *>(xs + j * kChunk + w * 16) = o;
-                const float2 a = __half22float2(u32_as_h2(o.x)), b = __half22float2(u32_as_h2(o.y));
-                const float2 e = __half22float2(u32_as_h2(o.z)), f = __half22float2(u32_as_h2(o.w));
-                lo += (a.x + a.y) + (e.x + e.y);
-                hi += (b.x + b.y) + (f.x + f.y);
-            }
-            pq[j] = make_float2(1024.f * (lo + hi), lo + 16.f * hi);
+        for (int u = tid; u < p.nchunks * 4; u += kThreads) {
+            const int j = u >> 2, w = u & 3;
+            const uint4 v = ldg_v4(p.X + 8 * u);
+            uint4 o;
+            o.x = __byte_perm(v.x, v.z, 0x5410);
+            o.y = h2_as_u32(__hmul2(u32_as_h2(__byte_perm(v.x, v.z, 0x7632)), sixteenth));
+            o.z = __byte_perm(v.y, v.w, 0x5410);
+            o.w = h2_as_u32(__hmul2(u32_as_h2(__byte_perm(v.y, v.w, 0x7632)), sixteenth));
+            *reinterpret_cast<uint4 *>(xs + j * kChunk + w * 16) = o;
+            const float2 a = __half22float2(u32_as_h2(o.x)), b = __half22float2(u32_as_h2(o.y));
+            const float2 e = __half22float2(u32_as_h2(o.z)), f = __half22float2(u32_as_h2(o.w));
+            float lo = (a.x + a.y) + (e.x + e.y);   // the low-position x
+            float hi = (b.x + b.y) + (f.x + f.y);   // the high-position x~
+            lo += __shfl_xor_sync(0xffffffffu, lo, 1);
+            hi += __shfl_xor_sync(0xffffffffu, hi, 1);
+            lo += __shfl_xor_sync(0xffffffffu, lo, 2);
+            hi += __shfl_xor_sync(0xffffffffu, hi, 2);
+            if (w == 0)
+                pq[j] = make_float2(1024.f * (lo + hi), lo + 16.f * hi);
         }
         if (tid < kChunk / 16)
             reinterpret_cast<uint4 *>(zchunk)[tid] = make_uint4(0, 0, 0, 0);
@@ -251,6 +273,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     float ya = 0.f, yb = 0.f;   // rows g and g+8 of the current tile segment
     bool seg_from0 = false;
     int nseg = 0;               // segments of this warp emitted so far
+    float best_v = -INFINITY;   // greedy decoding: this thread's best stored logit
+    int best_i = 0x7fffffff;
     const int hm = g - 2 * c;   // the half (0 or 1) in which this thread's column takes x, if any
     for (int u = u0; u < u1; u++) {
         const int tl = u / p.nbx, box = u - tl * p.nbx;
@@ -263,12 +287,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         const unsigned char *bx = my_box_ptr + cslot * kBoxBytes;
         const unsigned char *par = my_par_ptr + cslot * kParBytes;
         const float4 pqv = *reinterpret_cast<const float4 *>(pq + box * 8 + 2 * c);   // P, Q of columns 2c, 2c+1
-        // two independent MMA chains (one per half of the box), the first
-        // started from -P
-        float acc2[2][4] = {{-pqv.x, -pqv.z, -pqv.x, -pqv.z}, {0.f, 0.f, 0.f, 0.f}};
+        // four independent MMA chains (half of the box x parity of the word),
+        // the first started from -P: the 16 MMAs of a box form chains of four
+        float acc4[4][4] = {{-pqv.x, -pqv.z, -pqv.x, -pqv.z}, {0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f},
+                            {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
         for (int h = 0; h < 2; h++) {
-            float *acc = acc2[h];
             const int chunk = 2 * c + h;
             const uint4 va = *reinterpret_cast<const uint4 *>(bx + g * 128 + ((chunk ^ g) << 4));
             const uint4 vb = *reinterpret_cast<const uint4 *>(bx + (g + 8) * 128 + ((chunk ^ g) << 4));
@@ -289,6 +313,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const uint32_t b1 = lop3_and_or(wb[w], 0x00F000F0u, 0x64006400u);
                 const uint32_t b2 = lop3_and_or(b8, 0x000F000Fu, 0x64006400u);
                 const uint32_t b3 = lop3_and_or(b8, 0x00F000F0u, 0x64006400u);
+                float *acc = acc4[2 * h + (w & 1)];
                 mma16816(acc, a0, b0, a1, b1, xv.x, xv.y);
                 mma16816(acc, a2, b2, a3, b3, xv.z, xv.w);
             }
@@ -297,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         {
             float acc[4];
 #pragma unroll
-            for (int e = 0; e < 4; e++) acc[e] = acc2[0][e] + acc2[1][e];
+            for (int e = 0; e < 4; e++) acc[e] = (acc4[0][e] + acc4[1][e]) + (acc4[2][e] + acc4[3][e]);
             const float2 sa = scale_pair<BS64>(par, g, c), sb = scale_pair<BS64>(par, g + 8, c);
             const float2 za = zp_pair<BS64, ZP>(par, g, c, box), zb = zp_pair<BS64, ZP>(par, g + 8, c, box);
             if (!dead) {
@@ -323,8 +348,15 @@ __global__ void __launch_bounds__(kThreads, 2)
             if (seg_from0 && box == p.nbx - 1) {
                 if (c == 0 && !dead) {
                     const int n = tile * kRows + g;
-                    if (n < p.N) p.Y[n] = __float2half_rn(ya);
-                    if (n + 8 < p.N) p.Y[n + 8] = __float2half_rn(yb);
+                    const __half ha = __float2half_rn(ya), hb = __float2half_rn(yb);
+                    if (n < p.N) {
+                        p.Y[n] = ha;
+                        keep_best(__half2float(ha), n, best_v, best_i);
+                    }
+                    if (n + 8 < p.N) {
+                        p.Y[n + 8] = hb;
+                        keep_best(__half2float(hb), n + 8, best_v, best_i);
+                    }
                 }
             } else {
                 // a partial: the first segment of the run in slot 0, the last in slot 1
@@ -355,8 +387,62 @@ __global__ void __launch_bounds__(kThreads, 2)
                 if (part_tile[q] == tile)
                     v += part[q * kRows + row];
             const int n = tile * kRows + row;
-            if (n < p.N && !dead)
-                p.Y[n] = __float2half_rn(v);
+            if (n < p.N && !dead) {
+                const __half h = __float2half_rn(v);
+                p.Y[n] = h;
+                keep_best(__half2float(h), n, best_v, best_i);
+            }
+        }
+    }
+
+    // ---- greedy decoding: the CTA's best into the workspace; the last CTA
+    // to finish reduces every CTA's and resets the counter for the next call
+    if (p.argmax) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, best_v, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, best_i, o);
+            keep_best(ov, oi, best_v, best_i);
+        }
+        if (lane == 0)
+            wbest[warp] = make_uint2(__float_as_uint(best_v), (unsigned)best_i);
+        __syncthreads();
+        __shared__ int s_last;
+        if (tid == 0) {
+            float v = -INFINITY;
+            int i = 0x7fffffff;
+            for (int w = 0; w < kWarps; w++)
+                keep_best(__uint_as_float(wbest[w].x), (int)wbest[w].y, v, i);
+            p.ws_part[blockIdx.x] = make_uint2(__float_as_uint(v), (unsigned)i);
+            __threadfence();
+            s_last = (atomicAdd(p.ws_count, 1u) == gridDim.x - 1);
+        }
+        __syncthreads();
+        if (s_last) {
+            __threadfence();
+            float v = -INFINITY;
+            int i = 0x7fffffff;
+            for (int b = tid; b < (int)gridDim.x; b += kThreads) {
+                const uint2 e = __ldcg(p.ws_part + b);
+                keep_best(__uint_as_float(e.x), (int)e.y, v, i);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, v, o);
+                const int oi = __shfl_xor_sync(0xffffffffu, i, o);
+                keep_best(ov, oi, v, i);
+            }
+            if (lane == 0)
+                wbest[warp] = make_uint2(__float_as_uint(v), (unsigned)i);
+            __syncthreads();
+            if (tid == 0) {
+                for (int w = 1; w < kWarps; w++)
+                    keep_best(__uint_as_float(wbest[w].x), (int)wbest[w].y, v, i);
+                p.ids[0] = i;
+                if (p.max_out)
+                    p.max_out[0] = v;
+                *p.ws_count = 0u;   // ready for the next call
+            }
         }
     }
 
@@ -375,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 
 size_t res_smem_bytes(int depth, int nchunks) {
     return 1024 + (size_t)kWarps * depth * (kBoxBytes + kParBytes + 8) + (size_t)nchunks * (kChunk + 8) + kChunk +
-           (size_t)kWarps * 2 * (kRows * 4 + 4);
+           (size_t)kWarps * 2 * (kRows * 4 + 4) + (size_t)kWarps * 8;
 }
 
 template <bool BS64, bool ZP>
@@ -410,7 +496,8 @@ int launch_res_t(const CUtensorMap &map, const ResParams &p, int grid, size_t sm
 }  // namespace
 
 int launch_gemv_resident(const void *X, const uint8_t *packed, const void *scales, const uint8_t *zp, void *Y, int N,
-                         int K, int bs, unsigned flags, cudaStream_t s) {
+                         int K, int bs, unsigned flags, cudaStream_t s, int32_t *ids, float *max_out,
+                         void *workspace) {
     const bool bs64 = (bs == 64), has_zp = (zp != nullptr);
     if (K % kBoxK != 0 || (bs64 && has_zp && K % 512 != 0) || !aligned(scales, bs64 ? 8 : 16) ||
         (has_zp && !aligned(zp, 4)))
@@ -427,8 +514,11 @@ int launch_gemv_resident(const void *X, const uint8_t *packed, const void *scale
     p.ntiles = (N + kRows - 1) / kRows;
     p.nbx = K / kBoxK;
     p.nchunks = K / 32;
+    // one CTA per SM (the next kernel's CTAs take the other half); a weight
+    // stream of more than 16 tiles per SM (the lm_head) takes both halves, as
+    // the ring of one CTA leaves the SM with too few warps to hide its latency
     const int sms = device_sm_count();
-    const int grid = p.ntiles < sms ? p.ntiles : sms;
+    const int grid = p.ntiles < sms ? p.ntiles : (p.ntiles > 16 * sms ? 2 * sms : sms);
     p.tq = p.ntiles / grid;
     p.tr = p.ntiles % grid;
     // the deepest ring (up to the most units a warp owns) that keeps two CTAs per SM
@@ -440,6 +530,11 @@ int launch_gemv_resident(const void *X, const uint8_t *packed, const void *scale
     if (res_smem_bytes(depth, p.nchunks) > (size_t)kSmemBudget)
         return 1;
     p.depth = depth;
+    p.argmax = ids ? 1 : 0;
+    p.ids = ids;
+    p.max_out = max_out;
+    p.ws_count = static_cast<unsigned *>(workspace);
+    p.ws_part = workspace ? reinterpret_cast<uint2 *>(static_cast<unsigned char *>(workspace) + 256) : nullptr;
     const size_t smem = res_smem_bytes(depth, p.nchunks);
 
     EncodeTiledFn encode = tensor_map_encoder();

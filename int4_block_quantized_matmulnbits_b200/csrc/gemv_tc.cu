@@ -803,6 +803,11 @@ size_t gemv_argmax_workspace_bytes(int M) {
 int launch_gemv_argmax(const void *X, const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,
                        void *Y, int M, int N, int K, int bs, int32_t *ids, float *max_out, void *workspace,
                        unsigned flags, cudaStream_t s) {
+    if (M == 1 && scale_f16 && gemv_resident_enabled()) {   // the one-token kernel, as mnb_gemv at M = 1
+        const int rc = launch_gemv_resident(X, packed, scales, zp, Y, N, K, bs, flags, s, ids, max_out, workspace);
+        if (rc != 1)
+            return rc;
+    }
     ArgmaxArgs am{ids, max_out, workspace};
     return launch_tc_common(X, packed, scales, scale_f16, zp, Y, M, N, K, bs, flags, s, &am);
 }
@@ -856,8 +861,7 @@ int launch_gemv_argmax_noalloc(const void *X, const uint8_t *packed, const void 
     cudaError_t e = cudaMemsetAsync(scratch, 0, kArgmaxWsHeader, s);
     if (e != cudaSuccess)
         return fail(MNB_ERR_CUDA, "mnb_gemv_argmax_noalloc: clearing the scratch counter: %s", cudaGetErrorString(e));
-    ArgmaxArgs am{ids, max_out, scratch};
-    return launch_tc_common(X, packed, scales, scale_f16, zp, Y, M, N, K, bs, flags, s, &am);
+    return launch_gemv_argmax(X, packed, scales, scale_f16, zp, Y, M, N, K, bs, ids, max_out, scratch, flags, s);
 }
 
 int read_gemv_status(unsigned *out, int clear) {
