@@ -123,28 +123,57 @@ __device__ __forceinline__ void slot_wait(uint32_t bar, uint32_t parity, bool &d
     }
 }
 
-// Requests unit (tile, box) into a ring slot: the packed box by TMA (lane 0),
+// A warp's request cursor: the next unit (tile, box) and, for this lane, the
+// global address of its parameter bytes of that box (lanes 0-15: the scales of
+// row n0 + lane; lanes 16-31: the zero points of row n0 + lane - 16) and
+// whether that row exists.  Advancing by a box is a pointer increment; only a
+// new tile recomputes the addresses.
+struct IssueCursor {
+    int tile, box;
+    const uint8_t *src;
+    bool row_ok;
+};
+
+template <bool BS64, bool ZP>
+__device__ __forceinline__ void cursor_at_tile(const ResParams &p, IssueCursor &q, int tile, int box, int lane) {
+    q.tile = tile;
+    q.box = box;
+    const int n = tile * kRows + (lane & 15);
+    q.row_ok = n < p.N;
+    if (lane < 16)
+        q.src = p.scales + ((int64_t)n * p.nb + box * (BS64 ? 4 : 8)) * 2;
+    else
+        q.src = ZP ? p.zp + (int64_t)n * p.zpb + (BS64 ? (box >> 1) * 4 : box * 4) : nullptr;
+}
+
+template <bool BS64, bool ZP>
+__device__ __forceinline__ void cursor_next(const ResParams &p, IssueCursor &q, int lane) {
+    if (++q.box == p.nbx) {
+        cursor_at_tile<BS64, ZP>(p, q, q.tile + 1, 0, lane);
+        return;
+    }
+    if (lane < 16)
+        q.src += BS64 ? 8 : 16;
+    else if (ZP && (!BS64 || (q.box & 1) == 0))
+        q.src += 4;   // block 64: one 4-byte load of zero points serves two boxes
+}
+
+// Requests the cursor's unit into a ring slot: the packed box by TMA (lane 0),
 // the box's scales (lanes 0-15) and zero points (lanes 16-31) by cp.async.
 // Rows past N get no parameters (their sums are never stored).  Every lane
 // arrives on the slot's barrier once its copies have landed.
 template <bool BS64, bool ZP>
-__device__ __forceinline__ void issue(const CUtensorMap *wmap, const ResParams &p, int tile, int box, uint32_t box_dst,
+__device__ __forceinline__ void issue(const CUtensorMap *wmap, const IssueCursor &q, uint32_t box_dst,
                                       uint32_t par_dst, uint32_t full, int lane) {
-    const int n0 = tile * kRows;
     if (lane == 0) {
         mbar_expect_tx(full, kBoxBytes);
-        tma_load_2d(box_dst, wmap, full, box * 128, n0);
+        tma_load_2d(box_dst, wmap, full, q.box * 128, q.tile * kRows);
     }
-    if (lane < 16) {
-        if (n0 + lane < p.N) {
-            const uint8_t *src = p.scales + ((int64_t)(n0 + lane) * p.nb + box * (BS64 ? 4 : 8)) * 2;
-            if (BS64) cp_async_8(par_dst + lane * 16, src); else cp_async_16(par_dst + lane * 16, src);
-        }
-    } else if (ZP) {
-        const int row = lane - 16;
-        if (n0 + row < p.N) {
-            const uint8_t *src = p.zp + (int64_t)(n0 + row) * p.zpb + (BS64 ? (box >> 1) * 4 : box * 4);
-            cp_async_4(par_dst + 256 + row * 4, src);
+    if (q.row_ok) {
+        if (lane < 16) {
+            if (BS64) cp_async_8(par_dst + lane * 16, q.src); else cp_async_16(par_dst + lane * 16, q.src);
+        } else if (ZP) {
+            cp_async_4(par_dst + 256 + (lane - 16) * 4, q.src);
         }
     }
     cp_async_arrive(full);
@@ -168,12 +197,14 @@ template <bool BS64, bool ZP>
 __device__ __forceinline__ float2 zp_pair(const unsigned char *par, int row, int c, int box) {
     if (!ZP)
         return make_float2(8.f, 8.f);
+    // a nibble z as fp32 without the conversion unit: (2^23 + z) - 2^23
     if (!BS64) {
         const uint32_t zb = par[256 + row * 4 + c];   // blocks 2c (low nibble) and 2c+1 (high)
-        return make_float2((float)(zb & 15u), (float)(zb >> 4));
+        return make_float2(__uint_as_float(0x4B000000u | (zb & 15u)) - 8388608.f,
+                           __uint_as_float(0x4B000000u | (zb >> 4)) - 8388608.f);
     }
     const uint32_t zb = par[256 + row * 4 + (box & 1) * 2 + (c >> 1)];
-    const float z = (float)((c & 1) ? (zb >> 4) : (zb & 15u));
+    const float z = __uint_as_float(0x4B000000u | ((c & 1) ? (zb >> 4) : (zb & 15u))) - 8388608.f;
     return make_float2(z, z);
 }
 
@@ -220,11 +251,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncwarp();
 
     // ---- weights first: they do not depend on the previous kernel
-    int iu = u0, islot = 0;   // next unit to request, its slot
+    const int tl0 = u0 / p.nbx;          // this warp's first unit
+    const int box0 = u0 - tl0 * p.nbx;
+    int iu = u0, islot = 0;              // next unit to request, its slot
+    IssueCursor ic;
+    cursor_at_tile<BS64, ZP>(p, ic, t0 + tl0, box0, lane);
     auto request = [&]() {
-        const int tl = iu / p.nbx;
-        issue<BS64, ZP>(&wmap, p, t0 + tl, iu - tl * p.nbx, my_box + islot * kBoxBytes, my_par + islot * kParBytes,
-                        my_bars + 8 * islot, lane);
+        issue<BS64, ZP>(&wmap, ic, my_box + islot * kBoxBytes, my_par + islot * kParBytes, my_bars + 8 * islot, lane);
+        cursor_next<BS64, ZP>(p, ic, lane);
         ++iu;
         if (++islot == D) islot = 0;
     };
@@ -276,8 +310,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     float best_v = -INFINITY;   // greedy decoding: this thread's best stored logit
     int best_i = 0x7fffffff;
     const int hm = g - 2 * c;   // the half (0 or 1) in which this thread's column takes x, if any
-    for (int u = u0; u < u1; u++) {
-        const int tl = u / p.nbx, box = u - tl * p.nbx;
+    int tl = tl0, box = box0;   // the unit being consumed (CTA-local tile, box)
+    for (int u = u0; u < u1; u++, box = (box + 1 == p.nbx) ? 0 : box + 1, tl += (box == 0) ? 1 : 0) {
         if (u == u0 || box == 0) {
             ya = yb = 0.f;
             seg_from0 = (box == 0);
