@@ -77,11 +77,17 @@ struct ResParams {
     // stored), max_out[0] its value; per-CTA partials in a caller workspace,
     // reduced by the last CTA to finish (counter in the workspace's header)
     int argmax;
+    // SwiGLU epilogue: weight rows in 16-row groups, 8 gate rows then the 8 up
+    // rows of the same outputs; y[8 t + i] = silu(gate) * up, N / 2 outputs
+    int swiglu;
     int32_t *ids;
     float *max_out;
     uint2 *ws_part;           // [gridDim.x] (value bits, index)
     unsigned *ws_count;
 };
+
+// silu(x) = x * sigmoid(x), in fp32.
+__device__ __forceinline__ float silu(float x) { return x / (1.0f + __expf(-x)); }
 
 // (value, index) pairs ordered by value, then by the SMALLER index: the greedy
 // token is the first maximum.
@@ -405,7 +411,10 @@ __global__ void __launch_bounds__(kThreads, 2)
             yb += __shfl_xor_sync(0xffffffffu, yb, 2);
             const int tile = t0 + tl;
             if (seg_from0 && box == p.nbx - 1) {
-                if (c == 0 && !dead) {
+                if (c == 0 && !dead && p.swiglu) {   // row g is a gate, row g + 8 its up
+                    if (tile * kRows + g < p.N)
+                        p.Y[tile * 8 + g] = __float2half_rn(silu(ya) * yb);
+                } else if (c == 0 && !dead) {
                     const int n = tile * kRows + g;
                     const __half ha = __float2half_rn(ya), hb = __float2half_rn(yb);
                     if (n < p.N) {
@@ -440,7 +449,18 @@ __global__ void __launch_bounds__(kThreads, 2)
         bool leader = tile >= 0;
         for (int q = 0; q < sl && leader; q++)
             leader = part_tile[q] != tile;
-        if (leader) {
+        if (leader && p.swiglu) {   // rows < 8: the gates; row + 8: their ups
+            if (row < 8) {
+                float gv = 0.f, uv = 0.f;
+                for (int q = sl; q < kWarps * 2; q++)
+                    if (part_tile[q] == tile) {
+                        gv += part[q * kRows + row];
+                        uv += part[q * kRows + row + 8];
+                    }
+                if (tile * kRows + row < p.N && !dead)
+                    p.Y[tile * 8 + row] = __float2half_rn(silu(gv) * uv);
+            }
+        } else if (leader) {
             float v = 0.f;
             for (int q = sl; q < kWarps * 2; q++)
                 if (part_tile[q] == tile)
@@ -556,7 +576,7 @@ int launch_res_t(const CUtensorMap &map, const ResParams &p, int grid, size_t sm
 
 int launch_gemv_resident(const void *X, const uint8_t *packed, const void *scales, const uint8_t *zp, void *Y, int N,
                          int K, int bs, unsigned flags, cudaStream_t s, int32_t *ids, float *max_out,
-                         void *workspace) {
+                         void *workspace, int swiglu) {
     const bool bs64 = (bs == 64), has_zp = (zp != nullptr);
     if (K % kBoxK != 0 || (bs64 && has_zp && K % 512 != 0) || !aligned(scales, bs64 ? 8 : 16) ||
         (has_zp && !aligned(zp, 4)))
@@ -593,6 +613,7 @@ int launch_gemv_resident(const void *X, const uint8_t *packed, const void *scale
         return 1;
     p.depth = depth;
     p.argmax = ids ? 1 : 0;
+    p.swiglu = swiglu;
     p.ids = ids;
     p.max_out = max_out;
     p.ws_count = static_cast<unsigned *>(workspace);

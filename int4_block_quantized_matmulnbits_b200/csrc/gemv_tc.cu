@@ -792,6 +792,11 @@ int launch_gemv_tc(const void *X, const uint8_t *packed, const void *scales, int
 
 int launch_gemv_swiglu(const void *X, const uint8_t *packed, const void *scales, int scale_f16, const uint8_t *zp,
                        void *Y, int M, int N, int K, int bs, unsigned flags, cudaStream_t s) {
+    if (M == 1 && scale_f16 && gemv_resident_enabled()) {   // the one-token kernel, as mnb_gemv at M = 1
+        const int rc = launch_gemv_resident(X, packed, scales, zp, Y, N, K, bs, flags, s, nullptr, nullptr, nullptr, 1);
+        if (rc != 1)
+            return rc;
+    }
     return launch_tc_common(X, packed, scales, scale_f16, zp, Y, M, N, K, bs, flags, s, nullptr, 1);
 }
 

@@ -26,10 +26,11 @@ int launch_gemv_tc(const void *X, const uint8_t *packed, const void *scales, int
 // whole share of the weights in shared memory; returns 1 without launching
 // anything for shapes it does not serve.  With ids != null it also does greedy
 // decoding, with the workspace layout of mnb_gemv_argmax (256-byte counter
-// header, then one (value, index) pair per CTA; at most two CTAs per SM).
+// header, then one (value, index) pair per CTA; at most two CTAs per SM); with
+// swiglu != 0 the SwiGLU epilogue of mnb_gemv_swiglu.
 int launch_gemv_resident(const void *X, const uint8_t *packed, const void *scales, const uint8_t *zp, void *Y, int N,
                          int K, int bs, unsigned flags, cudaStream_t s, int32_t *ids = nullptr,
-                         float *max_out = nullptr, void *workspace = nullptr);
+                         float *max_out = nullptr, void *workspace = nullptr, int swiglu = 0);
 // Whether one-token fp16 calls go to the resident kernel (tuning hook).
 int gemv_resident_enabled();
 

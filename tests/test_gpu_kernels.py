@@ -266,6 +266,9 @@ def _interleave8(g, u):
 
 
 @pytest.mark.parametrize("M,I,K,bs,has_zp,sdt", [(1, 6144, 2048, 32, True, np.float16),
+                                                 (1, 1024, 2048, 32, True, np.float16),
+                                                 (1, 3000, 1024, 64, False, np.float16),
+                                                 (1, 1024, 6144, 32, True, np.float16),
                                                  (4, 3072, 1024, 32, True, np.float16),
                                                  (16, 1000, 1024, 64, True, np.float32),
                                                  (3, 8, 256, 32, False, np.float16),
@@ -312,6 +315,8 @@ def test_gemv_swiglu_layout_helper(mnb, cuda_dev):
 ARGMAX_CASES = [
     # M, N, K, bs, has_zp, scale
     (1, 151936, 2048, 32, True, np.float16),   # the 1.7B lm_head
+    (1, 1000, 2048, 32, True, np.float16),     # one token: tiles cut between warps
+    (1, 33, 256, 32, False, np.float16),
     (4, 5000, 1024, 64, True, np.float16),
     (3, 777, 512, 32, False, np.float32),
     (16, 1000, 2048, 32, True, np.float16),
