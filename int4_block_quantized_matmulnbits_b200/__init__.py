@@ -258,8 +258,15 @@ def mnb_device_status(clear=False) -> int:
     return v.value
 
 
+def _contiguous(fn, *ts):
+    for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise MnbError(fn, -1, "tensors must be contiguous (row-major)")
+
+
 def mnb_gptq_hessian(X, H, accumulate=False, stream=None):
     """H [K, K] fp32 (+)= X^T X for calibration inputs X [T, K] (fp32 or fp16)."""
+    _contiguous("mnb_gptq_hessian", X, H)
     T, K = X.shape
     _check("mnb_gptq_hessian", _lib.mnb_gptq_hessian(_ptr(X), _dt(X), T, K, _ptr(H), int(bool(accumulate)),
                                                      _stream(stream)))
@@ -272,6 +279,7 @@ def mnb_gptq_workspace_bytes(K) -> int:
 def mnb_gptq_prepare(H, U, dead, workspace, percdamp=0.01, stream=None) -> float:
     """U [K, K] fp32 = upper Cholesky factor of the damped H^-1; dead [K] uint8.
     Synchronizes the stream; returns the damping that succeeded."""
+    _contiguous("mnb_gptq_prepare", H, U, dead)
     K = H.shape[0]
     d = ctypes.c_float()
     _check("mnb_gptq_prepare", _lib.mnb_gptq_prepare(
@@ -282,6 +290,7 @@ def mnb_gptq_prepare(H, U, dead, workspace, percdamp=0.01, stream=None) -> float
 
 def mnb_gptq_quantize(W, U, dead, bs, has_zp, packed, scales, zp, stream=None):
     """GPTQ of fp32 W [N, K] into packed / scales / zp (the layout of mnb_quantize_rtn)."""
+    _contiguous("mnb_gptq_quantize", W, U, dead, packed, scales, zp)
     N, K = W.shape
     _check("mnb_gptq_quantize", _lib.mnb_gptq_quantize(
         _ptr(W), _ptr(U), _ptr(dead), N, K, bs, int(bool(has_zp)), _ptr(packed), _ptr(scales), _dt(scales),

@@ -193,7 +193,7 @@ def gptq_prepare(H, percdamp=0.01):
     damp = percdamp * np.mean(d)
     H[np.arange(K), np.arange(K)] += damp
     Hinv = np.linalg.inv(H)
-    U = np.linalg.cholesky(Hinv).T        # lower L with Hinv = L L^T; U = L^T
+    U = np.ascontiguousarray(np.linalg.cholesky(Hinv).T)   # lower L with Hinv = L L^T; U = L^T, row-major
     return U, dead.astype(np.uint8)
 
 

@@ -104,7 +104,7 @@ def test_gptq_quantize_bit_exact(mnb, cuda_dev, N, K, bs, has_zp, sdt):
     X = _calib(rng, max(2 * K, 256), K)
     X[:, 5] = 0.0
     Uo, deado = oracle.gptq_prepare(oracle.gptq_hessian(X))
-    U32 = Uo.astype(np.float32)
+    U32 = np.ascontiguousarray(Uo, dtype=np.float32)
     W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
     W[rng.random((N, K)) < 0.01] *= 8.0       # outliers
     ref = oracle.gptq_quantize(W, U32, bs, has_zp, sdt, deado)
