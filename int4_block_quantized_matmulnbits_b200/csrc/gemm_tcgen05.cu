@@ -216,7 +216,7 @@ __device__ __forceinline__ void dq_store(const uint2 &v, uint32_t s16, uint32_t 
 
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap wmap,
-                const GemmParams p) {
+                const __grid_constant__ CUtensorMap ymap, const GemmParams p) {
     extern __shared__ unsigned char smem_raw[];
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -403,7 +403,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         };
         if (p.S == 1) {
-            // two 16-column chunks per tensor-memory load round trip
+            // the tile goes through shared memory (the idle fp16 weight ring) as
+            // [BN tokens][128 rows] fp16 and leaves in one TMA store; two 16-column
+            // chunks per tensor-memory load round trip
+            __half *stage = reinterpret_cast<__half *>(base_ptr);
             for (int c16 = grp; c16 < nchunk; c16 += 8) {
                 const bool two = c16 + 4 < nchunk;
                 uint32_t v[2][16];
@@ -417,11 +420,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int h = 0; h < 2; h++) {
                     if (h == 1 && !two)
                         break;
-                    float f[16];
+                    const int col = (c16 + 4 * h) * 16;
 #pragma unroll
-                    for (int j = 0; j < 16; j++) f[j] = have ? __uint_as_float(v[h][j]) : 0.f;
-                    store_y((c16 + 4 * h) * 16, f);
+                    for (int j = 0; j < 16; j++)
+                        stage[(col + j) * kBM + row] = __float2half_rn(have ? __uint_as_float(v[h][j]) : 0.f);
                 }
+            }
+            fence_proxy_async_smem();   // the TMA store reads what the generic stores wrote
+            asm volatile("bar.sync 1, %0;" ::"n"(kDqWarps * 32) : "memory");
+            if (warp == 3 && lane == 0 && have) {
+                asm volatile(
+                    "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(&ymap),
+                    "r"(n_tile * kBM), "r"(m0), "r"(smem_u32(stage))
+                    : "memory");
+                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");   // written before the CTA leaves
             }
         } else {
             // K split over the cluster.  Each rank parks its partial sums
@@ -604,6 +617,19 @@ int launch_gemm(const void *X, const uint8_t *packed, const void *scales, int sc
             return fail(MNB_ERR_CUDA, "mnb_gemm: cuTensorMapEncodeTiled (W) failed (%d)", (int)cr);
     }
 
+    CUtensorMap ymap;   // Y [M][N] fp16, box [BN tokens][128 rows]: the epilogue's TMA store
+    {
+        const cuuint64_t gdim[2] = {(cuuint64_t)N, (cuuint64_t)M};
+        const cuuint64_t gstride[1] = {(cuuint64_t)N * 2};
+        const cuuint32_t box[2] = {(cuuint32_t)kBM, (cuuint32_t)BN};
+        const cuuint32_t estride[2] = {1, 1};
+        CUresult cr = encode(&ymap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, Y, gdim, gstride, box, estride,
+                             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (cr != CUDA_SUCCESS)
+            return fail(MNB_ERR_CUDA, "mnb_gemm: cuTensorMapEncodeTiled (Y) failed (%d)", (int)cr);
+    }
+
     static int configured[kMaxDevices] = {};
     {
         cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(gemm_kernel), (int)smem, configured);
@@ -631,7 +657,7 @@ int launch_gemm(const void *X, const uint8_t *packed, const void *scales, int sc
     }
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel, xmap, wmap, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel, xmap, wmap, ymap, p);
     if (e != cudaSuccess)
         return fail(MNB_ERR_CUDA, "mnb_gemm: launch: %s", cudaGetErrorString(e));
     return MNB_OK;
