@@ -70,7 +70,6 @@ struct ResParams {
     __half *Y;                // [N]
     int N, K, nb, zpb;
     int ntiles, nbx, nchunks; // ceil(N / 16), K / 256, K / 32
-    int xwarp;                // 1: each warp stages the x of its own units (all of them fit its ring)
     int tq, tr;               // tiles per CTA: tq, one more for CTAs below tr
     int depth;                // ring slots per warp
     // greedy decoding: ids[0] = the first n of max y[n] (over the fp16 values
@@ -228,12 +227,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
     unsigned char *bp = smem_raw + (base - smem_u32(smem_raw));
     unsigned char *pars = bp + kWarps * D * kBoxBytes;
-    // x: [chunk] for the CTA, or [warp][unit][8 chunks] when each warp stages its own
-    const int xchunks = p.xwarp ? kWarps * D * 8 : p.nchunks;
     unsigned char *xs = pars + kWarps * D * kParBytes;
-    unsigned char *zchunk = xs + xchunks * kChunk;
+    unsigned char *zchunk = xs + p.nchunks * kChunk;
     float2 *pq = reinterpret_cast<float2 *>(zchunk + kChunk);
-    float *part = reinterpret_cast<float *>(pq + xchunks);        // [warp][2 slots][16 rows]
+    float *part = reinterpret_cast<float *>(pq + p.nchunks);      // [warp][2 slots][16 rows]
     int *part_tile = reinterpret_cast<int *>(part + kWarps * 2 * kRows);
     uint2 *wbest = reinterpret_cast<uint2 *>(part_tile + kWarps * 2);   // greedy decoding: per warp
     const uint32_t bars = smem_u32(wbest + kWarps);
@@ -257,8 +254,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     if (tid < kWarps * 2)
         part_tile[tid] = -1;
-    if (tid < kChunk / 16)
-        reinterpret_cast<uint4 *>(zchunk)[tid] = make_uint4(0, 0, 0, 0);
     __syncwarp();
 
     // ---- weights first: they do not depend on the previous kernel
@@ -276,60 +271,41 @@ __global__ void __launch_bounds__(kThreads, 2)
     while (iu < u1 && iu - u0 < D)
         request();
     pdl_launch_dependents();
-    __syncthreads();   // the zero chunk and the partial-sum tiles are set (before the wait: off the critical path)
     pdl_wait();
 
     // ---- stage x: chunk j (k = 32j .. 32j+31) as four 16-byte words, word w =
     // (x0,x4) (x1,x5)/16 (x2,x6) (x3,x7)/16 of k = 32j + 8w ..; and per chunk
     // P = 1024 sum x~ and Q = sum x over the staged values x~ (x/16 counted
     // back as 16 x~), so the correction matches the MMA's operands exactly.
-    // A 16-byte word per lane: the four words of a chunk sit in four
-    // consecutive lanes, which add their sums by shuffles.
-    const half2 sixteenth = __floats2half2_rn(0.0625f, 0.0625f);
-    auto stage_word = [&](const uint4 v, int jx, int w) {   // jx: chunk slot in xs / pq
-        uint4 o;
-        o.x = __byte_perm(v.x, v.z, 0x5410);
-        o.y = h2_as_u32(__hmul2(u32_as_h2(__byte_perm(v.x, v.z, 0x7632)), sixteenth));
-        o.z = __byte_perm(v.y, v.w, 0x5410);
-        o.w = h2_as_u32(__hmul2(u32_as_h2(__byte_perm(v.y, v.w, 0x7632)), sixteenth));
-        *reinterpret_cast<uint4 *>(xs + jx * kChunk + w * 16) = o;
-        const float2 a = __half22float2(u32_as_h2(o.x)), b = __half22float2(u32_as_h2(o.y));
-        const float2 e = __half22float2(u32_as_h2(o.z)), f = __half22float2(u32_as_h2(o.w));
-        float lo = (a.x + a.y) + (e.x + e.y);   // the low-position x
-        float hi = (b.x + b.y) + (f.x + f.y);   // the high-position x~
-        lo += __shfl_xor_sync(0xffffffffu, lo, 1);
-        hi += __shfl_xor_sync(0xffffffffu, hi, 1);
-        lo += __shfl_xor_sync(0xffffffffu, lo, 2);
-        hi += __shfl_xor_sync(0xffffffffu, hi, 2);
-        if (w == 0)
-            pq[jx] = make_float2(1024.f * (lo + hi), lo + 16.f * hi);
-    };
-    if (p.xwarp) {
-        // each warp stages the 256 k of each of its units: lane l takes word l
-        // of the box; every unit of the warp is in its ring, so no other warp
-        // waits for this and no CTA barrier is needed
-        uint4 vv[kMaxDepth];
-        {
-            int tl = tl0, box = box0;
-#pragma unroll
-            for (int i = 0; i < kMaxDepth; i++) {
-                if (u0 + i < u1)
-                    vv[i] = ldg_v4(p.X + box * kBoxK + 8 * lane);
-                if (++box == p.nbx) { box = 0; ++tl; }
-            }
+    // One 16-byte word per thread per pass (K / 8 is a multiple of 32, so every
+    // lane of a warp takes part in each pass); the four words of a chunk sit in
+    // four consecutive lanes, which add their sums by shuffles.
+    {
+        const half2 sixteenth = __floats2half2_rn(0.0625f, 0.0625f);
+        for (int u = tid; u < p.nchunks * 4; u += kThreads) {
+            const int j = u >> 2, w = u & 3;
+            const uint4 v = ldg_v4(p.X + 8 * u);
+            uint4 o;
+            o.x = __byte_perm(v.x, v.z, 0x5410);
+            o.y = h2_as_u32(__hmul2(u32_as_h2(__byte_perm(v.x, v.z, 0x7632)), sixteenth));
+            o.z = __byte_perm(v.y, v.w, 0x5410);
+            o.w = h2_as_u32(__hmul2(u32_as_h2(__byte_perm(v.y, v.w, 0x7632)), sixteenth));
+            *reinterpret_cast<uint4 *>(xs + j * kChunk + w * 16) = o;
+            const float2 a = __half22float2(u32_as_h2(o.x)), b = __half22float2(u32_as_h2(o.y));
+            const float2 e = __half22float2(u32_as_h2(o.z)), f = __half22float2(u32_as_h2(o.w));
+            float lo = (a.x + a.y) + (e.x + e.y);   // the low-position x
+            float hi = (b.x + b.y) + (f.x + f.y);   // the high-position x~
+            lo += __shfl_xor_sync(0xffffffffu, lo, 1);
+            hi += __shfl_xor_sync(0xffffffffu, hi, 1);
+            lo += __shfl_xor_sync(0xffffffffu, lo, 2);
+            hi += __shfl_xor_sync(0xffffffffu, hi, 2);
+            if (w == 0)
+                pq[j] = make_float2(1024.f * (lo + hi), lo + 16.f * hi);
         }
-#pragma unroll
-        for (int i = 0; i < kMaxDepth; i++)
-            if (u0 + i < u1)   // warp-uniform
-                stage_word(vv[i], (warp * D + i) * 8 + (lane >> 2), lane & 3);
-        __syncwarp();
-    } else {
-        // every warp walks the whole of K: the CTA stages x once (K / 8 is a
-        // multiple of 32, so all lanes of a warp take part in each pass)
-        for (int u = tid; u < p.nchunks * 4; u += kThreads)
-            stage_word(ldg_v4(p.X + 8 * u), u >> 2, u & 3);
-        __syncthreads();
+        if (tid < kChunk / 16)
+            reinterpret_cast<uint4 *>(zchunk)[tid] = make_uint4(0, 0, 0, 0);
     }
+    __syncthreads();
 
     // ---- this warp's units
     bool dead = false;
@@ -350,8 +326,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         dead = __any_sync(0xffffffffu, dead);   // one verdict per warp: it issues refills together
         const unsigned char *bx = my_box_ptr + cslot * kBoxBytes;
         const unsigned char *par = my_par_ptr + cslot * kParBytes;
-        const int cb = p.xwarp ? (warp * D + (u - u0)) * 8 : box * 8;   // the box's first chunk slot in xs / pq
-        const float4 pqv = *reinterpret_cast<const float4 *>(pq + cb + 2 * c);   // P, Q of columns 2c, 2c+1
+        const float4 pqv = *reinterpret_cast<const float4 *>(pq + box * 8 + 2 * c);   // P, Q of columns 2c, 2c+1
         // four independent MMA chains (half of the box x parity of the word),
         // the first started from -P: the 16 MMAs of a box form chains of four
         float acc4[4][4] = {{-pqv.x, -pqv.z, -pqv.x, -pqv.z}, {0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f},
@@ -363,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             const uint4 vb = *reinterpret_cast<const uint4 *>(bx + (g + 8) * 128 + ((chunk ^ g) << 4));
             // x of chunk `chunk` goes to column `chunk` only: the thread whose
             // column that is (g == chunk) reads it, every other thread zeros
-            const unsigned char *xa = (hm == h) ? xs + (cb + chunk) * kChunk : zchunk;
+            const unsigned char *xa = (hm == h) ? xs + (box * 8 + chunk) * kChunk : zchunk;
             const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
             const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
@@ -538,8 +513,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 }
 
-size_t res_smem_bytes(int depth, int xchunks) {
-    return 1024 + (size_t)kWarps * depth * (kBoxBytes + kParBytes + 8) + (size_t)xchunks * (kChunk + 8) + kChunk +
+size_t res_smem_bytes(int depth, int nchunks) {
+    return 1024 + (size_t)kWarps * depth * (kBoxBytes + kParBytes + 8) + (size_t)nchunks * (kChunk + 8) + kChunk +
            (size_t)kWarps * 2 * (kRows * 4 + 4) + (size_t)kWarps * 8;
 }
 
@@ -604,12 +579,9 @@ int launch_gemv_resident(const void *X, const uint8_t *packed, const void *scale
     const int Umax = (p.tq + (p.tr ? 1 : 0)) * p.nbx;
     const int per_warp = (Umax + kWarps - 1) / kWarps;
     int depth = per_warp < kMaxDepth ? (per_warp < 2 ? 2 : per_warp) : kMaxDepth;
-    // every unit of every warp in its ring: each warp stages its own x
-    p.xwarp = (per_warp <= depth && res_smem_bytes(depth, kWarps * depth * 8) <= (size_t)kSmemBudget) ? 1 : 0;
-    const int xchunks = [&] { return p.xwarp ? kWarps * depth * 8 : p.nchunks; }();
-    while (!p.xwarp && depth > 2 && res_smem_bytes(depth, xchunks) > (size_t)kSmemBudget)
+    while (depth > 2 && res_smem_bytes(depth, p.nchunks) > (size_t)kSmemBudget)
         --depth;
-    if (res_smem_bytes(depth, p.xwarp ? kWarps * depth * 8 : p.nchunks) > (size_t)kSmemBudget)
+    if (res_smem_bytes(depth, p.nchunks) > (size_t)kSmemBudget)
         return 1;
     p.depth = depth;
     p.argmax = ids ? 1 : 0;
@@ -618,7 +590,7 @@ int launch_gemv_resident(const void *X, const uint8_t *packed, const void *scale
     p.max_out = max_out;
     p.ws_count = static_cast<unsigned *>(workspace);
     p.ws_part = workspace ? reinterpret_cast<uint2 *>(static_cast<unsigned char *>(workspace) + 256) : nullptr;
-    const size_t smem = res_smem_bytes(depth, p.xwarp ? kWarps * depth * 8 : p.nchunks);
+    const size_t smem = res_smem_bytes(depth, p.nchunks);
 
     EncodeTiledFn encode = tensor_map_encoder();
     if (!encode)
