@@ -38,10 +38,16 @@
 //     The 16 MMAs of a box run as four independent accumulator chains: on
 //     the decoder's small projections each warp holds one to three boxes, so
 //     the latency of a chain, not the issue rate, sets the kernel's time.
+//   * Consecutive launches alternate between two resource shapes that cannot
+//     share an SM with themselves but can with each other, so the block
+//     scheduler never puts two CTAs of one launch on an SM (launch_res_t).
 // Every mbarrier wait is bounded in time; past the limit the kernel records
 // the failure in the device status word, lets its copies in flight land and
 // exits.
 #include <cuda.h>
+
+#include <atomic>
+#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -52,8 +58,10 @@ __device__ unsigned g_res_status = 0;
 
 namespace {
 
-constexpr int kWarps = 8;
+constexpr int kWarps = 8;                   // warps that work; a launch may add idle ones (see below)
 constexpr int kThreads = kWarps * 32;
+constexpr int kMaxThreads = 16 * 32;
+constexpr int kMaxRegs = 112;               // register cap of the kernel (the launch shapes depend on it)
 constexpr int kRows = 16;
 constexpr int kBoxK = 256;                  // k per box: 8 blocks of 32 (4 of 64)
 constexpr int kBoxBytes = kRows * 128;
@@ -215,7 +223,7 @@ __device__ __forceinline__ float2 zp_pair(const unsigned char *par, int row, int
 }
 
 template <bool BS64, bool ZP>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __maxnreg__(kMaxRegs)
     gemv_resident_kernel(const __grid_constant__ CUtensorMap wmap, const ResParams p) {
     extern __shared__ unsigned char smem_raw[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -239,15 +247,19 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t my_par = smem_u32(pars) + (uint32_t)(warp * D * kParBytes);
     const unsigned char *my_par_ptr = pars + warp * D * kParBytes;
     const uint32_t my_bars = bars + (uint32_t)(warp * D * 8);
+    // warps beyond kWarps only widen the launch (so that two CTAs of one
+    // launch cannot share an SM): no units, no barriers, no slots; they take
+    // part in the CTA barriers only
+    const bool worker = warp < kWarps;
 
     // this CTA's tiles and this warp's run of (tile, box) units
     const int cta = blockIdx.x;
     const int Tc = p.tq + (cta < p.tr ? 1 : 0);
     const int t0 = cta * p.tq + (cta < p.tr ? cta : p.tr);
     const int U = Tc * p.nbx;
-    const int u0 = warp * U / kWarps, u1 = (warp + 1) * U / kWarps;
+    const int u0 = (worker ? warp : kWarps) * U / kWarps, u1 = (worker ? warp + 1 : kWarps) * U / kWarps;
 
-    if (lane == 0) {
+    if (worker && lane == 0) {
         for (int d = 0; d < D; d++)
             mbar_init(my_bars + 8 * d, 33);   // lane 0's expect_tx + one cp.async arrival per lane
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -282,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     // four consecutive lanes, which add their sums by shuffles.
     {
         const half2 sixteenth = __floats2half2_rn(0.0625f, 0.0625f);
-        for (int u = tid; u < p.nchunks * 4; u += kThreads) {
+        for (int u = tid; worker && u < p.nchunks * 4; u += kThreads) {
             const int j = u >> 2, w = u & 3;
             const uint4 v = ldg_v4(p.X + 8 * u);
             uint4 o;
@@ -420,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     // every slot holding it, in warp order, and stores the rows
     {
         const int sl = tid >> 4, row = tid & 15;   // 16 slots x 16 rows = 256 threads
-        const int tile = part_tile[sl];
+        const int tile = worker ? part_tile[sl] : -1;
         bool leader = tile >= 0;
         for (int q = 0; q < sl && leader; q++)
             leader = part_tile[q] != tile;
@@ -458,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int oi = __shfl_xor_sync(0xffffffffu, best_i, o);
             keep_best(ov, oi, best_v, best_i);
         }
-        if (lane == 0)
+        if (worker && lane == 0)
             wbest[warp] = make_uint2(__float_as_uint(best_v), (unsigned)best_i);
         __syncthreads();
         __shared__ int s_last;
@@ -476,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             __threadfence();
             float v = -INFINITY;
             int i = 0x7fffffff;
-            for (int b = tid; b < (int)gridDim.x; b += kThreads) {
+            for (int b = tid; worker && b < (int)gridDim.x; b += kThreads) {
                 const uint2 e = __ldcg(p.ws_part + b);
                 keep_best(__uint_as_float(e.x), (int)e.y, v, i);
             }
@@ -486,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const int oi = __shfl_xor_sync(0xffffffffu, i, o);
                 keep_best(ov, oi, v, i);
             }
-            if (lane == 0)
+            if (worker && lane == 0)
                 wbest[warp] = make_uint2(__float_as_uint(v), (unsigned)i);
             __syncthreads();
             if (tid == 0) {
@@ -518,19 +530,74 @@ size_t res_smem_bytes(int depth, int nchunks) {
            (size_t)kWarps * 2 * (kRows * 4 + 4) + (size_t)kWarps * 8;
 }
 
+// Launch shapes.  The CTAs of kernel i+1 are placed while kernel i runs;
+// where an SM has both halves free (kernel i had no CTA there, or its CTA has
+// left) the block scheduler may put TWO CTAs of one launch on it, which then
+// share the SM and double its part of the critical path.  Consecutive
+// launches therefore alternate between two shapes that cannot pair with
+// themselves but pair with each other: shape A asks for just over half of
+// the SM's shared memory, shape B for just over half of its registers (idle
+// warps widen it).  One A and one B fit on an SM; two of either do not.  A
+// weight stream (the lm_head: two CTAs per SM by design) keeps the plain
+// shape.
+struct LaunchShape {
+    int threads;
+    size_t smem;
+};
+
 template <bool BS64, bool ZP>
-int launch_res_t(const CUtensorMap &map, const ResParams &p, int grid, size_t smem, unsigned flags, cudaStream_t s) {
+int launch_res_t(const CUtensorMap &map, const ResParams &p, int grid, size_t smem, bool stream_mode, unsigned flags,
+                 cudaStream_t s) {
     auto fn = gemv_resident_kernel<BS64, ZP>;
+    static int regs[kMaxDevices] = {}, smem_sm[kMaxDevices] = {}, reserved[kMaxDevices] = {}, rf[kMaxDevices] = {};
+    static std::atomic<unsigned> parity[kMaxDevices];
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        dev = 0;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (regs[dev] == 0) {
+            cudaFuncAttributes a;
+            cudaError_t e = cudaFuncGetAttributes(&a, fn);
+            if (e == cudaSuccess)
+                e = cudaDeviceGetAttribute(&smem_sm[dev], cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+            if (e == cudaSuccess)
+                e = cudaDeviceGetAttribute(&reserved[dev], cudaDevAttrReservedSharedMemoryPerBlock, dev);
+            if (e == cudaSuccess)
+                e = cudaDeviceGetAttribute(&rf[dev], cudaDevAttrMaxRegistersPerMultiprocessor, dev);
+            if (e == cudaSuccess)   // both halves of an SM's shared memory to this kernel's shapes
+                e = cudaFuncSetAttribute(reinterpret_cast<const void *>(fn),
+                                         cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+            if (e != cudaSuccess)
+                return fail(MNB_ERR_CUDA, "mnb_gemv: kernel attributes: %s", cudaGetErrorString(e));
+            regs[dev] = (a.numRegs + 7) & ~7;
+        }
+    }
+    LaunchShape shape{kThreads, smem};
+    if (!stream_mode) {
+        const int R = regs[dev], half_rf = rf[dev] / 2;
+        const int wB = half_rf / (32 * R) + 1;                              // B: more than half the registers
+        const size_t smemA = (size_t)(smem_sm[dev] - 2 * reserved[dev]) / 2 + 1024;   // A: more than half
+        const bool ok = 32 * R * (kWarps + wB) <= rf[dev] && 32 * wB <= kMaxThreads &&
+                        smemA + smem + 2 * (size_t)reserved[dev] <= (size_t)smem_sm[dev] && smem <= smemA;
+        if (ok) {
+            if (parity[dev].fetch_add(1u, std::memory_order_relaxed) & 1u)
+                shape.threads = 32 * wB;
+            else
+                shape.smem = smemA;
+        }
+    }
     static int configured[kMaxDevices] = {};
     {
-        cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(fn), (int)smem, configured);
+        cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(fn), (int)shape.smem, configured);
         if (e != cudaSuccess)
             return fail(MNB_ERR_CUDA, "mnb_gemv: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
+    cfg.blockDim = dim3((unsigned)shape.threads, 1, 1);
+    cfg.dynamicSmemBytes = shape.smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     int na = 0;
@@ -605,12 +672,13 @@ int launch_gemv_resident(const void *X, const uint8_t *packed, const void *scale
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (cr != CUDA_SUCCESS)
         return fail(MNB_ERR_CUDA, "mnb_gemv: cuTensorMapEncodeTiled failed (%d)", (int)cr);
+    const bool stream_mode = grid > sms;   // two CTAs per SM by design
     if (bs64) {
-        if (has_zp) return launch_res_t<true, true>(map, p, grid, smem, flags, s);
-        return launch_res_t<true, false>(map, p, grid, smem, flags, s);
+        if (has_zp) return launch_res_t<true, true>(map, p, grid, smem, stream_mode, flags, s);
+        return launch_res_t<true, false>(map, p, grid, smem, stream_mode, flags, s);
     }
-    if (has_zp) return launch_res_t<false, true>(map, p, grid, smem, flags, s);
-    return launch_res_t<false, false>(map, p, grid, smem, flags, s);
+    if (has_zp) return launch_res_t<false, true>(map, p, grid, smem, stream_mode, flags, s);
+    return launch_res_t<false, false>(map, p, grid, smem, stream_mode, flags, s);
 }
 
 int read_res_status(unsigned *out, int clear) {
