@@ -61,7 +61,7 @@ namespace {
 constexpr int kWarps = 8;                   // warps that work; a launch may add idle ones (see below)
 constexpr int kThreads = kWarps * 32;
 constexpr int kMaxThreads = 16 * 32;
-constexpr int kMaxRegs = 112;               // register cap of the kernel (the launch shapes depend on it)
+constexpr int kMaxRegs = 96;                // register cap of the kernel (the launch shapes depend on it)
 constexpr int kRows = 16;
 constexpr int kBoxK = 256;                  // k per box: 8 blocks of 32 (4 of 64)
 constexpr int kBoxBytes = kRows * 128;
@@ -536,8 +536,9 @@ size_t res_smem_bytes(int depth, int nchunks) {
 // share the SM and double its part of the critical path.  Consecutive
 // launches therefore alternate between two shapes that cannot pair with
 // themselves but pair with each other: shape A asks for just over half of
-// the SM's shared memory, shape B for just over half of its registers (idle
-// warps widen it).  One A and one B fit on an SM; two of either do not.  A
+// the SM's shared memory, shape B for just over half of the registers of
+// each SM sub-partition (idle warps widen it; hence the kernel's register
+// cap).  One A and one B fit on an SM; two of either do not.  A
 // weight stream (the lm_head: two CTAs per SM by design) keeps the plain
 // shape.
 struct LaunchShape {
@@ -576,11 +577,17 @@ int launch_res_t(const CUtensorMap &map, const ResParams &p, int grid, size_t sm
     }
     LaunchShape shape{kThreads, smem};
     if (!stream_mode) {
-        const int R = regs[dev], half_rf = rf[dev] / 2;
-        const int wB = half_rf / (32 * R) + 1;                              // B: more than half the registers
+        // registers are allocated per SM sub-partition (four per SM; a CTA's
+        // warps go round-robin over them): cap = warps of this kernel one
+        // sub-partition holds; A has kWarps / 4 per sub-partition, B just over
+        // half of the cap, so A + B fits and B + B does not
+        const int R = regs[dev];
+        const int cap = (rf[dev] / 4) / (32 * R);
+        const int a = kWarps / 4, b = cap / 2 + 1;
         const size_t smemA = (size_t)(smem_sm[dev] - 2 * reserved[dev]) / 2 + 1024;   // A: more than half
-        const bool ok = 32 * R * (kWarps + wB) <= rf[dev] && 32 * wB <= kMaxThreads &&
+        const bool ok = a + b <= cap && 4 * b * 32 <= kMaxThreads &&
                         smemA + smem + 2 * (size_t)reserved[dev] <= (size_t)smem_sm[dev] && smem <= smemA;
+        const int wB = 4 * b;
         if (ok) {
             if (parity[dev].fetch_add(1u, std::memory_order_relaxed) & 1u)
                 shape.threads = 32 * wB;
