@@ -61,6 +61,7 @@ namespace {
 constexpr int kWarps = 8;                   // warps that work; a launch may add idle ones (see below)
 constexpr int kThreads = kWarps * 32;
 constexpr int kMaxThreads = 16 * 32;
+constexpr int kMaxXWords = 4;              // 16-byte words of x per thread: K <= 8192
 constexpr int kMaxRegs = 96;                // register cap of the kernel (the launch shapes depend on it)
 constexpr int kRows = 16;
 constexpr int kBoxK = 256;                  // k per box: 8 blocks of 32 (4 of 64)
@@ -294,9 +295,22 @@ __global__ void __maxnreg__(kMaxRegs)
     // four consecutive lanes, which add their sums by shuffles.
     {
         const half2 sixteenth = __floats2half2_rn(0.0625f, 0.0625f);
-        for (int u = tid; worker && u < p.nchunks * 4; u += kThreads) {
+        // every load first (up to four per thread), then the stores: one
+        // trip to L2 on the critical path, whatever K
+        uint4 vv[kMaxXWords];
+#pragma unroll
+        for (int r = 0; r < kMaxXWords; r++) {
+            const int u = tid + r * kThreads;
+            if (worker && u < p.nchunks * 4)
+                vv[r] = ldg_v4(p.X + 8 * u);
+        }
+#pragma unroll
+        for (int r = 0; r < kMaxXWords; r++) {
+            const int u = tid + r * kThreads;
+            if (!worker || u >= p.nchunks * 4)   // warp-uniform: K / 8 is a multiple of 32
+                break;
             const int j = u >> 2, w = u & 3;
-            const uint4 v = ldg_v4(p.X + 8 * u);
+            const uint4 v = vv[r];
             uint4 o;
             o.x = __byte_perm(v.x, v.z, 0x5410);
             o.y = h2_as_u32(__hmul2(u32_as_h2(__byte_perm(v.x, v.z, 0x7632)), sixteenth));
@@ -429,18 +443,31 @@ __global__ void __maxnreg__(kMaxRegs)
     __syncthreads();
 
     // ---- tiles cut between warps: the first warp slot holding a tile adds
-    // every slot holding it, in warp order, and stores the rows
+    // every slot holding it, in warp order, and stores the rows.  The slots'
+    // tiles are read once into registers, so the scan and the sum are not
+    // chains of dependent shared-memory reads.
     {
         const int sl = tid >> 4, row = tid & 15;   // 16 slots x 16 rows = 256 threads
-        const int tile = worker ? part_tile[sl] : -1;
-        bool leader = tile >= 0;
-        for (int q = 0; q < sl && leader; q++)
-            leader = part_tile[q] != tile;
+        int tiles[kWarps * 2];
+#pragma unroll
+        for (int q = 0; q < kWarps * 2; q += 4) {
+            const int4 t4 = *reinterpret_cast<const int4 *>(part_tile + q);
+            tiles[q] = t4.x; tiles[q + 1] = t4.y; tiles[q + 2] = t4.z; tiles[q + 3] = t4.w;
+        }
+        int tile = -1;
+#pragma unroll
+        for (int q = 0; q < kWarps * 2; q++)
+            if (q == sl) tile = tiles[q];
+        bool leader = worker && tile >= 0;
+#pragma unroll
+        for (int q = 0; q < kWarps * 2; q++)
+            if (q < sl && tiles[q] == tile) leader = false;
         if (leader && p.swiglu) {   // rows < 8: the gates; row + 8: their ups
             if (row < 8) {
                 float gv = 0.f, uv = 0.f;
-                for (int q = sl; q < kWarps * 2; q++)
-                    if (part_tile[q] == tile) {
+#pragma unroll
+                for (int q = 0; q < kWarps * 2; q++)
+                    if (q >= sl && tiles[q] == tile) {
                         gv += part[q * kRows + row];
                         uv += part[q * kRows + row + 8];
                     }
@@ -449,8 +476,9 @@ __global__ void __maxnreg__(kMaxRegs)
             }
         } else if (leader) {
             float v = 0.f;
-            for (int q = sl; q < kWarps * 2; q++)
-                if (part_tile[q] == tile)
+#pragma unroll
+            for (int q = 0; q < kWarps * 2; q++)
+                if (q >= sl && tiles[q] == tile)
                     v += part[q * kRows + row];
             const int n = tile * kRows + row;
             if (n < p.N && !dead) {
@@ -627,7 +655,8 @@ int launch_gemv_resident(const void *X, const uint8_t *packed, const void *scale
                          int K, int bs, unsigned flags, cudaStream_t s, int32_t *ids, float *max_out,
                          void *workspace, int swiglu) {
     const bool bs64 = (bs == 64), has_zp = (zp != nullptr);
-    if (K % kBoxK != 0 || (bs64 && has_zp && K % 512 != 0) || !aligned(scales, bs64 ? 8 : 16) ||
+    if (K % kBoxK != 0 || K > kMaxXWords * kThreads * 8 || (bs64 && has_zp && K % 512 != 0) ||
+        !aligned(scales, bs64 ? 8 : 16) ||
         (has_zp && !aligned(zp, 4)))
         return 1;   // not a shape this kernel serves
     ResParams p;
