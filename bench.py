@@ -325,7 +325,9 @@ def run_reference(args, world, rank):
 
 def profile_part(args, dev, ranks):
     """Small cases for ncu captures: the lm_head GEMV alone (180 MB of weights,
-    larger than L2) or layer 0 of the prefill at M = 1024 on the tensor cores."""
+    larger than L2), layer 0 of the decode step and the lm_head (8 dependent
+    GEMV launches, as in the step), or layer 0 of the prefill at M = 1024 on
+    the tensor cores."""
     import torch
 
     import workloads
@@ -335,6 +337,9 @@ def profile_part(args, dev, ranks):
     if args.only == "lmhead":
         lin = [l for l in workloads.config_linears("qwen3_1p7b_decode") if l.name == "lm_head"]
         M, kind = 1, "gemv"
+    elif args.only == "decode-layer":
+        lin = [l for l in workloads.config_linears("qwen3_1p7b_decode") if l.layer in (0, 28)]
+        M, kind = 1, "gemv"
     else:
         lin = [l for l in workloads.config_linears("qwen3_1p7b_prefill") if l.layer == 0]
         M, kind = args.m, "gemm"
@@ -343,7 +348,7 @@ def profile_part(args, dev, ranks):
         W = workloads.weight(cfg["seed"], l.layer, l.proj, l.N, l.K, True, device=dev)
         lins.append(QLinear.quantize(W, cfg["bs"], True, torch.float16, name=l.name))
         del W
-    p = Pass(lins, M, kind, torch.float16, pdl=False)
+    p = Pass(lins, M, kind, torch.float16, pdl=(args.only == "decode-layer"))
     fill(p, cfg["seed"])
     torch.cuda.synchronize()
     torch.cuda.empty_cache()    # keep only the live buffers on the device
@@ -613,7 +618,7 @@ def run_gpu(args, world, rank, local):
     import int4_block_quantized_matmulnbits_b200 as mnb
     from int4_block_quantized_matmulnbits_b200.step import Pass
 
-    if args.only in ("lmhead", "gemm-layer"):
+    if args.only in ("lmhead", "gemm-layer", "decode-layer"):
         profile_part(args, dev, ranks)
         ranks.close()
         return
@@ -903,7 +908,7 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="mnb", choices=["mnb", "reference"])
-    ap.add_argument("--only", default="", choices=["", "decode", "lmhead", "gemm-layer"],
+    ap.add_argument("--only", default="", choices=["", "decode", "lmhead", "gemm-layer", "decode-layer"],
                     help="profiling modes: run one part only and print no JSON line")
     ap.add_argument("--m", type=int, default=1024, help="tokens of the gemm-layer profiling mode")
     args = ap.parse_args()

@@ -58,6 +58,22 @@ __device__ unsigned g_res_status = 0;
 
 namespace {
 
+// Index checks of the debug build (MNB_DEVICE_CHECKS, built as libmnb_debug.so):
+// an index outside [0, bound) sets bit 4 of the status word and is replaced by
+// 0, so the access stays inside its buffer; nothing traps.  The release build
+// compiles them away.
+__device__ __forceinline__ int checked(int idx, int bound) {
+#ifdef MNB_DEVICE_CHECKS
+    if (idx < 0 || idx >= bound) {
+        atomicOr(&g_res_status, 16u);
+        return 0;
+    }
+#else
+    (void)bound;
+#endif
+    return idx;
+}
+
 constexpr int kWarps = 8;                   // warps of the plain launch shape; others have more (launch_res_t)
 constexpr int kThreads = kWarps * 32;
 constexpr int kMaxWarps = 12;
@@ -179,11 +195,11 @@ __device__ __forceinline__ void cursor_next(const ResParams &p, IssueCursor &q, 
 // Rows past N get no parameters (their sums are never stored).  Every lane
 // arrives on the slot's barrier once its copies have landed.
 template <bool BS64, bool ZP>
-__device__ __forceinline__ void issue(const CUtensorMap *wmap, const IssueCursor &q, uint32_t box_dst,
-                                      uint32_t par_dst, uint32_t full, int lane) {
+__device__ __forceinline__ void issue(const CUtensorMap *wmap, const ResParams &p, const IssueCursor &q,
+                                      uint32_t box_dst, uint32_t par_dst, uint32_t full, int lane) {
     if (lane == 0) {
         mbar_expect_tx(full, kBoxBytes);
-        tma_load_2d(box_dst, wmap, full, q.box * 128, q.tile * kRows);
+        tma_load_2d(box_dst, wmap, full, checked(q.box, p.nbx) * 128, checked(q.tile, p.ntiles) * kRows);
     }
     if (q.row_ok) {
         if (lane < 16) {
@@ -275,7 +291,7 @@ __global__ void __maxnreg__(kMaxRegs)
     IssueCursor ic;
     cursor_at_tile<BS64, ZP>(p, ic, t0 + tl0, box0, lane);
     auto request = [&]() {
-        issue<BS64, ZP>(&wmap, ic, my_box + islot * kBoxBytes, my_par + islot * kParBytes, my_bars + 8 * islot, lane);
+        issue<BS64, ZP>(&wmap, p, ic, my_box + islot * kBoxBytes, my_par + islot * kParBytes, my_bars + 8 * islot, lane);
         cursor_next<BS64, ZP>(p, ic, lane);
         ++iu;
         if (++islot == D) islot = 0;
@@ -349,9 +365,9 @@ __global__ void __maxnreg__(kMaxRegs)
         }
         slot_wait(my_bars + 8 * cslot, (uint32_t)cph, dead);
         dead = __any_sync(0xffffffffu, dead);   // one verdict per warp: it issues refills together
-        const unsigned char *bx = my_box_ptr + cslot * kBoxBytes;
-        const unsigned char *par = my_par_ptr + cslot * kParBytes;
-        const float4 pqv = *reinterpret_cast<const float4 *>(pq + box * 8 + 2 * c);   // P, Q of columns 2c, 2c+1
+        const unsigned char *bx = my_box_ptr + checked(cslot, D) * kBoxBytes;
+        const unsigned char *par = my_par_ptr + checked(cslot, D) * kParBytes;
+        const float4 pqv = *reinterpret_cast<const float4 *>(pq + checked(box * 8 + 2 * c, p.nchunks - 1));   // P, Q of columns 2c, 2c+1
         // four independent MMA chains (half of the box x parity of the word),
         // the first started from -P: the 16 MMAs of a box form chains of four
         float acc4[4][4] = {{-pqv.x, -pqv.z, -pqv.x, -pqv.z}, {0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f},
@@ -363,7 +379,7 @@ __global__ void __maxnreg__(kMaxRegs)
             const uint4 vb = *reinterpret_cast<const uint4 *>(bx + (g + 8) * 128 + ((chunk ^ g) << 4));
             // x of chunk `chunk` goes to column `chunk` only: the thread whose
             // column that is (g == chunk) reads it, every other thread zeros
-            const unsigned char *xa = (hm == h) ? xs + (box * 8 + chunk) * kChunk : zchunk;
+            const unsigned char *xa = (hm == h) ? xs + checked(box * 8 + chunk, p.nchunks) * kChunk : zchunk;
             const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
             const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
@@ -428,13 +444,13 @@ __global__ void __maxnreg__(kMaxRegs)
                 }
             } else {
                 // a partial: the first segment of the run in slot 0, the last in slot 1
-                const int s = (nseg == 0) ? 0 : 1;
+                const int s = checked(warp * 2 + ((nseg == 0) ? 0 : 1), kMaxWarps * 2);
                 if (c == 0) {
-                    part[(warp * 2 + s) * kRows + g] = ya;
-                    part[(warp * 2 + s) * kRows + g + 8] = yb;
+                    part[s * kRows + g] = ya;
+                    part[s * kRows + g + 8] = yb;
                 }
                 if (lane == 0)
-                    part_tile[warp * 2 + s] = tile;
+                    part_tile[s] = tile;
             }
             ++nseg;
         }
@@ -737,7 +753,7 @@ int read_res_status(unsigned *out, int clear) {
     }
     if (e != cudaSuccess)
         return fail(MNB_ERR_CUDA, "mnb_device_status: %s", cudaGetErrorString(e));
-    *out |= v;   // bit 0, as the other decode kernels
+    *out |= v;   // bit 0, as the other decode kernels; bit 4: an index check of the debug build
     return MNB_OK;
 }
 
