@@ -628,6 +628,15 @@ def run_gpu(args, world, rank, local):
     tc_burst = float(peaks["bf16_tflops"])
     tc_sust = float(peaks.get("bf16_tflops_sustained", tc_burst))
 
+    if args.only == "prefill":   # profiling mode: the M = 1024 prefill pass alone
+        cfg, lins = build_model("qwen3_1p7b_decode", dev, lm_head=False)
+        pp = Pass(lins, 1024, "gemm", torch.float16, pdl=True)
+        fill(pp, cfg["seed"] + 1024)
+        pp.capture()
+        timed_replays(pp, args.steps, args.warmup, ranks, "prefill")
+        ranks.close()
+        return
+
     # ---- decode step, M = 1 (the headline)
     cfg, lins = build_model("qwen3_1p7b_decode", dev)
     dec = Pass(lins, 1, "gemv", torch.float16, pdl=True)
@@ -908,7 +917,7 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="mnb", choices=["mnb", "reference"])
-    ap.add_argument("--only", default="", choices=["", "decode", "lmhead", "gemm-layer", "decode-layer"],
+    ap.add_argument("--only", default="", choices=["", "decode", "prefill", "lmhead", "gemm-layer", "decode-layer"],
                     help="profiling modes: run one part only and print no JSON line")
     ap.add_argument("--m", type=int, default=1024, help="tokens of the gemm-layer profiling mode")
     args = ap.parse_args()

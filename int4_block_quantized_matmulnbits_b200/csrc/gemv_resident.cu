@@ -8,7 +8,7 @@
 // it.  Most move 1-7 MB of weights -- well under 2 us of HBM time -- so what
 // costs is the critical path from "previous kernel done" to "this kernel's y
 // stored".  This kernel is built to keep that path short:
-//   * Half an SM per CTA (8 warps, <= 128 registers, ~110 KB of shared
+//   * Half an SM per CTA (8 working warps, <= 96 registers, ~110 KB of shared
 //     memory), one CTA per SM.  While kernel i runs, the CTAs of kernel i+1
 //     (launched early by programmatic dependent launch) sit on the other half
 //     of every SM and pull ALL of their weights into shared memory: each warp
@@ -20,8 +20,10 @@
 //   * Work split: CTA b owns a contiguous run of 16-row tiles; its (tile, box)
 //     units are cut into one contiguous run per warp.  Tiles a warp covers
 //     whole are stored from registers; the partial sums of tiles cut between
-//     warps meet in shared memory and are added in warp order (deterministic).
-//     Nothing crosses CTAs: no cluster, no atomics, no global scratch.
+//     warps meet in shared memory and are added in warp order.  Both launch
+//     shapes (below) have the same 8 working warps, so every call cuts and
+//     adds the sums alike: the result is the same, bit for bit, from call to
+//     call.  Nothing crosses CTAs: no cluster, no atomics, no global scratch.
 //   * Zero point and scale are applied per block AFTER the tensor core, not
 //     per weight.  The MMA (mma.sync m16n8k16, fp32 accumulation) takes the
 //     raw codes: (nibble | 0x6400) is the fp16 1024+q exactly for a low
@@ -41,6 +43,9 @@
 //   * Consecutive launches alternate between two resource shapes that cannot
 //     share an SM with themselves but can with each other, so the block
 //     scheduler never puts two CTAs of one launch on an SM (launch_res_t).
+//     The second shape's extra warps only widen it.  (Giving them units too
+//     was measured slower over the decode step, and would make the two
+//     shapes cut the sums differently.)
 // Every mbarrier wait is bounded in time; past the limit the kernel records
 // the failure in the device status word, lets its copies in flight land and
 // exits.
@@ -74,11 +79,10 @@ __device__ __forceinline__ int checked(int idx, int bound) {
     return idx;
 }
 
-constexpr int kWarps = 8;                   // warps of the plain launch shape; others have more (launch_res_t)
+constexpr int kWarps = 8;                   // warps that work; a launch may add idle ones (see below)
 constexpr int kThreads = kWarps * 32;
-constexpr int kMaxWarps = 12;
-constexpr int kMaxThreads = kMaxWarps * 32;
-constexpr int kMaxXWords = 4;              // 16-byte words of x per thread of the 8-warp shape: K <= 8192
+constexpr int kMaxThreads = 16 * 32;
+constexpr int kMaxXWords = 4;              // 16-byte words of x per thread: K <= 8192
 constexpr int kMaxRegs = 96;                // register cap of the kernel (the launch shapes depend on it)
 constexpr int kRows = 16;
 constexpr int kBoxK = 256;                  // k per box: 8 blocks of 32 (4 of 64)
@@ -252,35 +256,37 @@ __global__ void __maxnreg__(kMaxRegs)
     // partial sums | their tiles | barriers
     const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
     unsigned char *bp = smem_raw + (base - smem_u32(smem_raw));
-    const int W = blockDim.x >> 5;        // warps of this launch, all of them working
-    unsigned char *pars = bp + W * D * kBoxBytes;
-    unsigned char *xs = pars + W * D * kParBytes;
+    unsigned char *pars = bp + kWarps * D * kBoxBytes;
+    unsigned char *xs = pars + kWarps * D * kParBytes;
     unsigned char *zchunk = xs + p.nchunks * kChunk;
     float2 *pq = reinterpret_cast<float2 *>(zchunk + kChunk);
     float *part = reinterpret_cast<float *>(pq + p.nchunks);      // [warp][2 slots][16 rows]
-    int *part_tile = reinterpret_cast<int *>(part + kMaxWarps * 2 * kRows);
-    uint2 *wbest = reinterpret_cast<uint2 *>(part_tile + kMaxWarps * 2);   // greedy decoding: per warp
-    const uint32_t bars = smem_u32(wbest + kMaxWarps);
+    int *part_tile = reinterpret_cast<int *>(part + kWarps * 2 * kRows);
+    uint2 *wbest = reinterpret_cast<uint2 *>(part_tile + kWarps * 2);   // greedy decoding: per warp
+    const uint32_t bars = smem_u32(wbest + kWarps);
     const uint32_t my_box = base + (uint32_t)(warp * D * kBoxBytes);
     const unsigned char *my_box_ptr = bp + warp * D * kBoxBytes;
     const uint32_t my_par = smem_u32(pars) + (uint32_t)(warp * D * kParBytes);
     const unsigned char *my_par_ptr = pars + warp * D * kParBytes;
     const uint32_t my_bars = bars + (uint32_t)(warp * D * 8);
-    const bool worker = true;   // every warp of the launch works
+    // warps beyond kWarps only widen the launch (so that two CTAs of one
+    // launch cannot share an SM): no units, no barriers, no slots; they take
+    // part in the CTA barriers only
+    const bool worker = warp < kWarps;
 
     // this CTA's tiles and this warp's run of (tile, box) units
     const int cta = blockIdx.x;
     const int Tc = p.tq + (cta < p.tr ? 1 : 0);
     const int t0 = cta * p.tq + (cta < p.tr ? cta : p.tr);
     const int U = Tc * p.nbx;
-    const int u0 = warp * U / W, u1 = (warp + 1) * U / W;
+    const int u0 = (worker ? warp : kWarps) * U / kWarps, u1 = (worker ? warp + 1 : kWarps) * U / kWarps;
 
     if (worker && lane == 0) {
         for (int d = 0; d < D; d++)
             mbar_init(my_bars + 8 * d, 33);   // lane 0's expect_tx + one cp.async arrival per lane
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (tid < kMaxWarps * 2)
+    if (tid < kWarps * 2)
         part_tile[tid] = -1;
     __syncwarp();
 
@@ -315,13 +321,13 @@ __global__ void __maxnreg__(kMaxRegs)
         uint4 vv[kMaxXWords];
 #pragma unroll
         for (int r = 0; r < kMaxXWords; r++) {
-            const int u = tid + r * (int)blockDim.x;
+            const int u = tid + r * kThreads;
             if (worker && u < p.nchunks * 4)
                 vv[r] = ldg_v4(p.X + 8 * u);
         }
 #pragma unroll
         for (int r = 0; r < kMaxXWords; r++) {
-            const int u = tid + r * (int)blockDim.x;
+            const int u = tid + r * kThreads;
             if (!worker || u >= p.nchunks * 4)   // warp-uniform: K / 8 is a multiple of 32
                 break;
             const int j = u >> 2, w = u & 3;
@@ -444,7 +450,7 @@ __global__ void __maxnreg__(kMaxRegs)
                 }
             } else {
                 // a partial: the first segment of the run in slot 0, the last in slot 1
-                const int s = checked(warp * 2 + ((nseg == 0) ? 0 : 1), kMaxWarps * 2);
+                const int s = checked(warp * 2 + ((nseg == 0) ? 0 : 1), kWarps * 2);
                 if (c == 0) {
                     part[s * kRows + g] = ya;
                     part[s * kRows + g + 8] = yb;
@@ -462,26 +468,26 @@ __global__ void __maxnreg__(kMaxRegs)
     // tiles are read once into registers, so the scan and the sum are not
     // chains of dependent shared-memory reads.
     {
-        const int sl = tid >> 4, row = tid & 15;   // 2 W slots x 16 rows = the CTA's threads
-        int tiles[kMaxWarps * 2];
+        const int sl = tid >> 4, row = tid & 15;   // 16 slots x 16 rows = 256 threads
+        int tiles[kWarps * 2];
 #pragma unroll
-        for (int q = 0; q < kMaxWarps * 2; q += 4) {
+        for (int q = 0; q < kWarps * 2; q += 4) {
             const int4 t4 = *reinterpret_cast<const int4 *>(part_tile + q);
             tiles[q] = t4.x; tiles[q + 1] = t4.y; tiles[q + 2] = t4.z; tiles[q + 3] = t4.w;
         }
         int tile = -1;
 #pragma unroll
-        for (int q = 0; q < kMaxWarps * 2; q++)
+        for (int q = 0; q < kWarps * 2; q++)
             if (q == sl) tile = tiles[q];
         bool leader = worker && tile >= 0;
 #pragma unroll
-        for (int q = 0; q < kMaxWarps * 2; q++)
+        for (int q = 0; q < kWarps * 2; q++)
             if (q < sl && tiles[q] == tile) leader = false;
         if (leader && p.swiglu) {   // rows < 8: the gates; row + 8: their ups
             if (row < 8) {
                 float gv = 0.f, uv = 0.f;
 #pragma unroll
-                for (int q = 0; q < kMaxWarps * 2; q++)
+                for (int q = 0; q < kWarps * 2; q++)
                     if (q >= sl && tiles[q] == tile) {
                         gv += part[q * kRows + row];
                         uv += part[q * kRows + row + 8];
@@ -492,7 +498,7 @@ __global__ void __maxnreg__(kMaxRegs)
         } else if (leader) {
             float v = 0.f;
 #pragma unroll
-            for (int q = 0; q < kMaxWarps * 2; q++)
+            for (int q = 0; q < kWarps * 2; q++)
                 if (q >= sl && tiles[q] == tile)
                     v += part[q * kRows + row];
             const int n = tile * kRows + row;
@@ -520,7 +526,7 @@ __global__ void __maxnreg__(kMaxRegs)
         if (tid == 0) {
             float v = -INFINITY;
             int i = 0x7fffffff;
-            for (int w = 0; w < W; w++)
+            for (int w = 0; w < kWarps; w++)
                 keep_best(__uint_as_float(wbest[w].x), (int)wbest[w].y, v, i);
             p.ws_part[blockIdx.x] = make_uint2(__float_as_uint(v), (unsigned)i);
             __threadfence();
@@ -531,7 +537,7 @@ __global__ void __maxnreg__(kMaxRegs)
             __threadfence();
             float v = -INFINITY;
             int i = 0x7fffffff;
-            for (int b = tid; worker && b < (int)gridDim.x; b += (int)blockDim.x) {
+            for (int b = tid; worker && b < (int)gridDim.x; b += kThreads) {
                 const uint2 e = __ldcg(p.ws_part + b);
                 keep_best(__uint_as_float(e.x), (int)e.y, v, i);
             }
@@ -545,7 +551,7 @@ __global__ void __maxnreg__(kMaxRegs)
                 wbest[warp] = make_uint2(__float_as_uint(v), (unsigned)i);
             __syncthreads();
             if (tid == 0) {
-                for (int w = 1; w < W; w++)
+                for (int w = 1; w < kWarps; w++)
                     keep_best(__uint_as_float(wbest[w].x), (int)wbest[w].y, v, i);
                 p.ids[0] = i;
                 if (p.max_out)
@@ -568,19 +574,9 @@ __global__ void __maxnreg__(kMaxRegs)
     }
 }
 
-size_t res_smem_bytes(int warps, int depth, int nchunks) {
-    return 1024 + (size_t)warps * depth * (kBoxBytes + kParBytes + 8) + (size_t)nchunks * (kChunk + 8) + kChunk +
-           (size_t)kMaxWarps * 2 * (kRows * 4 + 4) + (size_t)kMaxWarps * 8;
-}
-
-// The deepest ring, up to the most units a warp owns, for `warps` warps
-// within `budget` bytes; 0 when none fits.
-int res_depth(int warps, int Umax, int nchunks, size_t budget) {
-    const int per_warp = (Umax + warps - 1) / warps;
-    int depth = per_warp < kMaxDepth ? (per_warp < 2 ? 2 : per_warp) : kMaxDepth;
-    while (depth > 2 && res_smem_bytes(warps, depth, nchunks) > budget)
-        --depth;
-    return res_smem_bytes(warps, depth, nchunks) <= budget ? depth : 0;
+size_t res_smem_bytes(int depth, int nchunks) {
+    return 1024 + (size_t)kWarps * depth * (kBoxBytes + kParBytes + 8) + (size_t)nchunks * (kChunk + 8) + kChunk +
+           (size_t)kWarps * 2 * (kRows * 4 + 4) + (size_t)kWarps * 8;
 }
 
 // Launch shapes.  The CTAs of kernel i+1 are placed while kernel i runs;
@@ -600,7 +596,7 @@ struct LaunchShape {
 };
 
 template <bool BS64, bool ZP>
-int launch_res_t(const CUtensorMap &map, ResParams p, int grid, int Umax, bool stream_mode, unsigned flags,
+int launch_res_t(const CUtensorMap &map, const ResParams &p, int grid, size_t smem, bool stream_mode, unsigned flags,
                  cudaStream_t s) {
     auto fn = gemv_resident_kernel<BS64, ZP>;
     static int regs[kMaxDevices] = {}, smem_sm[kMaxDevices] = {}, reserved[kMaxDevices] = {}, rf[kMaxDevices] = {};
@@ -628,35 +624,26 @@ int launch_res_t(const CUtensorMap &map, ResParams p, int grid, int Umax, bool s
             regs[dev] = (a.numRegs + 7) & ~7;
         }
     }
-    // the plain shape: 8 warps, the deepest ring within the budget
-    int depth = res_depth(kWarps, Umax, p.nchunks, (size_t)kSmemBudget);
-    if (!depth)
-        return 1;
-    LaunchShape shape{kThreads, res_smem_bytes(kWarps, depth, p.nchunks)};
+    LaunchShape shape{kThreads, smem};
     if (!stream_mode) {
         // registers are allocated per SM sub-partition (four per SM; a CTA's
         // warps go round-robin over them): cap = warps of this kernel one
-        // sub-partition holds; A has 8 warps (2 per sub-partition), B just over
-        // half of the cap, so A + B fits and B + B does not.  B's extra warps
-        // take units too.
+        // sub-partition holds; A has kWarps / 4 per sub-partition, B just over
+        // half of the cap, so A + B fits and B + B does not
         const int R = regs[dev];
         const int cap = (rf[dev] / 4) / (32 * R);
-        const int a = kWarps / 4, b = cap / 2 + 1, wB = 4 * b;
+        const int a = kWarps / 4, b = cap / 2 + 1;
         const size_t smemA = (size_t)(smem_sm[dev] - 2 * reserved[dev]) / 2 + 1024;   // A: more than half
-        const size_t budgetB = (size_t)smem_sm[dev] - 2 * (size_t)reserved[dev] - smemA;
-        const int depthB = (wB <= kMaxWarps) ? res_depth(wB, Umax, p.nchunks, budgetB < (size_t)kSmemBudget ? budgetB : (size_t)kSmemBudget) : 0;
-        const bool ok = a + b <= cap && depthB && shape.smem <= smemA;
+        const bool ok = a + b <= cap && 4 * b * 32 <= kMaxThreads &&
+                        smemA + smem + 2 * (size_t)reserved[dev] <= (size_t)smem_sm[dev] && smem <= smemA;
+        const int wB = 4 * b;
         if (ok) {
-            if (parity[dev].fetch_add(1u, std::memory_order_relaxed) & 1u) {
+            if (parity[dev].fetch_add(1u, std::memory_order_relaxed) & 1u)
                 shape.threads = 32 * wB;
-                depth = depthB;
-                shape.smem = res_smem_bytes(wB, depthB, p.nchunks);
-            } else {
+            else
                 shape.smem = smemA;
-            }
         }
     }
-    p.depth = depth;
     static int configured[kMaxDevices] = {};
     {
         cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(fn), (int)shape.smem, configured);
@@ -712,15 +699,22 @@ int launch_gemv_resident(const void *X, const uint8_t *packed, const void *scale
     const int grid = p.ntiles < sms ? p.ntiles : (p.ntiles > 16 * sms ? 2 * sms : sms);
     p.tq = p.ntiles / grid;
     p.tr = p.ntiles % grid;
-    const int Umax = (p.tq + (p.tr ? 1 : 0)) * p.nbx;   // the most units of any CTA
-    if (!res_depth(kWarps, Umax, p.nchunks, (size_t)kSmemBudget))
+    // the deepest ring (up to the most units a warp owns) that keeps two CTAs per SM
+    const int Umax = (p.tq + (p.tr ? 1 : 0)) * p.nbx;
+    const int per_warp = (Umax + kWarps - 1) / kWarps;
+    int depth = per_warp < kMaxDepth ? (per_warp < 2 ? 2 : per_warp) : kMaxDepth;
+    while (depth > 2 && res_smem_bytes(depth, p.nchunks) > (size_t)kSmemBudget)
+        --depth;
+    if (res_smem_bytes(depth, p.nchunks) > (size_t)kSmemBudget)
         return 1;
+    p.depth = depth;
     p.argmax = ids ? 1 : 0;
     p.swiglu = swiglu;
     p.ids = ids;
     p.max_out = max_out;
     p.ws_count = static_cast<unsigned *>(workspace);
     p.ws_part = workspace ? reinterpret_cast<uint2 *>(static_cast<unsigned char *>(workspace) + 256) : nullptr;
+    const size_t smem = res_smem_bytes(depth, p.nchunks);
 
     EncodeTiledFn encode = tensor_map_encoder();
     if (!encode)
@@ -737,11 +731,11 @@ int launch_gemv_resident(const void *X, const uint8_t *packed, const void *scale
         return fail(MNB_ERR_CUDA, "mnb_gemv: cuTensorMapEncodeTiled failed (%d)", (int)cr);
     const bool stream_mode = grid > sms;   // two CTAs per SM by design
     if (bs64) {
-        if (has_zp) return launch_res_t<true, true>(map, p, grid, Umax, stream_mode, flags, s);
-        return launch_res_t<true, false>(map, p, grid, Umax, stream_mode, flags, s);
+        if (has_zp) return launch_res_t<true, true>(map, p, grid, smem, stream_mode, flags, s);
+        return launch_res_t<true, false>(map, p, grid, smem, stream_mode, flags, s);
     }
-    if (has_zp) return launch_res_t<false, true>(map, p, grid, Umax, stream_mode, flags, s);
-    return launch_res_t<false, false>(map, p, grid, Umax, stream_mode, flags, s);
+    if (has_zp) return launch_res_t<false, true>(map, p, grid, smem, stream_mode, flags, s);
+    return launch_res_t<false, false>(map, p, grid, smem, stream_mode, flags, s);
 }
 
 int read_res_status(unsigned *out, int clear) {

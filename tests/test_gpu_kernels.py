@@ -166,6 +166,30 @@ def test_gemv_resident_one_token(mnb, cuda_dev, N, K, bs, has_zp):
     assert mnb.mnb_device_status() == 0
 
 
+@pytest.mark.parametrize("N,K,bs,has_zp", [(2048, 2048, 32, True), (6144, 2048, 32, True),
+                                           (2048, 6144, 32, True), (4736, 3072, 64, True), (777, 512, 64, False)])
+def test_gemv_resident_is_deterministic(mnb, cuda_dev, N, K, bs, has_zp):
+    # consecutive one-token launches alternate between two launch shapes with
+    # different warp counts; the sums are cut at the same places in both, so
+    # every call returns the same bits (plain and with the SwiGLU epilogue)
+    rng = np.random.default_rng(N + K + bs)
+    packed, scales, zp = (to_dev(a, cuda_dev) for a in random_packed(rng, N, K, bs, has_zp, np.float16))
+    X = torch.randn((1, K), generator=torch.Generator().manual_seed(K + 1)).half().to(cuda_dev)
+    for swiglu in ((False, True) if N % 16 == 0 else (False,)):
+        outs = []
+        for _ in range(5):
+            Y = torch.empty((1, N // 2 if swiglu else N), dtype=torch.float16, device=cuda_dev)
+            if swiglu:
+                mnb.mnb_gemv_swiglu(X, packed, scales, zp, Y, 1, N, K, bs)
+            else:
+                mnb.mnb_gemv(X, packed, scales, zp, Y, 1, N, K, bs)
+            outs.append(Y)
+        torch.cuda.synchronize()
+        for Y in outs[1:]:
+            assert torch.equal(Y, outs[0])
+    assert mnb.mnb_device_status() == 0
+
+
 def test_gemv_resident_large_inputs_and_pdl(mnb, cuda_dev):
     # activations far from unit scale (the raw-code sums grow with |x|), and a
     # chain of dependent PDL launches: each GEMV reads the previous one's output
