@@ -589,6 +589,18 @@ def bench_gptq(dev, ranks, with_oracle):
            "hessian_ms": round(float(t[0]), 3), "prepare_ms": round(float(t[1]), 3),
            "quantize_ms": round(float(t[2]), 3), "total_ms": round(float(t.sum()), 3),
            "weights_per_s": round(N * K / (float(t.sum()) * 1e-3), 1)}
+    # quality: mean squared output error over the calibration inputs, GPTQ's
+    # codes against round-to-nearest ones of the same weights (both
+    # dequantized by the library)
+    rp, rs, rz = torch.empty_like(packed), torch.empty_like(scales), torch.empty_like(zp)
+    mnb.mnb_quantize_rtn(W, N, K, bs, True, rp, rs, rz)
+    Wd = torch.empty((N, K), dtype=torch.float32, device=dev)
+    errs = []
+    for cp, cs, cz in ((packed, scales, zp), (rp, rs, rz)):
+        mnb.mnb_dequantize(cp, cs, cz, N, K, bs, Wd)
+        errs.append(float(((X.float() @ (W - Wd).T) ** 2).mean()))
+    out["output_mse"] = {"gptq": errs[0], "rtn": errs[1], "ratio": round(errs[0] / errs[1], 4)}
+    del Wd
     if with_oracle:
         import oracle
 

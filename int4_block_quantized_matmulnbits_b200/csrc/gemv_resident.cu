@@ -81,9 +81,12 @@ __device__ __forceinline__ int checked(int idx, int bound) {
 
 constexpr int kWarps = 8;                   // warps that work; a launch may add idle ones (see below)
 constexpr int kThreads = kWarps * 32;
+constexpr int kStreamWarps = 20;            // working warps of a weight stream's CTA
+constexpr int kStreamCtas = 1;              // ... and its CTAs per SM
 constexpr int kMaxThreads = 16 * 32;
 constexpr int kMaxXWords = 4;              // 16-byte words of x per thread: K <= 8192
 constexpr int kMaxRegs = 96;                // register cap of the kernel (the launch shapes depend on it)
+constexpr int kMaxRegsWide = 80;            // ... of a CTA of more than 20 working warps
 constexpr int kRows = 16;
 constexpr int kBoxK = 256;                  // k per box: 8 blocks of 32 (4 of 64)
 constexpr int kBoxBytes = kRows * 128;
@@ -244,8 +247,8 @@ __device__ __forceinline__ float2 zp_pair(const unsigned char *par, int row, int
     return make_float2(z, z);
 }
 
-template <bool BS64, bool ZP>
-__global__ void __maxnreg__(kMaxRegs)
+template <bool BS64, bool ZP, int NW>
+__global__ void __maxnreg__(NW > 20 ? kMaxRegsWide : kMaxRegs)
     gemv_resident_kernel(const __grid_constant__ CUtensorMap wmap, const ResParams p) {
     extern __shared__ unsigned char smem_raw[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -256,37 +259,37 @@ __global__ void __maxnreg__(kMaxRegs)
     // partial sums | their tiles | barriers
     const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
     unsigned char *bp = smem_raw + (base - smem_u32(smem_raw));
-    unsigned char *pars = bp + kWarps * D * kBoxBytes;
-    unsigned char *xs = pars + kWarps * D * kParBytes;
+    unsigned char *pars = bp + NW * D * kBoxBytes;
+    unsigned char *xs = pars + NW * D * kParBytes;
     unsigned char *zchunk = xs + p.nchunks * kChunk;
     float2 *pq = reinterpret_cast<float2 *>(zchunk + kChunk);
     float *part = reinterpret_cast<float *>(pq + p.nchunks);      // [warp][2 slots][16 rows]
-    int *part_tile = reinterpret_cast<int *>(part + kWarps * 2 * kRows);
-    uint2 *wbest = reinterpret_cast<uint2 *>(part_tile + kWarps * 2);   // greedy decoding: per warp
-    const uint32_t bars = smem_u32(wbest + kWarps);
+    int *part_tile = reinterpret_cast<int *>(part + NW * 2 * kRows);
+    uint2 *wbest = reinterpret_cast<uint2 *>(part_tile + NW * 2);   // greedy decoding: per warp
+    const uint32_t bars = smem_u32(wbest + NW);
     const uint32_t my_box = base + (uint32_t)(warp * D * kBoxBytes);
     const unsigned char *my_box_ptr = bp + warp * D * kBoxBytes;
     const uint32_t my_par = smem_u32(pars) + (uint32_t)(warp * D * kParBytes);
     const unsigned char *my_par_ptr = pars + warp * D * kParBytes;
     const uint32_t my_bars = bars + (uint32_t)(warp * D * 8);
-    // warps beyond kWarps only widen the launch (so that two CTAs of one
+    // warps beyond NW only widen the launch (so that two CTAs of one
     // launch cannot share an SM): no units, no barriers, no slots; they take
     // part in the CTA barriers only
-    const bool worker = warp < kWarps;
+    const bool worker = warp < NW;
 
     // this CTA's tiles and this warp's run of (tile, box) units
     const int cta = blockIdx.x;
     const int Tc = p.tq + (cta < p.tr ? 1 : 0);
     const int t0 = cta * p.tq + (cta < p.tr ? cta : p.tr);
     const int U = Tc * p.nbx;
-    const int u0 = (worker ? warp : kWarps) * U / kWarps, u1 = (worker ? warp + 1 : kWarps) * U / kWarps;
+    const int u0 = (worker ? warp : NW) * U / NW, u1 = (worker ? warp + 1 : NW) * U / NW;
 
     if (worker && lane == 0) {
         for (int d = 0; d < D; d++)
             mbar_init(my_bars + 8 * d, 33);   // lane 0's expect_tx + one cp.async arrival per lane
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (tid < kWarps * 2)
+    if (tid < NW * 2)
         part_tile[tid] = -1;
     __syncwarp();
 
@@ -321,13 +324,13 @@ __global__ void __maxnreg__(kMaxRegs)
         uint4 vv[kMaxXWords];
 #pragma unroll
         for (int r = 0; r < kMaxXWords; r++) {
-            const int u = tid + r * kThreads;
+            const int u = tid + r * (NW * 32);
             if (worker && u < p.nchunks * 4)
                 vv[r] = ldg_v4(p.X + 8 * u);
         }
 #pragma unroll
         for (int r = 0; r < kMaxXWords; r++) {
-            const int u = tid + r * kThreads;
+            const int u = tid + r * (NW * 32);
             if (!worker || u >= p.nchunks * 4)   // warp-uniform: K / 8 is a multiple of 32
                 break;
             const int j = u >> 2, w = u & 3;
@@ -450,7 +453,7 @@ __global__ void __maxnreg__(kMaxRegs)
                 }
             } else {
                 // a partial: the first segment of the run in slot 0, the last in slot 1
-                const int s = checked(warp * 2 + ((nseg == 0) ? 0 : 1), kWarps * 2);
+                const int s = checked(warp * 2 + ((nseg == 0) ? 0 : 1), NW * 2);
                 if (c == 0) {
                     part[s * kRows + g] = ya;
                     part[s * kRows + g + 8] = yb;
@@ -468,26 +471,26 @@ __global__ void __maxnreg__(kMaxRegs)
     // tiles are read once into registers, so the scan and the sum are not
     // chains of dependent shared-memory reads.
     {
-        const int sl = tid >> 4, row = tid & 15;   // 16 slots x 16 rows = 256 threads
-        int tiles[kWarps * 2];
+        const int sl = tid >> 4, row = tid & 15;   // 2 NW slots x 16 rows = the working warps' threads
+        int tiles[NW * 2];
 #pragma unroll
-        for (int q = 0; q < kWarps * 2; q += 4) {
+        for (int q = 0; q < NW * 2; q += 4) {
             const int4 t4 = *reinterpret_cast<const int4 *>(part_tile + q);
             tiles[q] = t4.x; tiles[q + 1] = t4.y; tiles[q + 2] = t4.z; tiles[q + 3] = t4.w;
         }
         int tile = -1;
 #pragma unroll
-        for (int q = 0; q < kWarps * 2; q++)
+        for (int q = 0; q < NW * 2; q++)
             if (q == sl) tile = tiles[q];
         bool leader = worker && tile >= 0;
 #pragma unroll
-        for (int q = 0; q < kWarps * 2; q++)
+        for (int q = 0; q < NW * 2; q++)
             if (q < sl && tiles[q] == tile) leader = false;
         if (leader && p.swiglu) {   // rows < 8: the gates; row + 8: their ups
             if (row < 8) {
                 float gv = 0.f, uv = 0.f;
 #pragma unroll
-                for (int q = 0; q < kWarps * 2; q++)
+                for (int q = 0; q < NW * 2; q++)
                     if (q >= sl && tiles[q] == tile) {
                         gv += part[q * kRows + row];
                         uv += part[q * kRows + row + 8];
@@ -498,7 +501,7 @@ __global__ void __maxnreg__(kMaxRegs)
         } else if (leader) {
             float v = 0.f;
 #pragma unroll
-            for (int q = 0; q < kWarps * 2; q++)
+            for (int q = 0; q < NW * 2; q++)
                 if (q >= sl && tiles[q] == tile)
                     v += part[q * kRows + row];
             const int n = tile * kRows + row;
@@ -526,7 +529,7 @@ __global__ void __maxnreg__(kMaxRegs)
         if (tid == 0) {
             float v = -INFINITY;
             int i = 0x7fffffff;
-            for (int w = 0; w < kWarps; w++)
+            for (int w = 0; w < NW; w++)
                 keep_best(__uint_as_float(wbest[w].x), (int)wbest[w].y, v, i);
             p.ws_part[blockIdx.x] = make_uint2(__float_as_uint(v), (unsigned)i);
             __threadfence();
@@ -537,7 +540,7 @@ __global__ void __maxnreg__(kMaxRegs)
             __threadfence();
             float v = -INFINITY;
             int i = 0x7fffffff;
-            for (int b = tid; worker && b < (int)gridDim.x; b += kThreads) {
+            for (int b = tid; worker && b < (int)gridDim.x; b += (NW * 32)) {
                 const uint2 e = __ldcg(p.ws_part + b);
                 keep_best(__uint_as_float(e.x), (int)e.y, v, i);
             }
@@ -551,7 +554,7 @@ __global__ void __maxnreg__(kMaxRegs)
                 wbest[warp] = make_uint2(__float_as_uint(v), (unsigned)i);
             __syncthreads();
             if (tid == 0) {
-                for (int w = 1; w < kWarps; w++)
+                for (int w = 1; w < NW; w++)
                     keep_best(__uint_as_float(wbest[w].x), (int)wbest[w].y, v, i);
                 p.ids[0] = i;
                 if (p.max_out)
@@ -574,9 +577,19 @@ __global__ void __maxnreg__(kMaxRegs)
     }
 }
 
-size_t res_smem_bytes(int depth, int nchunks) {
-    return 1024 + (size_t)kWarps * depth * (kBoxBytes + kParBytes + 8) + (size_t)nchunks * (kChunk + 8) + kChunk +
-           (size_t)kWarps * 2 * (kRows * 4 + 4) + (size_t)kWarps * 8;
+size_t res_smem_bytes(int nw, int depth, int nchunks) {
+    return 1024 + (size_t)nw * depth * (kBoxBytes + kParBytes + 8) + (size_t)nchunks * (kChunk + 8) + kChunk +
+           (size_t)nw * 2 * (kRows * 4 + 4) + (size_t)nw * 8;
+}
+
+// The deepest ring (up to the most units a warp owns) for nw working warps
+// within `budget` bytes of shared memory; 0 when none fits.
+int res_depth(int nw, int Umax, int nchunks, size_t budget) {
+    const int per_warp = (Umax + nw - 1) / nw;
+    int depth = per_warp < kMaxDepth ? (per_warp < 2 ? 2 : per_warp) : kMaxDepth;
+    while (depth > 2 && res_smem_bytes(nw, depth, nchunks) > budget)
+        --depth;
+    return res_smem_bytes(nw, depth, nchunks) <= budget ? depth : 0;
 }
 
 // Launch shapes.  The CTAs of kernel i+1 are placed while kernel i runs;
@@ -588,17 +601,21 @@ size_t res_smem_bytes(int depth, int nchunks) {
 // the SM's shared memory, shape B for just over half of the registers of
 // each SM sub-partition (idle warps widen it; hence the kernel's register
 // cap).  One A and one B fit on an SM; two of either do not.  A
-// weight stream (the lm_head: two CTAs per SM by design) keeps the plain
-// shape.
+// weight stream (the lm_head) takes one shape: a CTA with the whole SM, 20
+// working warps (five per sub-partition, the most this kernel's registers
+// allow).  Its time is set by how fast each warp gets through its boxes, so
+// more warps per SM stream faster.
 struct LaunchShape {
     int threads;
     size_t smem;
 };
 
-template <bool BS64, bool ZP>
-int launch_res_t(const CUtensorMap &map, const ResParams &p, int grid, size_t smem, bool stream_mode, unsigned flags,
+template <bool BS64, bool ZP, int NW>
+int launch_res_t(const CUtensorMap &map, ResParams p, int grid, int depth, bool stream_mode, unsigned flags,
                  cudaStream_t s) {
-    auto fn = gemv_resident_kernel<BS64, ZP>;
+    auto fn = gemv_resident_kernel<BS64, ZP, NW>;
+    p.depth = depth;
+    const size_t smem = res_smem_bytes(NW, depth, p.nchunks);
     static int regs[kMaxDevices] = {}, smem_sm[kMaxDevices] = {}, reserved[kMaxDevices] = {}, rf[kMaxDevices] = {};
     static std::atomic<unsigned> parity[kMaxDevices];
     static std::mutex mu;
@@ -624,7 +641,7 @@ int launch_res_t(const CUtensorMap &map, const ResParams &p, int grid, size_t sm
             regs[dev] = (a.numRegs + 7) & ~7;
         }
     }
-    LaunchShape shape{kThreads, smem};
+    LaunchShape shape{NW * 32, smem};
     if (!stream_mode) {
         // registers are allocated per SM sub-partition (four per SM; a CTA's
         // warps go round-robin over them): cap = warps of this kernel one
@@ -694,27 +711,23 @@ int launch_gemv_resident(const void *X, const uint8_t *packed, const void *scale
     p.nchunks = K / 32;
     // one CTA per SM (the next kernel's CTAs take the other half); a weight
     // stream of more than 16 tiles per SM (the lm_head) takes both halves, as
-    // the ring of one CTA leaves the SM with too few warps to hide its latency
+    // 8 warps leave the SM with too few to hide their latency
     const int sms = device_sm_count();
-    const int grid = p.ntiles < sms ? p.ntiles : (p.ntiles > 16 * sms ? 2 * sms : sms);
+    const bool stream_mode = p.ntiles > 16 * sms;
+    const int grid = stream_mode ? kStreamCtas * sms : (p.ntiles < sms ? p.ntiles : sms);
     p.tq = p.ntiles / grid;
     p.tr = p.ntiles % grid;
-    // the deepest ring (up to the most units a warp owns) that keeps two CTAs per SM
-    const int Umax = (p.tq + (p.tr ? 1 : 0)) * p.nbx;
-    const int per_warp = (Umax + kWarps - 1) / kWarps;
-    int depth = per_warp < kMaxDepth ? (per_warp < 2 ? 2 : per_warp) : kMaxDepth;
-    while (depth > 2 && res_smem_bytes(depth, p.nchunks) > (size_t)kSmemBudget)
-        --depth;
-    if (res_smem_bytes(depth, p.nchunks) > (size_t)kSmemBudget)
+    const int Umax = (p.tq + (p.tr ? 1 : 0)) * p.nbx;   // the most units of any CTA
+    const int depth = res_depth(kWarps, Umax, p.nchunks, (size_t)kSmemBudget);
+    const int depth_s = stream_mode ? res_depth(kStreamWarps, Umax, p.nchunks, (size_t)kSmemBudget * 2 / kStreamCtas) : 0;
+    if (!depth)
         return 1;
-    p.depth = depth;
     p.argmax = ids ? 1 : 0;
     p.swiglu = swiglu;
     p.ids = ids;
     p.max_out = max_out;
     p.ws_count = static_cast<unsigned *>(workspace);
     p.ws_part = workspace ? reinterpret_cast<uint2 *>(static_cast<unsigned char *>(workspace) + 256) : nullptr;
-    const size_t smem = res_smem_bytes(depth, p.nchunks);
 
     EncodeTiledFn encode = tensor_map_encoder();
     if (!encode)
@@ -729,13 +742,20 @@ int launch_gemv_resident(const void *X, const uint8_t *packed, const void *scale
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (cr != CUDA_SUCCESS)
         return fail(MNB_ERR_CUDA, "mnb_gemv: cuTensorMapEncodeTiled failed (%d)", (int)cr);
-    const bool stream_mode = grid > sms;   // two CTAs per SM by design
-    if (bs64) {
-        if (has_zp) return launch_res_t<true, true>(map, p, grid, smem, stream_mode, flags, s);
-        return launch_res_t<true, false>(map, p, grid, smem, stream_mode, flags, s);
+    if (depth_s) {   // a weight stream: one shape, the wider CTAs
+        if (bs64) {
+            if (has_zp) return launch_res_t<true, true, kStreamWarps>(map, p, grid, depth_s, true, flags, s);
+            return launch_res_t<true, false, kStreamWarps>(map, p, grid, depth_s, true, flags, s);
+        }
+        if (has_zp) return launch_res_t<false, true, kStreamWarps>(map, p, grid, depth_s, true, flags, s);
+        return launch_res_t<false, false, kStreamWarps>(map, p, grid, depth_s, true, flags, s);
     }
-    if (has_zp) return launch_res_t<false, true>(map, p, grid, smem, stream_mode, flags, s);
-    return launch_res_t<false, false>(map, p, grid, smem, stream_mode, flags, s);
+    if (bs64) {
+        if (has_zp) return launch_res_t<true, true, kWarps>(map, p, grid, depth, stream_mode, flags, s);
+        return launch_res_t<true, false, kWarps>(map, p, grid, depth, stream_mode, flags, s);
+    }
+    if (has_zp) return launch_res_t<false, true, kWarps>(map, p, grid, depth, stream_mode, flags, s);
+    return launch_res_t<false, false, kWarps>(map, p, grid, depth, stream_mode, flags, s);
 }
 
 int read_res_status(unsigned *out, int clear) {
