@@ -202,6 +202,10 @@ MNB_API int mnb_gemv_argmax_noalloc(const void *X, const uint8_t *packed, const 
  * variant"); each weight is dequantized to fp16_rn((q - zp) * scale), the
  * value mnb_dequantize writes, and the products are accumulated in fp32.
  *   act_t and scale_t must be MNB_F16; N must be a multiple of 128 and K of 64.
+ * One CTA per (128-row tile, token tile); when those leave SMs idle, K is
+ * split over a thread-block cluster whose ranks add their partial sums in
+ * rank order through distributed shared memory, so results are the same, bit
+ * for bit, on every call.
  * A device-side wait that exceeds its iteration limit makes the kernel stop,
  * sets a bit in the library's device status word (see mnb_device_status) and
  * leaves Y incomplete; the call itself returned MNB_OK by then.

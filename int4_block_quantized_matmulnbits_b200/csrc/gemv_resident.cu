@@ -86,7 +86,6 @@ constexpr int kStreamCtas = 1;              // ... and its CTAs per SM
 constexpr int kMaxThreads = 16 * 32;
 constexpr int kMaxXWords = 4;              // 16-byte words of x per thread: K <= 8192
 constexpr int kMaxRegs = 96;                // register cap of the kernel (the launch shapes depend on it)
-constexpr int kMaxRegsWide = 80;            // ... of a CTA of more than 20 working warps
 constexpr int kRows = 16;
 constexpr int kBoxK = 256;                  // k per box: 8 blocks of 32 (4 of 64)
 constexpr int kBoxBytes = kRows * 128;
@@ -248,7 +247,7 @@ __device__ __forceinline__ float2 zp_pair(const unsigned char *par, int row, int
 }
 
 template <bool BS64, bool ZP, int NW>
-__global__ void __maxnreg__(NW > 20 ? kMaxRegsWide : kMaxRegs)
+__global__ void __maxnreg__(kMaxRegs)
     gemv_resident_kernel(const __grid_constant__ CUtensorMap wmap, const ResParams p) {
     extern __shared__ unsigned char smem_raw[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;

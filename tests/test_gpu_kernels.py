@@ -410,6 +410,12 @@ GEMM_CASES = [
     (300, 128, 6144, 32, True, np.float16),
     (420, 2048, 1024, 32, True, np.float16),
     (1024, 256, 512, 64, False, np.float16),
+    # more tilings: 48 tiles of 256 tokens, one tile per SM, more tiles than
+    # SMs, ragged token tiles with block 64
+    (1024, 1536, 1024, 32, True, np.float16),
+    (256, 18944, 256, 32, True, np.float16),
+    (256, 20480, 512, 32, True, np.float16),
+    (260, 1280, 768, 64, True, np.float16),
 ]
 
 
@@ -441,7 +447,7 @@ def test_gemm_matches_dequantized_weights_exactly_where_exact(mnb, cuda_dev):
     assert np.array_equal(np_of(Y).astype(np.float64), ref.astype(np.float16).astype(np.float64))
 
 
-@pytest.mark.parametrize("M,N,K", [(1024, 256, 512), (64, 1024, 2048), (256, 512, 2048)])
+@pytest.mark.parametrize("M,N,K", [(1024, 256, 512), (64, 1024, 2048), (256, 512, 2048), (1024, 1536, 1024)])
 def test_gemm_split_k_is_deterministic(mnb, cuda_dev, M, N, K):
     # these shapes split K over 2- and 4-CTA clusters; the owner of each column
     # chunk adds the other ranks' partial sums in rank order, so repeated calls
