@@ -442,8 +442,9 @@ def oracle_layer_gbs(cfg_name, layer=0, M=1, seconds=1.5):
             oracle.matmul(X, pk, sc, zp, K, cfg["bs"])
 
     gbs, reps = oracle_rate(run, nbytes, seconds)
-    return {"weight_gbs": round(gbs / 1e9, 4), "cores": oracle.num_threads(),
-            "sample": f"the 7 projections of layer {layer} at M={M}, {reps} passes"}
+    flops = 2 * M * sum(q[0].shape[0] * K for _, q, K in items)
+    return {"weight_gbs": round(gbs / 1e9, 4), "gflops": round(gbs / nbytes * flops / 1e9, 3),
+            "cores": oracle.num_threads(), "sample": f"the 7 projections of layer {layer} at M={M}, {reps} passes"}
 
 
 def bench_step(cfg_name, dev, ranks, hbm, Ms, steps=50):
@@ -853,6 +854,9 @@ def run_gpu(args, world, rank, local):
     torch.cuda.empty_cache()
     if with_oracle:
         step06["cpu_oracle"] = oracle_layer_gbs("qwen3_0p6b_decode")
+        # the prefill's arithmetic on the oracle: layer 0 at 16 of the 1024
+        # tokens (the oracle's cost is linear in the token count)
+        prefill["1024"]["cpu_oracle"] = oracle_layer_gbs("qwen3_1p7b_decode", M=16)
     variants = {v: bench_layout_variant(v, dev, ranks, hbm, tc_burst, with_oracle)
                 for v in ("qwen3_0p6b_bs64", "qwen3_0p6b_nozp")}
     embed = bench_embed(dev, ranks, hbm, with_oracle)
