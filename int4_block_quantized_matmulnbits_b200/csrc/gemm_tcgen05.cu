@@ -29,10 +29,11 @@
 //               After the K loop the same warps are the epilogue: tcgen05.ld of
 //               their 32 TMEM lanes, fp16 conversion, stores of Y.
 // When rows x token tiles cannot occupy the SMs, K is split over a cluster of S
-// CTAs; each keeps its partial sum in its own tensor memory, parks it in its
-// shared memory, and every rank reduces one slice of the token columns by
-// reading the others' partials through distributed shared memory (no global
-// scratch).
+// CTAs; each keeps its partial sum in its own tensor memory.  Every rank owns
+// a contiguous slice of the token columns: the others write their parts of it
+// straight from tensor memory into its shared memory (distributed shared
+// memory stores), and it adds them to its own in rank order and stores the
+// slice by TMA (no global scratch).
 // Every mbarrier wait is bounded in time: past the limit the kernel records
 // the failure in a device status word, drains what it issued, frees tensor
 // memory and exits.
@@ -149,17 +150,6 @@ __device__ __forceinline__ uint32_t map_cluster(uint32_t local, uint32_t rank) {
     return remote;
 }
 
-// Copies `bytes` from this CTA's shared memory into a cluster rank's, completing
-// on that rank's mbarrier.
-__device__ __forceinline__ void bulk_copy_to_rank(uint32_t dst_cluster, uint32_t src, uint32_t bytes,
-                                                  uint32_t bar_cluster) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            dst_cluster),
-        "r"(src), "r"(bytes), "r"(bar_cluster)
-        : "memory");
-}
-
 // Scale (fp16 bits) and zero point of one thread's 32-k half of a stage (one
 // block of 32, or half a block of 64).
 struct SZ {
@@ -247,7 +237,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto xfull = [&](int i) { return bars + 8u * (uint32_t)(2 * PS + 2 * WS + i % XS); };
     auto xempty = [&](int i) { return bars + 8u * (uint32_t)(2 * PS + 2 * WS + XS + i % XS); };
     const uint32_t acc_full = bars + 8u * (uint32_t)(2 * PS + 2 * WS + 2 * XS);
-    const uint32_t red_bar = acc_full + 8;   // K split: the other ranks' partial sums have landed
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + (acc_full + 16 - base));
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -265,7 +254,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(xempty(i), 1);
         }
         mbar_init(acc_full, 1);
-        mbar_init(red_bar, 1);
         *abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -387,21 +375,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q = warp & 3;                  // TMEM lane quarter of this warp
         const int grp = (warp - 3) >> 2;         // 0..3: this warp's share of the column chunks
         const int row = q * 32 + lane;
-        const int ny = n_tile * kBM + row;
         const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16);
         const int m0 = m_tile * BN;
         const int nchunk = BN / 16;
         const bool have = mbar_wait(acc_full, 0, abort) && nk > 0;
         tc_fence_after();
         pdl_wait();
-        auto store_y = [&](int col, const float *f) {
-#pragma unroll
-            for (int j = 0; j < 16; j++) {
-                const int m = m0 + col + j;
-                if (m < p.M)
-                    p.Y[(int64_t)m * p.N + ny] = __float2half_rn(f[j]);
-            }
-        };
         if (p.S == 1) {
             // the tile goes through shared memory (the idle fp16 weight ring) as
             // [BN tokens][128 rows] fp16 and leaves in one TMA store; two 16-column
@@ -437,77 +416,76 @@ __global__ void __launch_bounds__(kThreads, 1)
                 asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");   // written before the CTA leaves
             }
         } else {
-            // K split over the cluster.  Each rank parks its partial sums
-            // chunk-major ([16-column chunk][row][16] fp32, 8 KB per chunk); chunk c
-            // belongs to rank c % S.  Every rank then sends each chunk it does not
-            // own to its owner with one bulk copy into the owner's receive area
-            // (shared-memory loads across the cluster, 16 bytes per request, were
-            // measured ~4x slower), completing on the owner's barrier; each owner
-            // adds the copies to its own sums in rank order and stores its chunks.
-            float *park = reinterpret_cast<float *>(base_ptr);   // reuses the ring buffers
-            const int owned_max = (nchunk + p.S - 1) / p.S;
-            float *recv = park + nchunk * kBM * 16;             // [S - 1 senders][owned_max][chunk]
-            for (int c16 = grp; c16 < nchunk; c16 += 8) {
-                const bool two = c16 + 4 < nchunk;
-                uint32_t v[2][16];
+            // K split over the cluster.  Chunk c (16 token columns) belongs to
+            // rank c / per: contiguous ranges.  Once every rank's K loop is over
+            // (its rings are free), each rank writes the chunks it does not own
+            // straight from tensor memory into the owner's receive area
+            // (distributed shared memory stores; [sender slot][owned chunk]
+            // [row][16] fp32).  After a second cluster barrier each owner adds
+            // to its own sums, read again from tensor memory, the received
+            // parts in rank order, and its chunks leave through shared memory
+            // and TMA stores.
+            const int per = (nchunk + p.S - 1) / p.S;
+            float *recv = reinterpret_cast<float *>(base_ptr);   // reuses the ring buffers
+            __half *stage = reinterpret_cast<__half *>(recv + (size_t)(p.S - 1) * per * kBM * 16);   // [per][16][128]
+            cluster_sync();   // every rank is past its K loop: its shared memory may be written
+            for (int c16 = grp; c16 < nchunk; c16 += 4) {
+                const int owner = c16 / per;
+                if (owner == rank)
+                    continue;
+                uint32_t v[16];
                 if (have) {
-                    tc_ld16(taddr + (uint32_t)(c16 * 16), v[0]);
-                    if (two)
-                        tc_ld16(taddr + (uint32_t)((c16 + 4) * 16), v[1]);
+                    tc_ld16(taddr + (uint32_t)(c16 * 16), v);
+                    tc_wait_ld();
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; j++)
+                        v[j] = 0u;
+                }
+                const int slot = rank - (rank > owner ? 1 : 0);   // senders in rank order
+                const uint32_t dst = map_cluster(
+                    smem_u32(recv + (((size_t)slot * per + (c16 - owner * per)) * kBM + row) * 16), (uint32_t)owner);
+#pragma unroll
+                for (int i = 0; i < 4; i++)
+                    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16u * i),
+                                 "r"(v[4 * i]), "r"(v[4 * i + 1]), "r"(v[4 * i + 2]), "r"(v[4 * i + 3])
+                                 : "memory");
+            }
+            cluster_sync();   // every part has landed
+            const int c_lo = rank * per, c_hi = min(nchunk, c_lo + per);
+            for (int c16 = c_lo + grp; c16 < c_hi; c16 += 4) {
+                uint32_t v[16];
+                if (have) {
+                    tc_ld16(taddr + (uint32_t)(c16 * 16), v);
                     tc_wait_ld();
                 }
-#pragma unroll
-                for (int h = 0; h < 2; h++) {
-                    if (h == 1 && !two)
-                        break;
-                    float4 *dst = reinterpret_cast<float4 *>(park + ((c16 + 4 * h) * kBM + row) * 16);
-#pragma unroll
-                    for (int j = 0; j < 4; j++)
-                        dst[j] = have ? make_float4(__uint_as_float(v[h][4 * j]), __uint_as_float(v[h][4 * j + 1]),
-                                                    __uint_as_float(v[h][4 * j + 2]), __uint_as_float(v[h][4 * j + 3]))
-                                      : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-            }
-            fence_proxy_async_smem();   // the bulk copies read the parked sums
-            if (warp == 3 && lane == 0) {
-                const int owned = (nchunk - rank + p.S - 1) / p.S;
-                mbar_expect_tx(red_bar, (uint32_t)((p.S - 1) * owned) * kChunkBytes);
-            }
-            cluster_sync();   // every rank has parked and armed its barrier
-            if (warp == 3 && lane == 0) {
-                for (int c16 = 0; c16 < nchunk; c16++) {
-                    const int owner = c16 % p.S;
-                    if (owner == rank)
-                        continue;
-                    const int slot = rank - (rank > owner ? 1 : 0);   // senders in rank order
-                    const uint32_t src = smem_u32(park + c16 * kBM * 16);
-                    const uint32_t dst = smem_u32(recv + (slot * owned_max + c16 / p.S) * kBM * 16);
-                    bulk_copy_to_rank(map_cluster(dst, (uint32_t)owner), src, kChunkBytes,
-                                      map_cluster(red_bar, (uint32_t)owner));
-                }
-            }
-            const bool got = mbar_wait(red_bar, 0, abort);
-            for (int c16 = rank + p.S * grp; c16 < nchunk; c16 += 4 * p.S) {
                 float f[16];
-                const float4 *own = reinterpret_cast<const float4 *>(park + (c16 * kBM + row) * 16);
 #pragma unroll
-                for (int j = 0; j < 4; j++) {
-                    const float4 o = own[j];
-                    f[4 * j] = o.x; f[4 * j + 1] = o.y; f[4 * j + 2] = o.z; f[4 * j + 3] = o.w;
-                }
+                for (int j = 0; j < 16; j++)
+                    f[j] = have ? __uint_as_float(v[j]) : 0.f;
                 for (int sl = 0; sl < p.S - 1; sl++) {
-                    const float4 *in = reinterpret_cast<const float4 *>(recv + ((sl * owned_max + c16 / p.S) * kBM + row) * 16);
+                    const float4 *in = reinterpret_cast<const float4 *>(recv + (((size_t)sl * per + (c16 - c_lo)) * kBM + row) * 16);
 #pragma unroll
                     for (int j = 0; j < 4; j++) {
                         const float4 o = in[j];
                         f[4 * j] += o.x; f[4 * j + 1] += o.y; f[4 * j + 2] += o.z; f[4 * j + 3] += o.w;
                     }
                 }
-                if (!got)
-                    continue;
-                store_y(c16 * 16, f);
+#pragma unroll
+                for (int j = 0; j < 16; j++)
+                    stage[((c16 - c_lo) * 16 + j) * kBM + row] = __float2half_rn(f[j]);
             }
-            cluster_sync();   // every copy into a rank has landed (it waited) before any rank exits
+            fence_proxy_async_smem();   // the TMA stores read what the generic stores wrote
+            asm volatile("bar.sync 1, %0;" ::"n"(kDqWarps * 32) : "memory");
+            if (warp == 3 && lane == 0 && have) {
+                for (int c16 = c_lo; c16 < c_hi && m0 + c16 * 16 < p.M; c16++)   // no box wholly past M
+                    asm volatile(
+                        "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(&ymap),
+                        "r"(n_tile * kBM), "r"(m0 + c16 * 16), "r"(smem_u32(stage + (size_t)(c16 - c_lo) * 16 * kBM))
+                        : "memory");
+                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");   // written before the CTA leaves
+            }
         }
     }
     if (p.S > 1 && warp < 3) {
@@ -583,10 +561,11 @@ int launch_gemm(const void *X, const uint8_t *packed, const void *scales, int sc
     if (xstages > 8) xstages = 8;
     if (xstages < 2) xstages = 2;
     const size_t ring_bytes = (size_t)fixed + (size_t)xstages * BN * 128;
-    // the cluster reduction reuses the rings: the parked sums [BN / 16][128][16]
-    // fp32 and the copies received from the other S - 1 ranks
-    const size_t chunks = (size_t)BN / 16, owned_max = (chunks + S - 1) / S;
-    if (S > 1 && ring_bytes < (chunks + (size_t)(S - 1) * owned_max) * kChunkBytes)
+    // the cluster reduction reuses the rings: the parts received from the
+    // other S - 1 ranks ([per owned chunk][128][16] fp32 each) and the owned
+    // chunks' fp16 tile
+    const size_t chunks = (size_t)BN / 16, per = (chunks + S - 1) / S;
+    if (S > 1 && ring_bytes < (size_t)(S - 1) * per * kChunkBytes + per * 16 * kBM * 2)
         return fail(MNB_ERR_SHAPE, "mnb_gemm: reduction buffer does not fit");
     p.xstages = xstages;
     const size_t smem = 1024 + ring_bytes + 8 * (2 * kPS + 2 * kWS + 2 * xstages + 2) + 16;
@@ -617,11 +596,13 @@ int launch_gemm(const void *X, const uint8_t *packed, const void *scales, int sc
             return fail(MNB_ERR_CUDA, "mnb_gemm: cuTensorMapEncodeTiled (W) failed (%d)", (int)cr);
     }
 
-    CUtensorMap ymap;   // Y [M][N] fp16, box [BN tokens][128 rows]: the epilogue's TMA store
+    // Y [M][N] fp16: the epilogue's TMA stores, box [BN tokens][128 rows]
+    // (whole tiles) or [16 tokens][128 rows] (chunks of a split tile)
+    CUtensorMap ymap;
     {
         const cuuint64_t gdim[2] = {(cuuint64_t)N, (cuuint64_t)M};
         const cuuint64_t gstride[1] = {(cuuint64_t)N * 2};
-        const cuuint32_t box[2] = {(cuuint32_t)kBM, (cuuint32_t)BN};
+        const cuuint32_t box[2] = {(cuuint32_t)kBM, (cuuint32_t)(S > 1 ? 16 : BN)};
         const cuuint32_t estride[2] = {1, 1};
         CUresult cr = encode(&ymap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, Y, gdim, gstride, box, estride,
                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
