@@ -16,14 +16,17 @@
 //     packed bytes (TMA, 128-byte swizzle) plus its scales and zero points
 //     (cp.async), completing on one mbarrier.  For the decoder's projections
 //     every unit fits in the rings, so after griddepcontrol.wait only x is
-//     read from memory; the lm_head streams through the same rings.
+//     read from memory.  The lm_head streams through the same rings, with
+//     one 20-warp CTA per SM.
 //   * Work split: CTA b owns a contiguous run of 16-row tiles; its (tile, box)
 //     units are cut into one contiguous run per warp.  Tiles a warp covers
 //     whole are stored from registers; the partial sums of tiles cut between
 //     warps meet in shared memory and are added in warp order.  Both launch
 //     shapes (below) have the same 8 working warps, so every call cuts and
 //     adds the sums alike: the result is the same, bit for bit, from call to
-//     call.  Nothing crosses CTAs: no cluster, no atomics, no global scratch.
+//     call.  Nothing crosses CTAs (no cluster, no global scratch), except the
+//     greedy-decoding epilogue's last step: per-CTA maxima in a caller
+//     workspace, reduced by the last CTA to finish (an atomic count).
 //   * Zero point and scale are applied per block AFTER the tensor core, not
 //     per weight.  The MMA (mma.sync m16n8k16, fp32 accumulation) takes the
 //     raw codes: (nibble | 0x6400) is the fp16 1024+q exactly for a low
