@@ -203,12 +203,26 @@ __device__ __forceinline__ void cursor_next(const ResParams &p, IssueCursor &q, 
 // the box's scales (lanes 0-15) and zero points (lanes 16-31) by cp.async.
 // Rows past N get no parameters (their sums are never stored).  Every lane
 // arrives on the slot's barrier once its copies have landed.
+// A weight box by TMA, marked first to leave L2: each box is read once per
+// call, while a row's scales and zero points come in 32-byte sectors that
+// the row's next box reads again (the lm_head: 1.044x the algorithmic DRAM
+// bytes without the hint).
+__device__ __forceinline__ void tma_load_2d_evict_first(uint32_t dst, const void *map, uint32_t bar, int x, int y) {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+        "l"(map), "r"(bar), "r"(x), "r"(y), "l"(pol)
+        : "memory");
+}
+
 template <bool BS64, bool ZP>
 __device__ __forceinline__ void issue(const CUtensorMap *wmap, const ResParams &p, const IssueCursor &q,
                                       uint32_t box_dst, uint32_t par_dst, uint32_t full, int lane) {
     if (lane == 0) {
         mbar_expect_tx(full, kBoxBytes);
-        tma_load_2d(box_dst, wmap, full, checked(q.box, p.nbx) * 128, checked(q.tile, p.ntiles) * kRows);
+        tma_load_2d_evict_first(box_dst, wmap, full, checked(q.box, p.nbx) * 128, checked(q.tile, p.ntiles) * kRows);
     }
     if (q.row_ok) {
         if (lane < 16) {
